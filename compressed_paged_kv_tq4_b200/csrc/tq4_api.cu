@@ -1,0 +1,303 @@
+// C ABI of the TQ4 paged-KV attention library: context, argument checks,
+// planning and launches. Every kernel of the library is compiled in this one
+// translation unit (the kernel headers are included below).
+#include <cmath>
+#include <cstring>
+#include <new>
+
+#include <cuda_runtime.h>
+
+#include "../../include/tq4.h"
+#include "tq4_device.cuh"
+#include "tq4_encode.cuh"
+#include "tq4_decode.cuh"
+#include "tq4_prefill.cuh"
+
+struct tq4_ctx {
+  int device;
+  int num_sms;
+  tq4::Signs signs;
+  double centroids[16];
+  double boundaries[15];
+  int* d_status;
+};
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// 16-level Lloyd-Max quantiser for N(0, sigma^2) in fp64: alternate the two
+// optimality conditions (boundaries at centroid midpoints; centroids at the
+// Gaussian conditional mean of their cell) until nothing moves. The Gaussian
+// density is log-concave, so the fixed point is unique and the starting
+// spread does not matter.
+// ---------------------------------------------------------------------------
+double std_normal_pdf(double z) { return std::isinf(z) ? 0.0 : std::exp(-0.5 * z * z) / std::sqrt(2.0 * M_PI); }
+
+void lloyd_max_16(double sigma, double c[16], double b[15]) {
+  for (int j = 0; j < 16; ++j) c[j] = sigma * (-2.5 + 5.0 * j / 15.0);
+  for (int it = 0; it < 200000; ++it) {
+    for (int j = 0; j < 15; ++j) b[j] = 0.5 * (c[j] + c[j + 1]);
+    double moved = 0.0;
+    double cn[16];
+    for (int j = 0; j < 16; ++j) {
+      const double lo = j == 0 ? -INFINITY : b[j - 1] / sigma;
+      const double hi = j == 15 ? INFINITY : b[j] / sigma;
+      // P(lo < Z < hi) = (erfc(lo/sqrt2) - erfc(hi/sqrt2)) / 2
+      const double mass = 0.5 * (std::erfc(lo / M_SQRT2) - std::erfc(hi / M_SQRT2));
+      cn[j] = sigma * (std_normal_pdf(lo) - std_normal_pdf(hi)) / mass;
+      moved = std::fmax(moved, std::fabs(cn[j] - c[j]));
+    }
+    std::memcpy(c, cn, sizeof(cn));
+    if (moved < 1e-19) break;
+  }
+  for (int j = 0; j < 15; ++j) b[j] = 0.5 * (c[j] + c[j + 1]);
+}
+
+uint16_t half_bits(double x) {
+  const __half h = __double2half(x);
+  uint16_t u;
+  std::memcpy(&u, &h, 2);
+  return u;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? TQ4_OK : TQ4_ERR_CUDA; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_device(const tq4_ctx* ctx) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TQ4_ERR_CUDA;
+  return dev == ctx->device ? TQ4_OK : TQ4_ERR_ARG;
+}
+
+template <int NT>
+cudaError_t set_decode_attrs() {
+  return cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              int(tq4::decode_smem_bytes<NT>()));
+}
+
+struct DecodePlan {
+  int split_len;
+  int items_ub;
+  int rows_pad;
+  size_t ws_o_bytes;
+  size_t ws_ml_bytes;
+  size_t total;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+DecodePlan plan_decode(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len) {
+  DecodePlan pl{};
+  const int64_t ctas = int64_t(ctx->num_sms) * 2;            // two resident CTAs per SM
+  int64_t L = (total_seq_len * tq4::kHkv + ctas - 1) / ctas;  // positions per split
+  L = ((L + tq4::kChunk - 1) / tq4::kChunk) * tq4::kChunk;
+  if (L < tq4::kChunk) L = tq4::kChunk;
+  if (L > (1 << 30)) L = 1 << 30;
+  pl.split_len = int(L);
+  pl.items_ub = int(total_seq_len / L) + n_req;
+  pl.rows_pad = 8 * tq4::decode_nt(n_q);
+  const size_t recs = size_t(pl.items_ub) * tq4::kHkv * pl.rows_pad;
+  pl.ws_o_bytes = align256(recs * tq4::kD * sizeof(float));
+  pl.ws_ml_bytes = align256(recs * sizeof(float2));
+  pl.total = pl.ws_o_bytes + pl.ws_ml_bytes;
+  return pl;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
+  if (!signs || !out) return TQ4_ERR_ARG;
+  *out = nullptr;
+  tq4::Signs sb{};
+  for (int i = 0; i < 256; ++i) {
+    if (signs[i] != 1 && signs[i] != -1) return TQ4_ERR_ARG;
+    if (signs[i] < 0) sb.bits[i >> 5] |= 1u << (i & 31);
+  }
+  tq4_ctx* ctx = new (std::nothrow) tq4_ctx();
+  if (!ctx) return TQ4_ERR_ARG;
+  ctx->signs = sb;
+  lloyd_max_16(1.0 / 16.0, ctx->centroids, ctx->boundaries);
+  tq4::Codebook cb{};
+  for (int j = 0; j < 16; ++j) {
+    cb.c[j] = float(ctx->centroids[j]);
+    cb.c16[j] = half_bits(ctx->centroids[j]);
+  }
+  for (int j = 0; j < 15; ++j) cb.b[j] = float(ctx->boundaries[j]);
+  cudaError_t e = cudaGetDevice(&ctx->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(tq4::g_codebook, &cb, sizeof(cb));
+  if (e == cudaSuccess) e = set_decode_attrs<1>();
+  if (e == cudaSuccess) e = set_decode_attrs<2>();
+  if (e == cudaSuccess) e = set_decode_attrs<3>();
+  if (e == cudaSuccess) e = tq4::prefill_set_attrs();
+  if (e == cudaSuccess) e = cudaMalloc(&ctx->d_status, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(ctx->d_status, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    if (ctx->d_status) cudaFree(ctx->d_status);
+    delete ctx;
+    return TQ4_ERR_CUDA;
+  }
+  *out = ctx;
+  return TQ4_OK;
+}
+
+int tq4_ctx_destroy(tq4_ctx* ctx) {
+  if (!ctx) return TQ4_OK;
+  cudaDeviceSynchronize();
+  const cudaError_t e = cudaFree(ctx->d_status);
+  delete ctx;
+  return cuda_status(e);
+}
+
+int tq4_codebook(const tq4_ctx* ctx, double* centroids, double* boundaries) {
+  if (!ctx || !centroids || !boundaries) return TQ4_ERR_ARG;
+  std::memcpy(centroids, ctx->centroids, sizeof(ctx->centroids));
+  std::memcpy(boundaries, ctx->boundaries, sizeof(ctx->boundaries));
+  return TQ4_OK;
+}
+
+int tq4_encode_append(tq4_ctx* ctx, void* pool, int32_t num_pages, const int32_t* page_table,
+                      int32_t table_len, int32_t start_pos, int32_t n_tok, const void* k_new,
+                      const void* v_new, int dtype, void* stream) {
+  if (!ctx || n_tok < 0 || start_pos < 0) return TQ4_ERR_ARG;
+  if (n_tok == 0) return TQ4_OK;
+  if (!pool || !page_table || !k_new || !v_new || num_pages <= 0 || table_len <= 0) return TQ4_ERR_ARG;
+  if (dtype != TQ4_DTYPE_F32 && dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
+  if ((int64_t(start_pos) + n_tok + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
+  if (!aligned(pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16)) return TQ4_ERR_ARG;
+  if (int rc = check_device(ctx)) return rc;
+  return cuda_status(tq4::launch_encode_append(static_cast<uint8_t*>(pool), num_pages, page_table,
+                                               start_pos, n_tok, k_new, v_new, dtype, ctx->signs,
+                                               ctx->d_status, static_cast<cudaStream_t>(stream)));
+}
+
+int tq4_reconstruct(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int32_t* page_table,
+                    int32_t table_len, int32_t start, int32_t n, float* k_out, float* v_out,
+                    void* stream) {
+  if (!ctx || n < 0 || start < 0) return TQ4_ERR_ARG;
+  if (n == 0) return TQ4_OK;
+  if (!pool || !page_table || !k_out || !v_out || num_pages <= 0 || table_len <= 0) return TQ4_ERR_ARG;
+  if ((int64_t(start) + n + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
+  if (!aligned(pool, 16) || !aligned(k_out, 16) || !aligned(v_out, 16)) return TQ4_ERR_ARG;
+  if (int rc = check_device(ctx)) return rc;
+  return cuda_status(tq4::launch_reconstruct(static_cast<const uint8_t*>(pool), num_pages, page_table,
+                                             start, n, k_out, v_out, ctx->signs, ctx->d_status,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
+size_t tq4_decode_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len) {
+  if (!ctx || n_req <= 0 || n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS || total_seq_len <= 0) return 0;
+  return plan_decode(ctx, n_req, n_q, total_seq_len).total;
+}
+
+int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q,
+                         const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens,
+                         int32_t n_req, int32_t n_q, int64_t total_seq_len, float scale, void* out,
+                         int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx || n_req < 0) return TQ4_ERR_ARG;
+  if (n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS) return TQ4_ERR_UNSUPPORTED;
+  if (n_req == 0) return TQ4_OK;
+  if (!pool || !q || !page_tables || !seq_lens || !out || num_pages <= 0 || max_pages <= 0)
+    return TQ4_ERR_ARG;
+  if (out_dtype != TQ4_DTYPE_F32 && out_dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
+  if (!std::isfinite(scale)) return TQ4_ERR_ARG;
+  if (total_seq_len < int64_t(n_req) * n_q || total_seq_len > int64_t(n_req) * max_pages * tq4::kPage)
+    return TQ4_ERR_ARG;
+  if (!aligned(pool, 16) || !aligned(q, 16) || !aligned(out, 16)) return TQ4_ERR_ARG;
+  const DecodePlan pl = plan_decode(ctx, n_req, n_q, total_seq_len);
+  if (!workspace || workspace_bytes < pl.total || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
+  if (int rc = check_device(ctx)) return rc;
+
+  tq4::DecodeParams p{};
+  p.pool = static_cast<const uint8_t*>(pool);
+  p.num_pages = num_pages;
+  p.q = q;
+  p.page_tables = page_tables;
+  p.max_pages = max_pages;
+  p.seq_lens = seq_lens;
+  p.n_req = n_req;
+  p.n_q = n_q;
+  p.scale = scale;
+  p.split_len = pl.split_len;
+  p.items_ub = pl.items_ub;
+  p.rows_pad = pl.rows_pad;
+  p.ws_o = static_cast<float*>(workspace);
+  p.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + pl.ws_o_bytes);
+  p.out = out;
+  p.out_dtype = out_dtype;
+  p.signs = ctx->signs;
+  p.status = ctx->d_status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
+  switch (tq4::decode_nt(n_q)) {
+    case 1:
+      tq4::decode_splitk_kernel<1><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<1>(), st>>>(p);
+      break;
+    case 2:
+      tq4::decode_splitk_kernel<2><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<2>(), st>>>(p);
+      break;
+    default:
+      tq4::decode_splitk_kernel<3><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<3>(), st>>>(p);
+      break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return TQ4_ERR_CUDA;
+  const int rows = n_req * n_q * tq4::kHq;
+  tq4::decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p);
+  return cuda_status(cudaGetLastError());
+}
+
+size_t tq4_prefill_workspace_bytes(int32_t n_tok) {
+  if (n_tok <= 0) return 0;
+  return tq4::prefill_workspace_bytes(n_tok);
+}
+
+int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int32_t* page_table,
+                          int32_t table_len, int32_t prefix_len, const uint16_t* q,
+                          const uint16_t* k_chunk, const uint16_t* v_chunk, int32_t n_tok, float scale,
+                          uint16_t* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx || n_tok < 0 || prefix_len < 0) return TQ4_ERR_ARG;
+  if (n_tok == 0) return TQ4_OK;
+  if (!q || !k_chunk || !v_chunk || !out) return TQ4_ERR_ARG;
+  if (prefix_len > 0 && (!pool || !page_table || num_pages <= 0 || table_len <= 0)) return TQ4_ERR_ARG;
+  if (prefix_len > 0 && (int64_t(prefix_len) + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
+  if (!std::isfinite(scale)) return TQ4_ERR_ARG;
+  if ((pool && !aligned(pool, 16)) || !aligned(q, 16) || !aligned(k_chunk, 16) || !aligned(v_chunk, 16) ||
+      !aligned(out, 16))
+    return TQ4_ERR_ARG;
+  const size_t need = tq4::prefill_workspace_bytes(n_tok);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
+  if (int rc = check_device(ctx)) return rc;
+  return cuda_status(tq4::launch_prefill(static_cast<const uint8_t*>(pool), num_pages, page_table,
+                                         prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, workspace,
+                                         ctx->signs, ctx->d_status, ctx->num_sms,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int tq4_get_status(tq4_ctx* ctx, void* stream) {
+  if (!ctx) return TQ4_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TQ4_ERR_CUDA;
+  if (cudaMemcpy(&h, ctx->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TQ4_ERR_CUDA;
+  if (cudaMemset(ctx->d_status, 0, sizeof(int)) != cudaSuccess) return TQ4_ERR_CUDA;
+  return h;
+}
+
+const char* tq4_status_string(int status) {
+  switch (status) {
+    case TQ4_OK: return "ok";
+    case TQ4_ERR_ARG: return "invalid argument";
+    case TQ4_ERR_UNSUPPORTED: return "unsupported shape";
+    case TQ4_ERR_PAGE_RANGE: return "page id out of range";
+    case TQ4_ERR_CUDA: return "CUDA runtime error";
+    case TQ4_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case TQ4_ERR_SEQ: return "sequence length inconsistent with page table or plan";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

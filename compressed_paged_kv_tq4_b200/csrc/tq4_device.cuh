@@ -1,0 +1,166 @@
+// Device-side building blocks shared by the TQ4 kernels (sm_100a).
+//
+// Format ([KVEXEC]: simpleprog.com "Fitting a 27B-Parameter LLM into 24 GiB of
+// Laptop Memory", section "KVExec: Fused Reconstruction with Layer-Scoped
+// Lifetime"): a 256-dim head vector is 32 u32 words of eight 4-bit centroid
+// indices plus one fp16 norm; pages hold 256 positions of one layer.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "../../include/tq4.h"
+
+namespace tq4 {
+
+constexpr int kD = 256;          // head dim
+constexpr int kPage = 256;       // positions per page
+constexpr int kHkv = 4;          // KV heads
+constexpr int kHq = 24;          // query heads
+constexpr int kGroup = 6;        // query heads per KV head
+constexpr int kWords = 32;       // u32 words per vector
+
+// byte offsets inside one page (one layer)
+constexpr int64_t kPageBytes = TQ4_PAGE_BYTES;
+constexpr int64_t kKWords = 0;
+constexpr int64_t kVWords = int64_t(kHkv) * kPage * kWords * 4;   // 131072
+constexpr int64_t kKNorms = 2 * kVWords;                           // 262144
+constexpr int64_t kVNorms = kKNorms + int64_t(kHkv) * kPage * 2;   // 264192
+
+// codebook in constant memory, written once per process by the host from its
+// fp64 Lloyd-Max solution (same for every context; the signs are per context)
+struct Codebook {
+  float c[16];        // centroids (fp32 of the fp64 values)
+  float b[15];        // decision boundaries (fp32 of the fp64 midpoints)
+  uint16_t c16[16];   // centroids as fp16 bits (round to nearest even from fp64)
+};
+__constant__ Codebook g_codebook;  // one translation unit (tq4_api.cu) includes every kernel header
+
+// 256 sign bits: bit i set <=> s_i = -1. Passed by value to kernels.
+struct Signs {
+  uint32_t bits[8];
+};
+
+__device__ __forceinline__ void record_error(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// --------------------------------------------------------------------------
+// Unnormalised Walsh-Hadamard transform of a 256-vector held by one warp,
+// lane l owning coordinates 8l..8l+7 in v[0..7] (Sylvester / natural order).
+// Butterflies over index bits 0..2 are in registers, bits 3..7 cross lanes.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void warp_fwht256(float v[8]) {
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & h) == 0) {
+        float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float o = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (o - v[i]) : (v[i] + o);
+    }
+  }
+}
+
+// sign of coordinate 8*lane + i as a float multiplier
+__device__ __forceinline__ float sign_of(const Signs& s, int coord) {
+  return ((s.bits[coord >> 5] >> (coord & 31)) & 1u) ? -1.0f : 1.0f;
+}
+
+// --------------------------------------------------------------------------
+// Nibble-pair decode through a per-lane table in shared memory.
+// Row b (one byte = two 4-bit indices) is 256 bytes; lane l reads its own
+// 4-byte slot at b*256 + 4*l, so the 32 lanes of a warp always hit 32
+// different banks. The slot holds f16x2 {c[b & 15], c[b >> 4]}.
+// --------------------------------------------------------------------------
+constexpr int kLutBytes = 256 * 256;
+
+__device__ __forceinline__ void lut_fill(uint32_t* lut, int tid, int nthreads) {
+  for (int e = tid; e < 256 * 32; e += nthreads) {
+    const int b = e >> 5, l = e & 31;
+    const uint32_t lo = g_codebook.c16[b & 15], hi = g_codebook.c16[b >> 4];
+    lut[b * 64 + l] = lo | (hi << 16);
+  }
+}
+
+// byte k (0..3) of w -> f16x2 of its two nibbles (low nibble in the low half)
+template <int K>
+__device__ __forceinline__ uint32_t lut_decode(const char* lut, uint32_t w, uint32_t lane4) {
+  // result byte0 = lane*4 (from lane4), byte1 = byte K of w, bytes 2..3 = 0
+  constexpr uint32_t sel = (5u << 12) | (5u << 8) | (uint32_t(K) << 4) | 4u;
+  const uint32_t off = __byte_perm(w, lane4, sel);
+  return *reinterpret_cast<const uint32_t*>(lut + off);
+}
+
+// Interleave the nibbles of two words: lo byte k = x_{2k} | y_{2k} << 4,
+// hi byte k = x_{2k+1} | y_{2k+1} << 4 (x, y = words of two positions).
+__device__ __forceinline__ void interleave_nibbles(uint32_t x, uint32_t y, uint32_t& lo, uint32_t& hi) {
+  lo = (x & 0x0F0F0F0Fu) | ((y << 4) & 0xF0F0F0F0u);
+  hi = ((x >> 4) & 0x0F0F0F0Fu) | (y & 0xF0F0F0F0u);
+}
+
+// --------------------------------------------------------------------------
+// Warp-level tensor-core primitives (register operands).
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void mma_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3,
+                                            uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x2(uint32_t& r0, uint32_t& r1, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void stmatrix_x2_trans(uint32_t addr, uint32_t r0, uint32_t r1) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1,%2};\n" ::"r"(addr), "r"(r0),
+               "r"(r1)
+               : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// read-only global loads
+__device__ __forceinline__ uint4 ldg128(const void* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+__device__ __forceinline__ uint32_t ldg32(const void* p) {
+  return __ldg(reinterpret_cast<const unsigned int*>(p));
+}
+__device__ __forceinline__ float ldg_half(const void* p) {
+  return __half2float(__ldg(reinterpret_cast<const __half*>(p)));
+}
+
+}  // namespace tq4

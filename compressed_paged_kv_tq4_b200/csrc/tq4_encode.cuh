@@ -1,0 +1,165 @@
+// TQ4 encode + append, and explicit reconstruction (sm_100a).
+//
+// Encode ([KVEXEC] simpleprog.com "Fitting a 27B-Parameter LLM into 24 GiB of
+// Laptop Memory", section "KVExec": four-bit TurboQuant encoding, 32 U32 words
+// with eight indices each + one FP16 norm): per head vector x,
+//   n = ||x||_2, u = x / n, y = R u with R = H diag(s) / 16,
+//   idx_i = number of decision boundaries below y_i (nearest centroid, ties low),
+//   word w = sum_i idx_{8w+i} << 4i, norm stored as fp16(n).
+// Reconstruction (same section: centroid lookup, inverse Hadamard rotation,
+// norm restore): x_hat = fp16(n) * diag(s) H c[idx] / 16.
+//
+// One warp per vector; lane l owns coordinates 8l..8l+7, i.e. exactly word l.
+#pragma once
+#include "tq4_device.cuh"
+
+namespace tq4 {
+
+template <typename T>
+__device__ __forceinline__ void load8(const T* src, float v[8]);
+
+template <>
+__device__ __forceinline__ void load8<float>(const float* src, float v[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+template <>
+__device__ __forceinline__ void load8<uint16_t>(const uint16_t* src, float v[8]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// grid: ceil(n_tok * 8 / warps_per_block); warp -> (token, kv, head)
+template <typename T>
+__global__ void __launch_bounds__(256) encode_append_kernel(
+    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table,
+    int32_t start_pos, int32_t n_tok, const T* __restrict__ k_new, const T* __restrict__ v_new,
+    Signs signs, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (vec >= int64_t(n_tok) * 2 * kHkv) return;
+  const int tok = int(vec / (2 * kHkv));
+  const int kv = int(vec / kHkv) & 1;       // 0 = K, 1 = V
+  const int head = int(vec % kHkv);
+  const T* src = (kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8;
+
+  float x[8];
+  load8<T>(src, x);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  const float n = sqrtf(ss);
+
+  uint32_t word = 0;
+  if (n > 0.f) {
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = (x[i] / n) * sign_of(signs, lane * 8 + i);
+    warp_fwht256(y);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float yi = y[i] * 0.0625f;  // 1/16, exact
+      uint32_t idx = 0;
+#pragma unroll
+      for (int j = 0; j < 15; ++j) idx += (yi > g_codebook.b[j]) ? 1u : 0u;
+      word |= idx << (4 * i);
+    }
+  }
+
+  const int32_t p = start_pos + tok;
+  const int32_t page = __ldg(page_table + (p >> 8));
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+    return;
+  }
+  const int slot = p & (kPage - 1);
+  uint8_t* base = pool + int64_t(page) * kPageBytes;
+  uint32_t* words = reinterpret_cast<uint32_t*>(base + (kv ? kVWords : kKWords)) +
+                    (head * kPage + slot) * kWords;
+  words[lane] = word;
+  if (lane == 0) {
+    __half* norms = reinterpret_cast<__half*>(base + (kv ? kVNorms : kKNorms));
+    norms[head * kPage + slot] = __float2half_rn(n);
+  }
+}
+
+// grid: ceil(n * 8 / warps_per_block); writes fp32 [n][4][256] for K and V
+__global__ void __launch_bounds__(256) reconstruct_kernel(
+    const uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table,
+    int32_t start, int32_t n, float* __restrict__ k_out, float* __restrict__ v_out, Signs signs,
+    int* status) {
+  __shared__ float cb[16];
+  if (threadIdx.x < 16) cb[threadIdx.x] = g_codebook.c[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (vec >= int64_t(n) * 2 * kHkv) return;
+  const int tok = int(vec / (2 * kHkv));
+  const int kv = int(vec / kHkv) & 1;
+  const int head = int(vec % kHkv);
+  float* dst = (kv ? v_out : k_out) + (int64_t(tok) * kHkv + head) * kD + lane * 8;
+
+  const int32_t p = start + tok;
+  const int32_t page = __ldg(page_table + (p >> 8));
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = 0.f;
+    return;
+  }
+  const int slot = p & (kPage - 1);
+  const uint8_t* base = pool + int64_t(page) * kPageBytes;
+  const uint32_t word = ldg32(base + (kv ? kVWords : kKWords) + ((head * kPage + slot) * kWords + lane) * 4);
+  const float nrm = ldg_half(base + (kv ? kVNorms : kKNorms) + (head * kPage + slot) * 2);
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = cb[(word >> (4 * i)) & 15u];
+  warp_fwht256(v);
+  float o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = nrm * (v[i] * 0.0625f * sign_of(signs, lane * 8 + i));
+  reinterpret_cast<float4*>(dst)[0] = make_float4(o[0], o[1], o[2], o[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(o[4], o[5], o[6], o[7]);
+}
+
+// ---------------------------------------------------------------- launchers
+cudaError_t launch_encode_append(uint8_t* pool, int32_t num_pages, const int32_t* page_table,
+                                 int32_t start_pos, int32_t n_tok, const void* k_new,
+                                 const void* v_new, int dtype, const Signs& signs, int* status,
+                                 cudaStream_t stream) {
+  const int threads = 256, wpb = threads / 32;
+  const int64_t vecs = int64_t(n_tok) * 2 * kHkv;
+  const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
+  if (dtype == TQ4_DTYPE_F32)
+    encode_append_kernel<float><<<blocks, threads, 0, stream>>>(
+        pool, num_pages, page_table, start_pos, n_tok, static_cast<const float*>(k_new),
+        static_cast<const float*>(v_new), signs, status);
+  else
+    encode_append_kernel<uint16_t><<<blocks, threads, 0, stream>>>(
+        pool, num_pages, page_table, start_pos, n_tok, static_cast<const uint16_t*>(k_new),
+        static_cast<const uint16_t*>(v_new), signs, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reconstruct(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,
+                               int32_t start, int32_t n, float* k_out, float* v_out,
+                               const Signs& signs, int* status, cudaStream_t stream) {
+  const int threads = 256, wpb = threads / 32;
+  const int64_t vecs = int64_t(n) * 2 * kHkv;
+  const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
+  reconstruct_kernel<<<blocks, threads, 0, stream>>>(pool, num_pages, page_table, start, n, k_out,
+                                                      v_out, signs, status);
+  return cudaGetLastError();
+}
+
+}  // namespace tq4

@@ -1,0 +1,259 @@
+"""Thin Python binding of libtq4.so (ctypes). Argument marshalling only.
+
+Every function here forwards to the C ABI declared in include/tq4.h under the
+same name; torch is used only to own device memory and to name the stream.
+There is no fallback: if the shared library is missing, importing this module
+raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq4.so")
+
+TQ4_OK = 0
+TQ4_ERR_ARG = -1
+TQ4_ERR_UNSUPPORTED = -2
+TQ4_ERR_PAGE_RANGE = -3
+TQ4_ERR_CUDA = -4
+TQ4_ERR_WORKSPACE = -5
+TQ4_ERR_SEQ = -6
+
+HEAD_DIM = 256
+PAGE_POSITIONS = 256
+KV_HEADS = 4
+Q_HEADS = 24
+PAGE_BYTES = 266240
+POSITION_BYTES = 1040
+
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
+EXPORTS = (
+    "tq4_ctx_create", "tq4_ctx_destroy", "tq4_codebook", "tq4_encode_append", "tq4_reconstruct",
+    "tq4_decode_workspace_bytes", "tq4_decode_attention", "tq4_prefill_workspace_bytes",
+    "tq4_prefill_attention", "tq4_get_status", "tq4_status_string",
+)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m compressed_paged_kv_tq4_b200.build`")
+    return ctypes.CDLL(LIB_PATH)
+
+
+_lib = _load()
+
+_p = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+_sz = ctypes.c_size_t
+_f = ctypes.c_float
+
+_sig = {
+    "tq4_ctx_create": ([_p, ctypes.POINTER(_p)], ctypes.c_int),
+    "tq4_ctx_destroy": ([_p], ctypes.c_int),
+    "tq4_codebook": ([_p, _p, _p], ctypes.c_int),
+    "tq4_encode_append": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p], ctypes.c_int),
+    "tq4_reconstruct": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, _p], ctypes.c_int),
+    "tq4_decode_workspace_bytes": ([_p, _i32, _i32, _i64], _sz),
+    "tq4_decode_attention": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int,
+                              _p, _sz, _p], ctypes.c_int),
+    "tq4_prefill_workspace_bytes": ([_i32], _sz),
+    "tq4_prefill_attention": ([_p, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p, _p, _sz, _p],
+                              ctypes.c_int),
+    "tq4_get_status": ([_p, _p], ctypes.c_int),
+    "tq4_status_string": ([ctypes.c_int], ctypes.c_char_p),
+}
+for _name, (_args, _res) in _sig.items():
+    _fn = getattr(_lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+class TQ4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {tq4_status_string(code)} ({code})")
+        self.code = code
+
+
+def _check(code: int, what: str) -> int:
+    if code != TQ4_OK:
+        raise TQ4Error(code, what)
+    return code
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ---------------------------------------------------------------- raw ABI, same names
+def tq4_status_string(code: int) -> str:
+    return _lib.tq4_status_string(code).decode()
+
+
+def tq4_ctx_create(signs) -> int:
+    """signs: 256 values of +-1 (any int sequence / numpy array). Returns the context handle."""
+    buf = (ctypes.c_int8 * 256)(*[int(s) for s in signs])
+    out = _p()
+    _check(_lib.tq4_ctx_create(ctypes.cast(buf, _p), ctypes.byref(out)), "tq4_ctx_create")
+    return out.value
+
+
+def tq4_ctx_destroy(ctx: int) -> None:
+    _check(_lib.tq4_ctx_destroy(ctx), "tq4_ctx_destroy")
+
+
+def tq4_codebook(ctx: int):
+    c = (ctypes.c_double * 16)()
+    b = (ctypes.c_double * 15)()
+    _check(_lib.tq4_codebook(ctx, ctypes.cast(c, _p), ctypes.cast(b, _p)), "tq4_codebook")
+    return list(c), list(b)
+
+
+def tq4_encode_append(ctx, pool, num_pages, page_table, table_len, start_pos, n_tok, k_new, v_new,
+                      dtype, stream=None) -> int:
+    return _lib.tq4_encode_append(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, start_pos,
+                                  n_tok, _ptr(k_new), _ptr(v_new), dtype, _stream(stream))
+
+
+def tq4_reconstruct(ctx, pool, num_pages, page_table, table_len, start, n, k_out, v_out,
+                    stream=None) -> int:
+    return _lib.tq4_reconstruct(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, start, n,
+                                _ptr(k_out), _ptr(v_out), _stream(stream))
+
+
+def tq4_decode_workspace_bytes(ctx, n_req, n_q, total_seq_len) -> int:
+    return _lib.tq4_decode_workspace_bytes(ctx, n_req, n_q, total_seq_len)
+
+
+def tq4_decode_attention(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
+                         total_seq_len, scale, out, out_dtype, workspace, workspace_bytes,
+                         stream=None) -> int:
+    return _lib.tq4_decode_attention(ctx, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
+                                     _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out),
+                                     out_dtype, _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_prefill_workspace_bytes(n_tok) -> int:
+    return _lib.tq4_prefill_workspace_bytes(n_tok)
+
+
+def tq4_prefill_attention(ctx, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk, v_chunk,
+                          n_tok, scale, out, workspace, workspace_bytes, stream=None) -> int:
+    return _lib.tq4_prefill_attention(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, prefix_len,
+                                      _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale, _ptr(out),
+                                      _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_get_status(ctx, stream=None) -> int:
+    return _lib.tq4_get_status(ctx, _stream(stream))
+
+
+# ---------------------------------------------------------------- tensor-level helpers
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("TQ4 kernels take CUDA tensors")
+
+
+class Context:
+    """Owns a tq4_ctx for the current device."""
+
+    def __init__(self, signs):
+        self.handle = tq4_ctx_create(signs)
+
+    def close(self):
+        if self.handle:
+            tq4_ctx_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def codebook(self):
+        return tq4_codebook(self.handle)
+
+    def status(self, stream=None) -> int:
+        return tq4_get_status(self.handle, stream)
+
+    # -- pool helpers
+    @staticmethod
+    def new_pool(num_pages: int, device="cuda") -> torch.Tensor:
+        return torch.zeros(num_pages * PAGE_BYTES, dtype=torch.uint8, device=device)
+
+    def encode_append(self, pool, page_table, start_pos, k_new, v_new, stream=None):
+        _need_cuda(pool, page_table, k_new, v_new)
+        dtype = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(k_new.dtype)
+        if dtype is None or v_new.dtype != k_new.dtype:
+            raise ValueError("k_new/v_new must both be float32 or bfloat16")
+        n_tok = k_new.shape[0]
+        _check(tq4_encode_append(self.handle, pool, pool.numel() // PAGE_BYTES, page_table,
+                                 page_table.numel(), start_pos, n_tok, k_new, v_new, dtype, stream),
+               "tq4_encode_append")
+
+    def reconstruct(self, pool, page_table, start, n, stream=None):
+        _need_cuda(pool, page_table)
+        k = torch.empty((n, KV_HEADS, HEAD_DIM), dtype=torch.float32, device=pool.device)
+        v = torch.empty_like(k)
+        _check(tq4_reconstruct(self.handle, pool, pool.numel() // PAGE_BYTES, page_table, page_table.numel(),
+                               start, n, k, v, stream), "tq4_reconstruct")
+        return k, v
+
+    def decode_workspace(self, n_req, n_q, total_seq_len, device="cuda") -> torch.Tensor:
+        nbytes = tq4_decode_workspace_bytes(self.handle, n_req, n_q, total_seq_len)
+        return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+    def decode_attention(self, pool, q, page_tables, seq_lens, total_seq_len, scale, out=None,
+                         out_dtype=torch.bfloat16, workspace=None, stream=None):
+        """q: bf16 [n_req, n_q, 24, 256]; page_tables int32 [n_req, max_pages]; seq_lens int32 [n_req]."""
+        _need_cuda(pool, q, page_tables, seq_lens)
+        if q.dtype != torch.bfloat16:
+            raise ValueError("q must be bfloat16")
+        n_req, n_q = q.shape[0], q.shape[1]
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        if workspace is None:
+            workspace = self.decode_workspace(n_req, n_q, total_seq_len, q.device)
+        _check(tq4_decode_attention(self.handle, pool, pool.numel() // PAGE_BYTES, q, page_tables,
+                                    page_tables.shape[1], seq_lens, n_req, n_q, total_seq_len, scale, out,
+                                    od, workspace, workspace.numel(), stream), "tq4_decode_attention")
+        return out
+
+    def prefill_attention(self, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,
+                          workspace=None, stream=None):
+        """q: bf16 [n_tok, 24, 256]; k_chunk/v_chunk bf16 [n_tok, 4, 256]."""
+        _need_cuda(q, k_chunk, v_chunk)
+        n_tok = q.shape[0]
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+        if workspace is None:
+            workspace = torch.empty(max(tq4_prefill_workspace_bytes(n_tok), 256), dtype=torch.uint8,
+                                    device=q.device)
+        num_pages = pool.numel() // PAGE_BYTES if pool is not None else 0
+        tlen = page_table.numel() if page_table is not None else 0
+        _check(tq4_prefill_attention(self.handle, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk,
+                                     v_chunk, n_tok, scale, out, workspace, workspace.numel(), stream),
+               "tq4_prefill_attention")
+        return out

@@ -1,0 +1,178 @@
+/*
+ * tq4.h -- C ABI of the TQ4 paged-KV attention library (libtq4.so, CUDA sm_100a).
+ *
+ * The operation comes from the JustFit pages:
+ *   [KVEXEC] simpleprog.com, "Fitting a 27B-Parameter LLM into 24 GiB of Laptop
+ *            Memory", section "KVExec: Fused Reconstruction with Layer-Scoped
+ *            Lifetime": each 256-dim K or V head vector is stored as 32 U32 words
+ *            (eight 4-bit centroid indices per word) plus one FP16 norm;
+ *            reconstruction reads the packed page IDs, looks up centroids, applies
+ *            the inverse Hadamard rotation, restores the norm and feeds scaled
+ *            dot-product attention; single-query decode runs page-native on the
+ *            compressed data, multi-query prefill reconstructs then attends;
+ *            256-dim heads, 256-token pages.
+ *   [BUDGET] same page, section "The Memory Budget Equation": 16 attention
+ *            layers x 4 KV heads x 256 dims; 1,040 B per layer-position.
+ *   [V2]     wpnews.pro, "JustFit: Run Qwen 27B Fast with its full 256K context
+ *            on a 24 GB Mac", mechanism table, row KVExec: rotated-domain attention.
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   codebook   16-level Lloyd-Max quantiser for N(0, 1/256) (computed by the
+ *              library in fp64 at context creation); index j -> centroid c_j,
+ *              ascending; nearest centroid, ties to the lower index.
+ *   rotation   R = H diag(s) / 16, H the Sylvester Hadamard matrix, s the
+ *              caller's +-1 sign diagonal. Encode quantises y = R x / ||x||;
+ *              reconstruction is x_hat = fp16(||x||) * R^T c[idx].
+ *   packing    coordinate 8w+i is bits 4i..4i+3 of word w (little-endian u32).
+ *   norm       ||x||_2 rounded to fp16 (nearest even); zero vectors store 0.
+ *   GQA        24 query heads, query head h reads KV head h / 6.
+ *   page       one layer's pool is num_pages pages of TQ4_PAGE_BYTES bytes:
+ *                [0, 131072)       K words  [4 heads][256 slots][32 u32]
+ *                [131072, 262144)  V words  [4 heads][256 slots][32 u32]
+ *                [262144, 264192)  K norms  [4 heads][256 slots] fp16
+ *                [264192, 266240)  V norms  [4 heads][256 slots] fp16
+ *              Position p of a request lives in page page_table[p / 256],
+ *              slot p % 256. Page tables are int32 physical page ids.
+ *
+ * Memory: the caller owns every buffer. Pointers documented as "device" must be
+ * device memory (or managed memory) of the current device; "host" pointers are
+ * read before the call returns. The library allocates device memory only in
+ * tq4_ctx_create (a 4-byte status word) and frees it in tq4_ctx_destroy.
+ *
+ * Errors: every call returns TQ4_OK (0) or a negative TQ4_ERR_* code.
+ * Argument errors are detected on the host and returned synchronously, before
+ * anything is launched. Kernels run asynchronously on the given stream
+ * (a cudaStream_t passed as void*, NULL = legacy default stream). Problems that
+ * only the device can see (a page id outside [0, num_pages), a sequence length
+ * inconsistent with the table or the host-side bounds) make the kernel skip the
+ * affected work and record the first error code in the context's status word;
+ * tq4_get_status() reads and clears it. No kernel traps, and no kernel waits on
+ * another block.
+ *
+ * Dtypes: bf16 tensors are passed as raw uint16_t bit patterns.
+ */
+#ifndef TQ4_H
+#define TQ4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TQ4_OK                 0
+#define TQ4_ERR_ARG           -1  /* bad pointer, size, count or dtype             */
+#define TQ4_ERR_UNSUPPORTED   -2  /* shape this build is not specialised for       */
+#define TQ4_ERR_PAGE_RANGE    -3  /* page id outside [0, num_pages) (device check) */
+#define TQ4_ERR_CUDA          -4  /* a CUDA runtime call failed                    */
+#define TQ4_ERR_WORKSPACE     -5  /* workspace missing or smaller than required    */
+#define TQ4_ERR_SEQ           -6  /* device-side sequence length check failed      */
+
+#define TQ4_HEAD_DIM        256
+#define TQ4_PAGE_POSITIONS  256
+#define TQ4_KV_HEADS        4
+#define TQ4_Q_HEADS         24
+#define TQ4_WORDS           32
+#define TQ4_VECTOR_BYTES    130
+#define TQ4_POSITION_BYTES  1040          /* one layer-position: 4 heads x (K+V) x 130 B */
+#define TQ4_PAGE_BYTES      266240        /* 256 layer-positions                         */
+#define TQ4_MAX_QUERY_TOKENS 4
+
+#define TQ4_DTYPE_F32   0
+#define TQ4_DTYPE_BF16  1
+
+typedef struct tq4_ctx tq4_ctx;
+
+/* Create a context on the current CUDA device.
+ * signs: host, int8[256], each +1 or -1 (the rotation's sign diagonal).
+ * The context holds the signs, the codebook and a device status word.
+ * Returns TQ4_ERR_ARG for a NULL pointer or a sign that is not +-1. */
+int tq4_ctx_create(const int8_t* signs, tq4_ctx** out);
+
+/* Destroy a context; synchronises the device first. NULL is accepted. */
+int tq4_ctx_destroy(tq4_ctx* ctx);
+
+/* Copy the context's codebook: centroids[16] and decision boundaries[15]
+ * (midpoints of adjacent centroids), both host double arrays. */
+int tq4_codebook(const tq4_ctx* ctx, double* centroids, double* boundaries);
+
+/* Encode n_tok new positions of one layer and write them into the pool
+ * (step "rotate + quantize + pack new K/V into pages"; [KVEXEC], [BUDGET]).
+ *   pool        device, num_pages * TQ4_PAGE_BYTES bytes, written in place.
+ *   page_table  device int32[table_len], this request's physical page ids.
+ *   start_pos   position of the first new token; positions
+ *               [start_pos, start_pos + n_tok) must satisfy
+ *               (start_pos + n_tok + 255) / 256 <= table_len.
+ *   k_new,v_new device [n_tok][4][256] of dtype (TQ4_DTYPE_F32 or TQ4_DTYPE_BF16).
+ * n_tok == 0 is a no-op. Positions whose page id is out of range are skipped
+ * and TQ4_ERR_PAGE_RANGE is recorded in the status word. */
+int tq4_encode_append(tq4_ctx* ctx, void* pool, int32_t num_pages,
+                      const int32_t* page_table, int32_t table_len,
+                      int32_t start_pos, int32_t n_tok,
+                      const void* k_new, const void* v_new, int dtype, void* stream);
+
+/* Reconstruct positions [start, start + n) of one request as explicit fp32 K/V
+ * (centroid lookup, inverse rotation, norm restore; [KVEXEC]). Test/export path,
+ * not used by attention.
+ *   k_out, v_out device float[n][4][256]. */
+int tq4_reconstruct(tq4_ctx* ctx, const void* pool, int32_t num_pages,
+                    const int32_t* page_table, int32_t table_len,
+                    int32_t start, int32_t n, float* k_out, float* v_out, void* stream);
+
+/* Bytes of device workspace tq4_decode_attention needs for this problem
+ * (split-K partial results). total_seq_len = sum of seq_lens over requests. */
+size_t tq4_decode_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q,
+                                  int64_t total_seq_len);
+
+/* Decode attention: n_q (1..4) query tokens per request against the request's
+ * paged TQ4 history, fused with reconstruction, split-K with a combine pass
+ * ([KVEXEC] single-query page-native decode and packed verifier; [V2]
+ * rotated-domain attention). No full-precision K/V is written to memory.
+ *   pool         device, one layer, num_pages * TQ4_PAGE_BYTES bytes.
+ *   q            device bf16 [n_req][n_q][24][256].
+ *   page_tables  device int32 [n_req][max_pages].
+ *   seq_lens     device int32 [n_req]; positions per request INCLUDING the n_q
+ *                new ones, which must already be appended. Query token t of a
+ *                request sees positions [0, seq_len - n_q + t] (causal among the
+ *                n_q tokens).
+ *   total_seq_len host; sum of seq_lens (used to plan the split; the kernel
+ *                checks it and records TQ4_ERR_SEQ if the device values exceed it).
+ *   scale        softmax scale (e.g. 1/16 for dim 256).
+ *   out          device [n_req][n_q][24][256], out_dtype TQ4_DTYPE_BF16 or _F32.
+ *   workspace    device, at least tq4_decode_workspace_bytes(...) bytes, 256-B aligned.
+ * Softmax and all accumulation are fp32. */
+int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
+                         const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                         const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                         int64_t total_seq_len, float scale,
+                         void* out, int out_dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Prefill attention: a causal chunk of n_tok query tokens against the request's
+ * TQ4 prefix [0, prefix_len) plus the chunk itself, whose K/V are given at full
+ * precision ([KVEXEC] multi-query prefill). The chunk is not appended; call
+ * tq4_encode_append afterwards.
+ *   q                 device bf16 [n_tok][24][256].
+ *   k_chunk, v_chunk  device bf16 [n_tok][4][256].
+ *   page_table        device int32[table_len] covering the prefix.
+ *   out               device bf16 [n_tok][24][256].
+ *   workspace         device scratch of tq4_prefill_workspace_bytes(n_tok) bytes. */
+size_t tq4_prefill_workspace_bytes(int32_t n_tok);
+int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
+                          const int32_t* page_table, int32_t table_len, int32_t prefix_len,
+                          const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk,
+                          int32_t n_tok, float scale, uint16_t* out,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise the stream, return the first device-side error recorded since
+ * the last call (TQ4_OK if none) and clear it. */
+int tq4_get_status(tq4_ctx* ctx, void* stream);
+
+/* Static description of a status code. */
+const char* tq4_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ4_H */
