@@ -23,8 +23,15 @@ def _golden(name):
 
 
 @pytest.fixture(scope="module")
-def codebook():
+def solution():
+    """The fp64 Lloyd-Max solution (pinned against Max 1960)."""
     return O.lloyd_max_gaussian()
+
+
+@pytest.fixture(scope="module")
+def codebook():
+    """The stored (fp16) codebook that encode/decode use."""
+    return O.stored_codebook()
 
 
 @pytest.fixture(scope="module")
@@ -70,9 +77,9 @@ def test_gathered_state_is_1040_bytes_per_position(codebook, signs):
 
 
 # --------------------------------------------------------------------------- codebook
-def test_codebook_matches_max_1960(codebook):
+def test_codebook_matches_max_1960(solution):
     g = _golden("lloyd_max_gaussian_16.json")
-    c, b = codebook
+    c, b = solution
     unit_c = c * 16.0
     unit_b = b * 16.0
     def unit_in_last_place(v):
@@ -86,15 +93,27 @@ def test_codebook_matches_max_1960(codebook):
     assert abs(mse - g["mean_squared_error"]) < 1e-5
 
 
-def test_codebook_symmetric_and_midpoints(codebook):
-    c, b = codebook
+def test_codebook_symmetric_and_midpoints(solution):
+    c, b = solution
     assert np.all(np.diff(c) > 0)
     assert np.max(np.abs(c + c[::-1])) < 1e-15
     assert np.allclose(b, 0.5 * (c[1:] + c[:-1]), atol=0, rtol=0)
 
 
-def test_codebook_centroids_are_monte_carlo_conditional_means(codebook):
-    c, b = codebook
+def test_stored_codebook_is_fp16_of_solution(solution, codebook):
+    c, _ = solution
+    c16, b16 = codebook
+    for x, y in zip(c, c16):
+        assert np.float16(x) == y                       # round to nearest even of the fp64 value
+        assert abs(y - x) <= abs(x) * 2.0 ** -11        # within half an fp16 ulp (relative)
+    assert np.array_equal(c16, -c16[::-1])              # symmetric exactly after rounding
+    assert np.array_equal(b16, 0.5 * (c16[1:] + c16[:-1]))
+    # rounding the table costs nothing measurable in distortion
+    assert abs(O.quantiser_mse(c16 * 16, b16 * 16, 1.0) - O.quantiser_mse(c * 16, 0.5 * (c[1:] + c[:-1]) * 16, 1.0)) < 1e-6
+
+
+def test_codebook_centroids_are_monte_carlo_conditional_means(solution):
+    c, b = solution
     x = np.random.default_rng(11).standard_normal(20_000_000) / 16.0
     cell = np.searchsorted(b, x)
     sums = np.bincount(cell, weights=x, minlength=16)
