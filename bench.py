@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch without a CUDA graph (profiling)")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
+    ap.add_argument("--profile", action="store_true",
+                    help="eager steps only: no roofline replay, e2e or CPU leg (for ncu captures)")
     return ap.parse_args()
 
 
@@ -323,7 +326,7 @@ class OracleSample:
         from oracle import tq4_oracle as O
         self.O, self.w = O, w
         self.signs = I.signs(w.config)
-        self.c, _ = O.lloyd_max_gaussian()
+        self.c, _ = O.stored_codebook()
         self.tables = I.request_tables(w)
         if w.kind == "decode":
             T = min(int(w.seq_lens[0]), 8192)
@@ -422,6 +425,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
 
     w = I.WORKLOADS[args.workload]
+    if args.layers:
+        import dataclasses
+        w = dataclasses.replace(w, layers=args.layers)
+    if args.profile:
+        args.eager = True
     S = DecodeSetup(w, torch, tq4, device) if w.kind == "decode" else PrefillSetup(w, torch, tq4, device)
     stream = torch.cuda.Stream(device)
 
@@ -462,6 +470,10 @@ def main():
     if S.ctx.status() != tq4.TQ4_OK:
         raise RuntimeError("device status error during timing")
     value = S.units_per_step() * world / (ms * 1e-3)
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile": True, "workload": args.workload, "layers": w.layers, "ms_per_step": ms}))
+        return
 
     # dominant kernel: the attention call, timed alone (graph of the attention launches of all layers)
     hbm, bf16, bf16_sus, peak_kind = peaks()

@@ -11,6 +11,7 @@
 #include "tq4_device.cuh"
 #include "tq4_encode.cuh"
 #include "tq4_decode.cuh"
+#include "tq4_decode_q1.cuh"
 #include "tq4_prefill.cuh"
 
 struct tq4_ctx {
@@ -89,7 +90,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 DecodePlan plan_decode(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len) {
   DecodePlan pl{};
-  const int64_t ctas = int64_t(ctx->num_sms) * 2;            // two resident CTAs per SM
+  const int64_t ctas = int64_t(ctx->num_sms);                // one resident CTA per SM
   int64_t L = (total_seq_len * tq4::kHkv + ctas - 1) / ctas;  // positions per split
   L = ((L + tq4::kChunk - 1) / tq4::kChunk) * tq4::kChunk;
   if (L < tq4::kChunk) L = tq4::kChunk;
@@ -119,16 +120,27 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   tq4_ctx* ctx = new (std::nothrow) tq4_ctx();
   if (!ctx) return TQ4_ERR_ARG;
   ctx->signs = sb;
-  lloyd_max_16(1.0 / 16.0, ctx->centroids, ctx->boundaries);
+  // the format stores the 16 centroids as fp16; boundaries are midpoints of the stored values
+  double sol[16], sol_b[15];
+  lloyd_max_16(1.0 / 16.0, sol, sol_b);
   tq4::Codebook cb{};
   for (int j = 0; j < 16; ++j) {
-    cb.c[j] = float(ctx->centroids[j]);
-    cb.c16[j] = half_bits(ctx->centroids[j]);
+    cb.c16[j] = half_bits(sol[j]);
+    __half hh;
+    std::memcpy(&hh, &cb.c16[j], 2);
+    ctx->centroids[j] = double(__half2float(hh));
+    cb.c[j] = __half2float(hh);
   }
-  for (int j = 0; j < 15; ++j) cb.b[j] = float(ctx->boundaries[j]);
+  for (int j = 0; j < 15; ++j) {
+    ctx->boundaries[j] = 0.5 * (ctx->centroids[j] + ctx->centroids[j + 1]);
+    cb.b[j] = float(ctx->boundaries[j]);  // exact: the sum of two fp16 values fits in fp32
+  }
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(tq4::g_codebook, &cb, sizeof(cb));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tq4::decode_q1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(tq4::decode_q1_smem_bytes()));
   if (e == cudaSuccess) e = set_decode_attrs<1>();
   if (e == cudaSuccess) e = set_decode_attrs<2>();
   if (e == cudaSuccess) e = set_decode_attrs<3>();
@@ -233,20 +245,14 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   switch (tq4::decode_nt(n_q)) {
-    case 1:
-      tq4::decode_splitk_kernel<1><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<1>(), st>>>(p);
-      break;
-    case 2:
-      tq4::decode_splitk_kernel<2><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<2>(), st>>>(p);
-      break;
-    default:
-      tq4::decode_splitk_kernel<3><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<3>(), st>>>(p);
-      break;
+    case 1: tq4::decode_q1_kernel<<<grid, tq4::kQ1Threads, tq4::decode_q1_smem_bytes(), st>>>(p); break;
+    case 2: tq4::decode_splitk_kernel<2><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<2>(), st>>>(p); break;
+    default: tq4::decode_splitk_kernel<3><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<3>(), st>>>(p); break;
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return TQ4_ERR_CUDA;
   const int rows = n_req * n_q * tq4::kHq;
-  tq4::decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p);
+  tq4::decode_combine_kernel<<<rows, 32 * tq4::kCombWarps, 0, st>>>(p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -19,7 +19,7 @@
 //            on mma.m16n8k16 (M = positions, N = 6 query heads x n_q tokens,
 //            K = dims), nibble pairs decoded through a per-lane smem table.
 //   softmax  chunk max exchanged through smem; p = exp(s - m), P' = p * n_v
-//            written transposed (f16) to smem.
+//            written transposed to smem as an f16 hi + lo pair.
 //   V phase  warp w takes dims 64w..64w+63 of all 64 positions:
 //            O'^T += C_v^T . P'^T (M = dims, N = query rows, K = positions).
 // Per-split partial results (m, l, o') go to the workspace; the combine pass
@@ -29,12 +29,13 @@
 
 namespace tq4 {
 
-constexpr int kDecWarps = 4;
+constexpr int kDecWarps = 8;
 constexpr int kDecThreads = 32 * kDecWarps;
-constexpr int kChunk = 16 * kDecWarps;       // positions per chunk
+constexpr int kChunk = 16 * kDecWarps;       // positions per chunk (half a page)
+constexpr int kStages = 3;                   // cp.async ring depth
 constexpr int kQvStride = kD + 8;            // halves per Q' row in smem (bank-conflict pad)
 constexpr int kPsStride = kChunk + 8;        // halves per P' row in smem
-constexpr int kRowsMax = 24;                 // 6 query heads x 4 tokens
+constexpr int kStageBytes = 2 * kChunk * 128 + 2 * kChunk * 2;   // K words, V words, K norms, V norms
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeParams {
@@ -62,8 +63,8 @@ __host__ __device__ constexpr int decode_nt(int n_q) { return (6 * n_q + 7) / 8;
 
 template <int NT>
 constexpr size_t decode_smem_bytes() {
-  return size_t(kLutBytes) + size_t(8 * NT) * kQvStride * 2 + size_t(8 * NT) * kPsStride * 2 +
-         size_t(kDecWarps) * 8 * NT * 4;
+  return size_t(kLutBytes) + size_t(kStages) * kStageBytes + 2 * size_t(8 * NT) * kQvStride * 2 +
+         2 * size_t(8 * NT) * kPsStride * 2 + size_t(kDecWarps) * 8 * NT * 4;
 }
 
 __device__ __forceinline__ int warp_incl_scan(int v) {
@@ -110,13 +111,6 @@ __device__ __forceinline__ bool find_item(const DecodeParams& p, int x, int& req
   return found;
 }
 
-// Registers holding one chunk's packed data for one thread.
-struct ChunkRegs {
-  uint4 ka0, ka1, kb0, kb1;   // K words: positions g and g+8 of the warp's 16
-  uint32_t vw[16];            // V word (8w+g) of positions 16ks + {2t, 2t+1, 2t+8, 2t+9}
-  float kn[2], vn[2];         // K and V norms of positions g and g+8
-};
-
 __device__ __forceinline__ uint32_t pick(const uint4& a, const uint4& b, int i) {
   switch (i) {
     case 0: return a.x; case 1: return a.y; case 2: return a.z; case 3: return a.w;
@@ -124,14 +118,32 @@ __device__ __forceinline__ uint32_t pick(const uint4& a, const uint4& b, int i) 
   }
 }
 
+// 16-byte segment swizzle inside a staged 128-byte word row: the K phase
+// (segments t and 4+t of positions g, g+8 per quarter warp) and the V phase
+// (one word of positions 2t / 2t+1 per lane group) both hit 32 distinct banks.
+__device__ __forceinline__ int seg_swz(int pos) { return (((pos >> 1) & 3) << 1) ^ ((pos & 1) << 2); }
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
 template <int NT>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const char* lut = reinterpret_cast<const char*>(smem);
-  __half* qv = reinterpret_cast<__half*>(smem + kLutBytes);
-  __half* ps = qv + 8 * NT * kQvStride;
-  float* red = reinterpret_cast<float*>(ps + 8 * NT * kPsStride);   // [warps][8*NT]
-  __shared__ int s_item[3];
+  const uint32_t lut = smem_u32(smem);
+  uint8_t* ring = smem + kLutBytes;
+  __half* qv_hi = reinterpret_cast<__half*>(ring + kStages * kStageBytes);
+  __half* qv_lo = qv_hi + 8 * NT * kQvStride;
+  __half* ps_hi = qv_lo + 8 * NT * kQvStride;
+  __half* ps_lo = ps_hi + 8 * NT * kPsStride;   // P' = hi + lo, both f16
+  float* red = reinterpret_cast<float*>(ps_lo + 8 * NT * kPsStride);   // [warps][8*NT]
+  __shared__ int s_item[2];
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -154,9 +166,47 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
   const int seq_len = __ldg(p.seq_lens + r);
   const int pos_b = split * p.split_len;
   const int pos_e = min(pos_b + p.split_len, seq_len);
+  const int n_chunks = (pos_e - pos_b + kChunk - 1) / kChunk;
   const int NR = 6 * p.n_q;
+  const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
+  const int64_t head_slot0 = int64_t(h) * kPage;
 
-  // ---- rotate the queries of this (request, KV head): q' = R q * scale, f16, virtual order
+  // ---- staging: chunk i -> ring stage i % kStages (all threads issue 16-byte copies)
+  auto issue_chunk = [&](int i) {
+    if (i < n_chunks) {
+      const int c = pos_b + i * kChunk;
+      const int32_t page = __ldg(table + (c >> 8));
+      if (page < 0 || page >= p.num_pages) {
+        if (tid == 0) record_error(p.status, TQ4_ERR_PAGE_RANGE);
+      } else {
+        const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
+        const int64_t slot0 = head_slot0 + (c & (kPage - 1));
+        uint8_t* st = ring + (i % kStages) * kStageBytes;
+        const int nvalid = min(kChunk, pos_e - c);
+        // words: 2 x kChunk positions x 8 segments
+        for (int e = tid; e < 2 * kChunk * 8; e += kDecThreads) {
+          const int kv = e / (kChunk * 8), pl = (e >> 3) % kChunk, sg = e & 7;
+          if (pl < nvalid) {
+            const uint8_t* src = pg + (kv ? kVWords : kKWords) + (slot0 + pl) * 128 + sg * 16;
+            cp_async16(smem_u32(st + kv * kChunk * 128 + pl * 128 + ((sg ^ seg_swz(pl)) << 4)), src);
+          }
+        }
+        // norms: 2 x kChunk halves = 2 x (kChunk / 8) segments
+        if (tid < 2 * (kChunk / 8)) {
+          const int kv = tid / (kChunk / 8), sg = tid % (kChunk / 8);
+          if (sg * 8 < nvalid) {
+            const uint8_t* src = pg + (kv ? kVNorms : kKNorms) + (slot0 + sg * 8) * 2;
+            cp_async16(smem_u32(st + 2 * kChunk * 128 + kv * kChunk * 2 + sg * 16), src);
+          }
+        }
+      }
+    }
+    cp_async_commit();
+  };
+  issue_chunk(0);
+  issue_chunk(1);
+
+  // ---- rotate the queries of this (request, KV head): q' = R q * scale, split hi + lo f16, virtual order
   for (int row = w; row < 8 * NT; row += kDecWarps) {
     float v[8];
     if (row < NR) {
@@ -176,29 +226,38 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = 0.f;
     }
-    // lane owns real dims 8*lane + i (word lane). Word lane is loaded by K-phase thread
-    // t = (lane & 15) >> 2 as its word index ws = (lane & 3) + 4*(lane >> 4); k-step
-    // kk = 2*ws + (i >> 2), mma column 2t + (i & 1) + 8*((i >> 1) & 1).
+    // lane owns real dims 8*lane + i (word lane). Word lane is read in the K phase by
+    // thread t = (lane & 15) >> 2 as its word index ws = (lane & 3) + 4*(lane >> 4);
+    // k-step kk = 2*ws + (i >> 2), mma column 2t + (i & 1) + 8*((i >> 1) & 1).
     const int tt = (lane & 15) >> 2, wsel = (lane & 3) + 4 * (lane >> 4);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
       const int kk = 2 * wsel + (i >> 2);
       const int col = kk * 16 + ((i >> 1) & 1) * 8 + 2 * tt;
-      *reinterpret_cast<uint32_t*>(qv + row * kQvStride + col) = pack_half2(v[i], v[i + 1]);
+      const __half2 hi = __floats2half2_rn(v[i], v[i + 1]);
+      const float2 hf = __half22float2(hi);
+      *reinterpret_cast<__half2*>(qv_hi + row * kQvStride + col) = hi;
+      *reinterpret_cast<__half2*>(qv_lo + row * kQvStride + col) = __floats2half2_rn(v[i] - hf.x, v[i + 1] - hf.y);
     }
   }
-  lut_fill(reinterpret_cast<uint32_t*>(smem), tid, kDecThreads);
+  // centroid table: row b holds f16x2 {c[b & 15], c[b >> 4]} at +4*lane (the stored fp16 codebook)
+  for (int e = tid; e < 256 * 32; e += kDecThreads) {
+    const int b = e >> 5, l = e & 31;
+    reinterpret_cast<uint32_t*>(smem)[b * 64 + l] =
+        uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16);
+  }
   __syncthreads();
 
-  // ---- B fragments of Q' for the K phase (registers when they fit)
+  // ---- B fragments of Q' (hi, lo) for the K phase, in registers when they fit
   constexpr bool kQReg = (NT == 1);
-  uint32_t qb[kQReg ? 16 : 1][2];
+  uint32_t qh[kQReg ? 16 : 1][2], ql[kQReg ? 16 : 1][2];
   if constexpr (kQReg) {
 #pragma unroll
     for (int kk = 0; kk < 16; kk += 2) {
       const int m = lane >> 3;
-      const uint32_t addr = smem_u32(qv + (lane & 7) * kQvStride + (kk + (m >> 1)) * 16 + (m & 1) * 8);
-      ldmatrix_x4(qb[kk][0], qb[kk][1], qb[kk + 1][0], qb[kk + 1][1], addr);
+      const int off = (lane & 7) * kQvStride + (kk + (m >> 1)) * 16 + (m & 1) * 8;
+      ldmatrix_x4(qh[kk][0], qh[kk][1], qh[kk + 1][0], qh[kk + 1][1], smem_u32(qv_hi + off));
+      ldmatrix_x4(ql[kk][0], ql[kk][1], ql[kk + 1][0], ql[kk + 1][1], smem_u32(qv_lo + off));
     }
   }
 
@@ -223,60 +282,40 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
 #pragma unroll
       for (int i = 0; i < 4; ++i) o[nt][mt][i] = 0.f;
   }
+  const int dg = w & 3, ph = w >> 2;   // V phase: 64-dim group, 64-position half
 
-  const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
-  const int64_t head_slot0 = int64_t(h) * kPage;
+  for (int i = 0; i < n_chunks; ++i) {
+    cp_async_wait<1>();
+    __syncthreads();            // chunk i visible to all; everyone is done with chunk i-1
+    issue_chunk(i + 2);
+    const int c = pos_b + i * kChunk;
+    const uint8_t* st = ring + (i % kStages) * kStageBytes;
+    const uint8_t* kst = st;
+    const uint8_t* vst = st + kChunk * 128;
+    const __half* knr = reinterpret_cast<const __half*>(st + 2 * kChunk * 128);
+    const __half* vnr = knr + kChunk;
 
-  auto load_chunk = [&](int c, ChunkRegs& cr) {
-    int32_t page = __ldg(table + (c >> 8));
-    const bool page_ok = page >= 0 && page < p.num_pages;
-    if (!page_ok) {
-      if (tid == 0) record_error(p.status, TQ4_ERR_PAGE_RANGE);
-      page = 0;
-    }
-    const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
-    const int slot0 = c & (kPage - 1);
-    const int pk = c + 16 * w + g;  // K-phase positions pk, pk + 8
-    const bool v0 = page_ok && pk < pos_e, v8 = page_ok && pk + 8 < pos_e;
-    const uint8_t* kb = pg + kKWords + (head_slot0 + slot0 + 16 * w + g) * 128;
-    const uint4 z = make_uint4(0, 0, 0, 0);
-    cr.ka0 = v0 ? ldg128(kb + 16 * t) : z;
-    cr.ka1 = v0 ? ldg128(kb + 64 + 16 * t) : z;
-    cr.kb0 = v8 ? ldg128(kb + 8 * 128 + 16 * t) : z;
-    cr.kb1 = v8 ? ldg128(kb + 8 * 128 + 64 + 16 * t) : z;
-    const uint8_t* kn = pg + kKNorms + (head_slot0 + slot0 + 16 * w + g) * 2;
-    const uint8_t* vn = pg + kVNorms + (head_slot0 + slot0 + 16 * w + g) * 2;
-    cr.kn[0] = v0 ? ldg_half(kn) : 0.f;
-    cr.kn[1] = v8 ? ldg_half(kn + 16) : 0.f;
-    cr.vn[0] = v0 ? ldg_half(vn) : 0.f;
-    cr.vn[1] = v8 ? ldg_half(vn + 16) : 0.f;
-    const uint8_t* vb = pg + kVWords + (head_slot0 + slot0) * 128 + (8 * w + g) * 4;
+    // ---------------------------------------------------------- K phase: S = C_k Q'^T (fp32-grade)
+    const int pg0 = 16 * w + g;   // chunk-local positions pg0, pg0 + 8
+    const int sz = seg_swz(pg0);  // same for pg0 + 8
+    const uint4 ka0 = lds128(kst + pg0 * 128 + ((t ^ sz) << 4));
+    const uint4 ka1 = lds128(kst + pg0 * 128 + (((4 + t) ^ sz) << 4));
+    const uint4 kb0 = lds128(kst + (pg0 + 8) * 128 + ((t ^ sz) << 4));
+    const uint4 kb1 = lds128(kst + (pg0 + 8) * 128 + (((4 + t) ^ sz) << 4));
+    // scores = C_k (q'_hi + q'_lo): the centroid values are exact in f16, so two products
+    // with fp32 accumulation carry the scores to fp32 precision; even/odd k-steps use
+    // separate accumulators to halve the dependent mma chains
+    float shh[2][NT][4], sx[2][NT][4];
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks)
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int pl = 16 * ks + 2 * t + (j & 1) + 8 * (j >> 1);
-        cr.vw[ks * 4 + j] = (page_ok && c + pl < pos_e) ? ldg32(vb + pl * 128) : 0u;
-      }
-  };
-
-  ChunkRegs nxt;
-  if (pos_b < pos_e) load_chunk(pos_b, nxt);
-
-  for (int c = pos_b; c < pos_e; c += kChunk) {
-    const ChunkRegs cur = nxt;
-    if (c + kChunk < pos_e) load_chunk(c + kChunk, nxt);
-
-    // ------------------------------------------------------------ K phase: S = C_k Q'^T
-    float s[NT][4];
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) s[nt][i] = 0.f;
+        for (int j = 0; j < 4; ++j) shh[a][nt][j] = sx[a][nt][j] = 0.f;
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
-      const uint32_t wg = pick(cur.ka0, cur.ka1, kk >> 1);
-      const uint32_t wg8 = pick(cur.kb0, cur.kb1, kk >> 1);
+      const uint32_t wg = pick(ka0, ka1, kk >> 1);
+      const uint32_t wg8 = pick(kb0, kb1, kk >> 1);
       uint32_t a0, a1, a2, a3;
       if (kk & 1) {
         a0 = lut_decode<2>(lut, wg, lane4);
@@ -291,28 +330,33 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        uint32_t b0, b1;
+        uint32_t bh0, bh1, bl0, bl1;
         if constexpr (kQReg) {
-          b0 = qb[kk][0];
-          b1 = qb[kk][1];
+          bh0 = qh[kk][0]; bh1 = qh[kk][1]; bl0 = ql[kk][0]; bl1 = ql[kk][1];
         } else {
           const int m = (lane >> 3) & 1;
-          ldmatrix_x2(b0, b1, smem_u32(qv + (nt * 8 + (lane & 7)) * kQvStride + kk * 16 + m * 8));
+          const int off = (nt * 8 + (lane & 7)) * kQvStride + kk * 16 + m * 8;
+          ldmatrix_x2(bh0, bh1, smem_u32(qv_hi + off));
+          ldmatrix_x2(bl0, bl1, smem_u32(qv_lo + off));
         }
-        mma_16816(s[nt], a0, a1, a2, a3, b0, b1);
+        mma_16816(shh[kk & 1][nt], a0, a1, a2, a3, bh0, bh1);
+        mma_16816(sx[kk & 1][nt], a0, a1, a2, a3, bl0, bl1);
       }
     }
 
-    // ------------------------------------------------------------ online softmax
-    const int pk = c + 16 * w + g;
-    float mx[NT][2];
+    // ---------------------------------------------------------- online softmax over the chunk
+    const float kn0 = __half2float(knr[pg0]), kn8 = __half2float(knr[pg0 + 8]);
+    const float vn0 = __half2float(vnr[pg0]), vn8 = __half2float(vnr[pg0 + 8]);
+    const int pos0 = c + pg0;
+    float s[NT][4], mx[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int pos = pk + 8 * (i >> 1);
-        const bool ok = pos < pos_e && pos < lim[nt][i & 1];
-        s[nt][i] = ok ? s[nt][i] * cur.kn[i >> 1] : -INFINITY;
+      for (int j = 0; j < 4; ++j) {
+        const int pos = pos0 + 8 * (j >> 1);
+        const bool ok = pos < pos_e && pos < lim[nt][j & 1];
+        const float acc = (shh[0][nt][j] + shh[1][nt][j]) + (sx[0][nt][j] + sx[1][nt][j]);
+        s[nt][j] = ok ? acc * ((j >> 1) ? kn8 : kn0) : -INFINITY;
       }
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
@@ -338,23 +382,34 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
         for (int ww = 1; ww < kDecWarps; ++ww) mc = fmaxf(mc, red[ww * 8 * NT + nt * 8 + 2 * t + e]);
         const float m_new = fmaxf(m_run[nt][e], mc);
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[nt][e] = exp2f((m_run[nt][e] - m_use) * kLog2e);
+        alpha[nt][e] = fast_exp2((m_run[nt][e] - m_use) * kLog2e);
         m_run[nt][e] = m_new;
         mx[nt][e] = m_use;
       }
       float pr[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pr[i] = exp2f((s[nt][i] - mx[nt][i & 1]) * kLog2e);
+      for (int j = 0; j < 4; ++j) pr[j] = fast_exp2((s[nt][j] - mx[nt][j & 1]) * kLog2e);
       l_part[nt][0] = l_part[nt][0] * alpha[nt][0] + pr[0] + pr[2];
       l_part[nt][1] = l_part[nt][1] * alpha[nt][1] + pr[1] + pr[3];
-      const uint32_t p0 = pack_half2(pr[0] * cur.vn[0], pr[1] * cur.vn[0]);
-      const uint32_t p1 = pack_half2(pr[2] * cur.vn[1], pr[3] * cur.vn[1]);
-      const int j = lane & 7, mat = (lane >> 3) & 1;
-      stmatrix_x2_trans(smem_u32(ps + (nt * 8 + j) * kPsStride + 16 * w + 8 * mat), p0, p1);
+      // P' = p * n_v (zero where masked, so stale norms never enter)
+      const float w0 = s[nt][0] == -INFINITY ? 0.f : pr[0] * vn0;
+      const float w1 = s[nt][1] == -INFINITY ? 0.f : pr[1] * vn0;
+      const float w2 = s[nt][2] == -INFINITY ? 0.f : pr[2] * vn8;
+      const float w3 = s[nt][3] == -INFINITY ? 0.f : pr[3] * vn8;
+      const __half2 h01 = __floats2half2_rn(w0, w1), h23 = __floats2half2_rn(w2, w3);
+      const int jr = lane & 7, mat = (lane >> 3) & 1;
+      const int poff = (nt * 8 + jr) * kPsStride + 16 * w + 8 * mat;
+      stmatrix_x2_trans(smem_u32(ps_hi + poff), *reinterpret_cast<const uint32_t*>(&h01),
+                        *reinterpret_cast<const uint32_t*>(&h23));
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
+      const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
+      stmatrix_x2_trans(smem_u32(ps_lo + poff), *reinterpret_cast<const uint32_t*>(&l01),
+                        *reinterpret_cast<const uint32_t*>(&l23));
     }
     __syncthreads();
 
-    // ------------------------------------------------------------ V phase: O'^T += C_v^T P'^T
+    // ---------------------------------------------------------- V phase: O'^T += C_v^T P'^T
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -364,16 +419,25 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
         o[nt][mt][2] *= alpha[nt][0];
         o[nt][mt][3] *= alpha[nt][1];
       }
+    const int wd = 8 * dg + g;                       // the word (8 dims) this lane decodes
+    const int wseg = wd >> 2, wofs = (wd & 3) * 4;   // its 16-byte segment and offset
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
+      const int pb = 64 * ph + 16 * ks + 2 * t;
+      const uint32_t x0 = lds32(vst + pb * 128 + ((wseg ^ seg_swz(pb)) << 4) + wofs);
+      const uint32_t x1 = lds32(vst + (pb + 1) * 128 + ((wseg ^ seg_swz(pb + 1)) << 4) + wofs);
+      const uint32_t y0 = lds32(vst + (pb + 8) * 128 + ((wseg ^ seg_swz(pb + 8)) << 4) + wofs);
+      const uint32_t y1 = lds32(vst + (pb + 9) * 128 + ((wseg ^ seg_swz(pb + 9)) << 4) + wofs);
       uint32_t lo01, hi01, lo89, hi89;
-      interleave_nibbles(cur.vw[ks * 4 + 0], cur.vw[ks * 4 + 1], lo01, hi01);
-      interleave_nibbles(cur.vw[ks * 4 + 2], cur.vw[ks * 4 + 3], lo89, hi89);
-      uint32_t b[NT][2];
+      interleave_nibbles(x0, x1, lo01, hi01);
+      interleave_nibbles(y0, y1, lo89, hi89);
+      uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int m = (lane >> 3) & 1;
-        ldmatrix_x2(b[nt][0], b[nt][1], smem_u32(ps + (nt * 8 + (lane & 7)) * kPsStride + 16 * ks + 8 * m));
+        const int off = (nt * 8 + (lane & 7)) * kPsStride + 64 * ph + 16 * ks + 8 * m;
+        ldmatrix_x2(bh[nt][0], bh[nt][1], smem_u32(ps_hi + off));
+        ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
       }
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
@@ -397,14 +461,19 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
             break;
         }
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma_16816(o[nt][mt], a0, a1, a2, a3, b[nt][0], b[nt][1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          mma_16816(o[nt][mt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+          mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+        }
       }
     }
   }
+  cp_async_wait<0>();
 
   // ---------------------------------------------------------------- partial results
-  // l: sum over the lanes sharing t (positions g) and over the 4 warps' K phases
+  // l: over the lanes sharing t and over the 8 warps' K phases; o': over the two position halves
   __syncthreads();
+  float* ohalf = reinterpret_cast<float*>(ring);   // [4 dim groups][8*NT rows][64 dims] from warps 4..7
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -414,52 +483,54 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_splitk_kernel(const Dec
       v += __shfl_xor_sync(0xffffffffu, v, 8);
       v += __shfl_xor_sync(0xffffffffu, v, 16);
       if (g == 0) red[w * 8 * NT + nt * 8 + 2 * t + e] = v;
+      if (ph == 1) {
+        const int row = nt * 8 + 2 * t + e;
+        float* d = ohalf + (dg * 8 * NT + row) * 64 + 8 * g;
+        reinterpret_cast<float4*>(d)[0] = make_float4(o[nt][0][e], o[nt][0][e + 2], o[nt][1][e], o[nt][1][e + 2]);
+        reinterpret_cast<float4*>(d)[1] = make_float4(o[nt][2][e], o[nt][2][e + 2], o[nt][3][e], o[nt][3][e + 2]);
+      }
     }
   __syncthreads();
   const int64_t rec = (int64_t(blockIdx.x) * kHkv + h) * p.rows_pad;
-  if (tid < 8 * NT) {
-    float l = 0.f;
+  if (ph == 0) {
 #pragma unroll
-    for (int ww = 0; ww < kDecWarps; ++ww) l += red[ww * 8 * NT + tid];
-    // m of row tid: held by the lanes with t = (tid % 8) / 2 of n-tile tid / 8 (any warp)
-    red[tid] = l;  // only this thread reads/writes slot tid after the barrier above
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int row = nt * 8 + 2 * t + e;
+        const float* sidx = ohalf + (dg * 8 * NT + row) * 64 + 8 * g;
+        const float4 u0 = reinterpret_cast<const float4*>(sidx)[0];
+        const float4 u1 = reinterpret_cast<const float4*>(sidx)[1];
+        float* dst = p.ws_o + (rec + row) * kD + 64 * dg + 8 * g;
+        reinterpret_cast<float4*>(dst)[0] = make_float4(o[nt][0][e] + u0.x, o[nt][0][e + 2] + u0.y,
+                                                        o[nt][1][e] + u0.z, o[nt][1][e + 2] + u0.w);
+        reinterpret_cast<float4*>(dst)[1] = make_float4(o[nt][2][e] + u1.x, o[nt][2][e + 2] + u1.y,
+                                                        o[nt][3][e] + u1.z, o[nt][3][e + 2] + u1.w);
+      }
   }
-  // each thread with g == 0 knows m for its rows; publish through ws directly
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int row = nt * 8 + 2 * t + e;
-      float* dst = p.ws_o + (rec + row) * kD + 64 * w + 8 * g;
-      reinterpret_cast<float4*>(dst)[0] =
-          make_float4(o[nt][0][e], o[nt][0][e + 2], o[nt][1][e], o[nt][1][e + 2]);
-      reinterpret_cast<float4*>(dst)[1] =
-          make_float4(o[nt][2][e], o[nt][2][e + 2], o[nt][3][e], o[nt][3][e + 2]);
-    }
-  __syncthreads();
   if (w == 0 && g == 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int row = nt * 8 + 2 * t + e;
-        p.ws_ml[rec + row] = make_float2(m_run[nt][e], red[row]);
+        float l = 0.f;
+#pragma unroll
+        for (int ww = 0; ww < kDecWarps; ++ww) l += red[ww * 8 * NT + row];
+        p.ws_ml[rec + row] = make_float2(m_run[nt][e], l);
       }
   }
 }
 
-// One warp per output row (request, token, query head).
-__global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams p) {
-  const int lane = threadIdx.x & 31;
-  const int row_id = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (row_id >= p.n_req * p.n_q * kHq) return;
-  const int qh = row_id % kHq;
-  const int tok = (row_id / kHq) % p.n_q;
-  const int r = row_id / (kHq * p.n_q);
-  const int h = qh / kGroup;
-  const int row = tok * kGroup + qh % kGroup;
+// One CTA of 8 warps per output row (request, token, query head). Warp w
+// merges items first + w, first + w + 8, ... four at a time (all loads of a
+// group are issued before any is used, so the L2 round trips overlap), then
+// the 8 warp results are merged through shared memory, rotated back by R^T
+// and written out.
+constexpr int kCombWarps = 8;
 
-  // first item of request r and its number of splits
+__device__ __forceinline__ int request_first_item(const DecodeParams& p, int r) {
+  const int lane = threadIdx.x & 31;
   int first = 0;
   for (int r0 = 0; r0 < r; r0 += 32) {
     const int rr = r0 + lane;
@@ -472,40 +543,103 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const DecodeParams 
     for (int o = 16; o >= 1; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
     first += S;
   }
+  return first;
+}
+
+__global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const DecodeParams p) {
+  __shared__ float s_m[kCombWarps], s_l[kCombWarps];
+  __shared__ float4 s_acc[kCombWarps][32][2];
+  __shared__ int s_first;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row_id = blockIdx.x;
+  const int qh = row_id % kHq;
+  const int tok = (row_id / kHq) % p.n_q;
+  const int r = row_id / (kHq * p.n_q);
+  const int h = qh / kGroup;
+  const int row = tok * kGroup + qh % kGroup;
+
+  if (w == 0) {
+    const int f = request_first_item(p, r);
+    if (lane == 0) s_first = f;
+  }
+  __syncthreads();
+  const int first = s_first;
   const int s_len = __ldg(p.seq_lens + r);
-  float acc[8];
+  const bool ok = seq_ok(s_len, p.n_q, p.max_pages);
+  int n_split = ok ? (s_len + p.split_len - 1) / p.split_len : 0;
+  if (first + n_split > p.items_ub) n_split = 0;
+  if (threadIdx.x == 0 && (!ok || n_split == 0)) record_error(p.status, TQ4_ERR_SEQ);
+
+  float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  float l = 0.f;
-  const bool ok = seq_ok(s_len, p.n_q, p.max_pages);
-  const int n_split = ok ? (s_len + p.split_len - 1) / p.split_len : 0;
-  if (!ok && lane == 0) record_error(p.status, TQ4_ERR_SEQ);
-  if (first + n_split > p.items_ub) {
-    if (lane == 0) record_error(p.status, TQ4_ERR_SEQ);
-  } else if (n_split > 0) {
-    float m = -INFINITY;
-    for (int x = first; x < first + n_split; ++x)
-      m = fmaxf(m, p.ws_ml[(int64_t(x) * kHkv + h) * p.rows_pad + row].x);
-    for (int x = first; x < first + n_split; ++x) {
-      const int64_t rec = (int64_t(x) * kHkv + h) * p.rows_pad + row;
-      const float2 ml = p.ws_ml[rec];
-      if (ml.x == -INFINITY) continue;
-      const float wgt = exp2f((ml.x - m) * kLog2e);
-      l = fmaf(wgt, ml.y, l);
-      const float4* src = reinterpret_cast<const float4*>(p.ws_o + rec * kD + lane * 8);
-      const float4 u0 = src[0], u1 = src[1];
-      acc[0] = fmaf(wgt, u0.x, acc[0]); acc[1] = fmaf(wgt, u0.y, acc[1]);
-      acc[2] = fmaf(wgt, u0.z, acc[2]); acc[3] = fmaf(wgt, u0.w, acc[3]);
-      acc[4] = fmaf(wgt, u1.x, acc[4]); acc[5] = fmaf(wgt, u1.y, acc[5]);
-      acc[6] = fmaf(wgt, u1.z, acc[6]); acc[7] = fmaf(wgt, u1.w, acc[7]);
+  for (int x0 = first + w; x0 < first + n_split; x0 += 4 * kCombWarps) {
+    float2 ml[4];
+    float4 u[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int x = x0 + j * kCombWarps;
+      if (x < first + n_split) {
+        const int64_t rec = (int64_t(x) * kHkv + h) * p.rows_pad + row;
+        ml[j] = p.ws_ml[rec];
+        const float4* src = reinterpret_cast<const float4*>(p.ws_o + rec * kD + lane * 8);
+        u[j][0] = src[0];
+        u[j][1] = src[1];
+      } else {
+        ml[j] = make_float2(-INFINITY, 0.f);
+        u[j][0] = u[j][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    float mn = m;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) mn = fmaxf(mn, ml[j].x);
+    if (mn == -INFINITY) continue;
+    const float a = fast_exp2((m - mn) * kLog2e);
+    l *= a;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] *= a;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float wj = fast_exp2((ml[j].x - mn) * kLog2e);   // 0 for empty slots (m = -inf)
+      l = fmaf(wj, ml[j].y, l);
+      acc[0] = fmaf(wj, u[j][0].x, acc[0]); acc[1] = fmaf(wj, u[j][0].y, acc[1]);
+      acc[2] = fmaf(wj, u[j][0].z, acc[2]); acc[3] = fmaf(wj, u[j][0].w, acc[3]);
+      acc[4] = fmaf(wj, u[j][1].x, acc[4]); acc[5] = fmaf(wj, u[j][1].y, acc[5]);
+      acc[6] = fmaf(wj, u[j][1].z, acc[6]); acc[7] = fmaf(wj, u[j][1].w, acc[7]);
+    }
+    m = mn;
+  }
+  if (lane == 0) {
+    s_m[w] = m;
+    s_l[w] = l;
+  }
+  s_acc[w][lane][0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  s_acc[w][lane][1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  __syncthreads();
+  if (w != 0) return;
+  float M = -INFINITY;
+#pragma unroll
+  for (int ww = 0; ww < kCombWarps; ++ww) M = fmaxf(M, s_m[ww]);
+  float L = 0.f, o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int ww = 0; ww < kCombWarps; ++ww) {
+      const float a = fast_exp2((s_m[ww] - M) * kLog2e);
+      L = fmaf(a, s_l[ww], L);
+      const float4 v0 = s_acc[ww][lane][0], v1 = s_acc[ww][lane][1];
+      o[0] = fmaf(a, v0.x, o[0]); o[1] = fmaf(a, v0.y, o[1]); o[2] = fmaf(a, v0.z, o[2]);
+      o[3] = fmaf(a, v0.w, o[3]); o[4] = fmaf(a, v1.x, o[4]); o[5] = fmaf(a, v1.y, o[5]);
+      o[6] = fmaf(a, v1.z, o[6]); o[7] = fmaf(a, v1.w, o[7]);
     }
   }
   // o = R^T (o' / l) = diag(s) H (o' / l) / 16
-  warp_fwht256(acc);
-  const float inv = (l > 0.f) ? 0.0625f / l : 0.f;
+  warp_fwht256(o);
+  const float inv = (L > 0.f) ? 0.0625f / L : 0.f;
   float res[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) res[i] = acc[i] * inv * sign_of(p.signs, lane * 8 + i);
+  for (int i = 0; i < 8; ++i) res[i] = o[i] * inv * sign_of(p.signs, lane * 8 + i);
   const int64_t off = ((int64_t(r) * p.n_q + tok) * kHq + qh) * kD + lane * 8;
   if (p.out_dtype == TQ4_DTYPE_F32) {
     float* dst = static_cast<float*>(p.out) + off;

@@ -28,12 +28,13 @@ constexpr int64_t kVWords = int64_t(kHkv) * kPage * kWords * 4;   // 131072
 constexpr int64_t kKNorms = 2 * kVWords;                           // 262144
 constexpr int64_t kVNorms = kKNorms + int64_t(kHkv) * kPage * 2;   // 264192
 
-// codebook in constant memory, written once per process by the host from its
-// fp64 Lloyd-Max solution (same for every context; the signs are per context)
+// codebook in constant memory, written by the host from its fp64 Lloyd-Max
+// solution rounded to the stored fp16 table (same for every context; the signs
+// are per context)
 struct Codebook {
-  float c[16];        // centroids (fp32 of the fp64 values)
-  float b[15];        // decision boundaries (fp32 of the fp64 midpoints)
-  uint16_t c16[16];   // centroids as fp16 bits (round to nearest even from fp64)
+  float c[16];        // stored centroids (exact fp16 values held in fp32)
+  float b[15];        // decision boundaries: midpoints of adjacent stored centroids (exact in fp32)
+  uint16_t c16[16];   // stored centroids as fp16 bits (round to nearest even of the fp64 solution)
 };
 __constant__ Codebook g_codebook;  // one translation unit (tq4_api.cu) includes every kernel header
 
@@ -83,26 +84,34 @@ __device__ __forceinline__ float sign_of(const Signs& s, int coord) {
 // --------------------------------------------------------------------------
 // Nibble-pair decode through a per-lane table in shared memory.
 // Row b (one byte = two 4-bit indices) is 256 bytes; lane l reads its own
-// 4-byte slot at b*256 + 4*l, so the 32 lanes of a warp always hit 32
-// different banks. The slot holds f16x2 {c[b & 15], c[b >> 4]}.
+// 4-byte slot at b*256 + 4*l (and b*256 + 128 + 4*l for the low-order part),
+// so the 32 lanes of a warp always hit 32 different banks. A slot holds
+// f16x2 {c[b & 15], c[b >> 4]}.
 // --------------------------------------------------------------------------
 constexpr int kLutBytes = 256 * 256;
 
-__device__ __forceinline__ void lut_fill(uint32_t* lut, int tid, int nthreads) {
-  for (int e = tid; e < 256 * 32; e += nthreads) {
-    const int b = e >> 5, l = e & 31;
-    const uint32_t lo = g_codebook.c16[b & 15], hi = g_codebook.c16[b >> 4];
-    lut[b * 64 + l] = lo | (hi << 16);
-  }
+// shared-memory load through a 32-bit shared-window address
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(addr));
+  return v;
 }
 
-// byte k (0..3) of w -> f16x2 of its two nibbles (low nibble in the low half)
+// byte k (0..3) of w -> f16x2 of its two nibbles (low nibble in the low half).
+// lut_s is the table's 32-bit shared address; the byte lands in bits 8..15 of
+// the offset and the lane's slot in bits 0..7.
 template <int K>
-__device__ __forceinline__ uint32_t lut_decode(const char* lut, uint32_t w, uint32_t lane4) {
-  // result byte0 = lane*4 (from lane4), byte1 = byte K of w, bytes 2..3 = 0
+__device__ __forceinline__ uint32_t lut_decode(uint32_t lut_s, uint32_t w, uint32_t lane4) {
   constexpr uint32_t sel = (5u << 12) | (5u << 8) | (uint32_t(K) << 4) | 4u;
-  const uint32_t off = __byte_perm(w, lane4, sel);
-  return *reinterpret_cast<const uint32_t*>(lut + off);
+  return ld_shared_u32(lut_s + __byte_perm(w, lane4, sel));
+}
+
+// 2^x on the special-function unit (max relative error about 2^-22), used for
+// softmax weights; -inf maps to +0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Interleave the nibbles of two words: lo byte k = x_{2k} | y_{2k} << 4,

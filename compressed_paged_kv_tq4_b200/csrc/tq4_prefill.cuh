@@ -215,7 +215,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(const Prefi
       m_run[e] = m_new;
       l_run[e] *= alpha[e];
     }
-    uint32_t pa[8][2];
+    // P' = p * n_v as an f16 hi + lo pair (two mma per step keep PV at fp32 precision)
+    uint32_t pa[8][2], pb[8][2];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt) {
       float pr[4];
@@ -226,8 +227,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(const Prefi
       }
       const int pl = 8 * nt + 2 * t;
       const float v0 = nvs[pl], v1 = nvs[pl + 1];
-      pa[nt][0] = pack_half2(pr[0] * v0, pr[1] * v1);
-      pa[nt][1] = pack_half2(pr[2] * v0, pr[3] * v1);
+      const float w0 = s[nt][0] == -INFINITY ? 0.f : pr[0] * v0, w1 = s[nt][1] == -INFINITY ? 0.f : pr[1] * v1;
+      const float w2 = s[nt][2] == -INFINITY ? 0.f : pr[2] * v0, w3 = s[nt][3] == -INFINITY ? 0.f : pr[3] * v1;
+      const __half2 h01 = __floats2half2_rn(w0, w1), h23 = __floats2half2_rn(w2, w3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      pa[nt][0] = *reinterpret_cast<const uint32_t*>(&h01);
+      pa[nt][1] = *reinterpret_cast<const uint32_t*>(&h23);
+      pb[nt][0] = pack_half2(w0 - f01.x, w1 - f01.y);
+      pb[nt][1] = pack_half2(w2 - f23.x, w3 - f23.y);
     }
 #pragma unroll
     for (int nd = 0; nd < 32; ++nd) {
@@ -240,6 +247,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(const Prefi
 #pragma unroll
     for (int ks_ = 0; ks_ < 4; ++ks_) {
       const uint32_t a0 = pa[2 * ks_][0], a1 = pa[2 * ks_][1], a2 = pa[2 * ks_ + 1][0], a3 = pa[2 * ks_ + 1][1];
+      const uint32_t c0 = pb[2 * ks_][0], c1 = pb[2 * ks_][1], c2 = pb[2 * ks_ + 1][0], c3 = pb[2 * ks_ + 1][1];
 #pragma unroll
       for (int nd = 0; nd < 32; nd += 2) {
         uint32_t b0, b1, b2, b3;
@@ -248,6 +256,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_attn_kernel(const Prefi
                                    8 * (nd + (lane >> 4))));
         mma_16816(o[nd], a0, a1, a2, a3, b0, b1);
         mma_16816(o[nd + 1], a0, a1, a2, a3, b2, b3);
+        mma_16816(o[nd], c0, c1, c2, c3, b0, b1);
+        mma_16816(o[nd + 1], c0, c1, c2, c3, b2, b3);
       }
     }
   }
