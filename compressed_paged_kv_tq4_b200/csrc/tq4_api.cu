@@ -3,6 +3,7 @@
 // translation unit (the kernel headers are included below).
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <new>
 
 #include <cuda_runtime.h>
@@ -304,6 +305,57 @@ const char* tq4_status_string(int status) {
     case TQ4_ERR_SEQ: return "sequence length inconsistent with page table or plan";
     default: return "unknown status";
   }
+}
+
+// ---------------------------------------------------------------------------
+// Decode attention without any allocation by the caller or the library.
+//
+// Some callers cannot allocate device memory: plugin code running inside a host
+// program that owns the whole device-memory budget (a raw cudaMalloc would
+// bypass its accounting), and serving processes that reserve all device memory
+// up front and run under a hard memory guard. For them the split-K partial
+// results live in this fixed array instead of a caller-provided workspace.
+// The array is part of the library image: every GPU that loads the library
+// holds TQ4_NOALLOC_SCRATCH_BYTES of it until the process exits.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TQ4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is asked from the
+// runtime once per device (with that device current) and cached.
+int noalloc_scratch(int device, void** out) {
+  if (device < 0 || device >= kMaxDevices) return TQ4_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[device]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return TQ4_ERR_CUDA;
+    g_noalloc_ptr[device] = ptr;
+  }
+  *out = g_noalloc_ptr[device];
+  return TQ4_OK;
+}
+}  // namespace
+
+int tq4_decode_attention_noalloc(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q,
+                                 const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens,
+                                 int32_t n_req, int32_t n_q, int64_t total_seq_len, float scale, void* out,
+                                 int out_dtype, void* stream) {
+  if (!ctx) return TQ4_ERR_ARG;
+  if (n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS) return TQ4_ERR_UNSUPPORTED;
+  if (n_req == 0) return TQ4_OK;
+  if (n_req < 0 || total_seq_len <= 0) return TQ4_ERR_ARG;
+  if (tq4_decode_workspace_bytes(ctx, n_req, n_q, total_seq_len) > TQ4_NOALLOC_SCRATCH_BYTES)
+    return TQ4_ERR_WORKSPACE;
+  if (int rc = check_device(ctx)) return rc;
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(ctx->device, &scratch)) return rc;
+  return tq4_decode_attention(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
+                              total_seq_len, scale, out, out_dtype, scratch, TQ4_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

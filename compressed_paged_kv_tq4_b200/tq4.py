@@ -36,8 +36,9 @@ DTYPE_BF16 = 1
 EXPORTS = (
     "tq4_ctx_create", "tq4_ctx_destroy", "tq4_codebook", "tq4_encode_append", "tq4_reconstruct",
     "tq4_decode_workspace_bytes", "tq4_decode_attention", "tq4_prefill_workspace_bytes",
-    "tq4_prefill_attention", "tq4_get_status", "tq4_status_string",
+    "tq4_prefill_attention", "tq4_get_status", "tq4_status_string", "tq4_decode_attention_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def _load():
@@ -68,6 +69,8 @@ _sig = {
     "tq4_prefill_attention": ([_p, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p, _p, _sz, _p],
                               ctypes.c_int),
     "tq4_get_status": ([_p, _p], ctypes.c_int),
+    "tq4_decode_attention_noalloc": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int, _p],
+                                     ctypes.c_int),
     "tq4_status_string": ([ctypes.c_int], ctypes.c_char_p),
 }
 for _name, (_args, _res) in _sig.items():
@@ -161,6 +164,15 @@ def tq4_prefill_attention(ctx, pool, num_pages, page_table, table_len, prefix_le
     return _lib.tq4_prefill_attention(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, prefix_len,
                                       _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale, _ptr(out),
                                       _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_decode_attention_noalloc(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
+                                 total_seq_len, scale, out, out_dtype, stream=None) -> int:
+    """Decode attention whose split-K scratch is the library's fixed device array
+    (for callers that cannot allocate device memory; see include/tq4.h)."""
+    return _lib.tq4_decode_attention_noalloc(ctx, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
+                                             _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out),
+                                             out_dtype, _stream(stream))
 
 
 def tq4_get_status(ctx, stream=None) -> int:

@@ -165,6 +165,34 @@ int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                           int32_t n_tok, float scale, uint16_t* out,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode attention for callers that cannot allocate device memory.
+ * The pages have no counterpart to this call; it exists for the library's users.
+ * Some callers cannot allocate: plugin code inside a host program that owns the
+ * whole device-memory budget (a raw cudaMalloc would bypass its accounting),
+ * and serving processes that reserve all device memory up front and run under
+ * a hard memory guard. This call takes the same arguments as
+ * tq4_decode_attention minus the workspace, and keeps the split-K partial
+ * results in a fixed array of TQ4_NOALLOC_SCRATCH_BYTES (8 MiB) that is part of
+ * the library: every GPU that loads the library holds it until the process
+ * exits. It allocates nothing and calls no allocating routine.
+ *   - The first call on a device looks up the array's device address (the
+ *     runtime call cudaGetSymbolAddress, under a lock) and caches it; make that
+ *     first call on each device before any stream capture.
+ *   - Every call on a device shares the one array, so calls whose kernels may
+ *     overlap on the GPU (different streams, no ordering between them) race
+ *     and give wrong results; order them, e.g. issue them on one stream.
+ *   - Nothing in the array needs to start at zero: each call writes every
+ *     partial result it later reads.
+ *   - A problem whose tq4_decode_workspace_bytes() exceeds
+ *     TQ4_NOALLOC_SCRATCH_BYTES is rejected with TQ4_ERR_WORKSPACE before
+ *     anything is launched (about 200 single-token requests at most). */
+#define TQ4_NOALLOC_SCRATCH_BYTES (8u << 20)
+int tq4_decode_attention_noalloc(tq4_ctx* ctx, const void* pool, int32_t num_pages,
+                                 const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                 int64_t total_seq_len, float scale,
+                                 void* out, int out_dtype, void* stream);
+
 /* Synchronise the stream, return the first device-side error recorded since
  * the last call (TQ4_OK if none) and clear it. */
 int tq4_get_status(tq4_ctx* ctx, void* stream);
