@@ -6,6 +6,7 @@
 #include <mutex>
 #include <new>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/tq4.h"
@@ -88,6 +89,37 @@ struct DecodePlan {
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// cuTensorMapEncodeTiled, fetched from the driver through the runtime once.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// Tensor map over one layer's pool seen as rows of 128 B (32 u32), 2,080 rows
+// per page; boxes of 32 rows; 128-byte swizzle in shared memory.
+int pool_tensor_map(const void* pool, int32_t num_pages, CUtensorMap* map) {
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return TQ4_ERR_CUDA;
+  const cuuint64_t dims[2] = {32, cuuint64_t(num_pages) * (TQ4_PAGE_BYTES / 128)};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t elem[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(pool), dims, strides, box, elem,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? TQ4_OK : TQ4_ERR_CUDA;
+}
 
 DecodePlan plan_decode(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len) {
   DecodePlan pl{};
@@ -246,7 +278,12 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   switch (tq4::decode_nt(n_q)) {
-    case 1: tq4::decode_q1_kernel<<<grid, tq4::kQ1Threads, tq4::decode_q1_smem_bytes(), st>>>(p); break;
+    case 1: {
+      CUtensorMap map;
+      if (int rc = pool_tensor_map(pool, num_pages, &map)) return rc;
+      tq4::decode_q1_kernel<<<grid, tq4::kQ1Threads, tq4::decode_q1_smem_bytes(), st>>>(p, map);
+      break;
+    }
     case 2: tq4::decode_splitk_kernel<2><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<2>(), st>>>(p); break;
     default: tq4::decode_splitk_kernel<3><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<3>(), st>>>(p); break;
   }
@@ -303,6 +340,7 @@ const char* tq4_status_string(int status) {
     case TQ4_ERR_CUDA: return "CUDA runtime error";
     case TQ4_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
     case TQ4_ERR_SEQ: return "sequence length inconsistent with page table or plan";
+    case TQ4_ERR_TIMEOUT: return "a bounded device-side wait gave up";
     default: return "unknown status";
   }
 }

@@ -7,41 +7,59 @@
 // each other inside the main loop:
 //
 //   * a CTA (8 warps) owns one (request, KV head, split); warp w takes the
-//     16-position tiles w, w+8, w+16, ... of the split;
-//   * each warp stages its own tiles through a private cp.async ring
-//     (K words, V words, norms: 4,160 bytes per tile);
-//   * K phase: S = C_k (q'_hi + q'_lo) on mma.m16n8k16 (M = 16 positions,
-//     N = 6 query heads padded to 8, K = 256 dims);
-//   * in-warp online softmax; P' = p * n_v split into f16 hi + lo and moved
-//     into B-operand layout with movmatrix (no shared memory);
+//     32-position tiles w, w+8, w+16, ... of the split;
+//   * lane 0 of each warp streams its tiles with TMA (2D tensor loads of the
+//     K and V word rows with the 128-byte swizzle, bulk copies of the two norm
+//     rows) into a private two-stage ring, completion on an mbarrier;
+//   * K phase: S = C_k (q'_hi + q'_lo) on mma.m16n8k16 for two m-tiles
+//     (M = 16 positions, N = 6 query heads padded to 8, K = 256 dims);
+//   * in-warp online softmax with lazy rescaling (the reference max is raised
+//     only when a row max grows by more than 2^8); P' = p * n_v split into f16
+//     hi + lo and moved into B-operand layout with movmatrix;
 //   * V phase: O'^T += C_v^T P'^T over all 256 dims (M = dims, K = positions);
 //   * at the end the 8 warp states (m, l, o') are merged through shared memory
 //     and written as one split-K partial for the combine pass.
 #pragma once
+#include <cuda.h>
 #include "tq4_decode.cuh"
 
 namespace tq4 {
 
 constexpr int kQ1Warps = 8;
 constexpr int kQ1Threads = 32 * kQ1Warps;
-constexpr int kQ1Stages = 4;
-constexpr int kQ1TileBytes = 16 * 128 * 2 + 16 * 2 * 2;    // K words, V words, K norms, V norms
-constexpr int kQ1WarpRing = kQ1Stages * kQ1TileBytes;        // 16,640 B
-// Shared-window layout (absolute 32-bit shared addresses): the centroid table
+constexpr int kQ1Tile = 32;                    // positions per warp iteration (two mma m-tiles)
+constexpr int kQ1Stages = 2;                   // TMA ring depth per warp
+constexpr int kQ1KV = kQ1Tile * 128;           // 4,096 B: one K (or V) tile, 128-B swizzled rows
+constexpr int kQ1Buf = 2 * kQ1KV;              // K then V
+constexpr int kQ1Bufs = kQ1Warps * kQ1Stages;  // 16 tile buffers
+constexpr uint32_t kQ1TxBytes = 2 * kQ1KV + 2 * kQ1Tile * 2;   // words + both norm rows
+// Shared-window layout (absolute 32-bit shared addresses). The centroid table
 // sits at 0x10000 so that one byte permute builds a lookup address
-// (0x10000 | byte << 8 | lane * 4). Below it: control words, q' and the rings
-// of warps 0..2; above it: the rings of warps 3..7 (also the merge area).
+// (0x10000 | byte << 8 | lane * 4). Below it: control words, q', mbarriers,
+// norm rows and the first tile buffers; above it: the other tile buffers.
 constexpr uint32_t kQ1Lut = 0x10000;
 constexpr uint32_t kQ1Hi = 0x20000;
-constexpr int kQ1LowWarps = 3;
-constexpr uint32_t kQ1LowBytes = 128 + 2 * 8 * kQvStride * 2 + kQ1LowWarps * kQ1WarpRing;   // 58,496
-constexpr uint32_t kQ1DynBytes = kQ1Hi + (kQ1Warps - kQ1LowWarps) * kQ1WarpRing;            // 214,272
+constexpr uint32_t kQ1QvOff = 128;
+constexpr uint32_t kQ1BarOff = kQ1QvOff + 2 * 8 * kQvStride * 2;      // 8,576
+constexpr uint32_t kQ1NrmOff = kQ1BarOff + 128;                        // 16 x 128 B of norm rows
+constexpr uint32_t kQ1CtlBytes = kQ1NrmOff + kQ1Bufs * 128;           // 10,752
+constexpr int kQ1LowBufs = 6;
+constexpr uint32_t kQ1DynBytes = kQ1Hi + (kQ1Bufs - kQ1LowBufs) * kQ1Buf;   // 212,992
 constexpr int kQ1MergeBytes = kQ1Warps * (8 * kD + 16) * 4;
-static_assert(kQ1MergeBytes <= (kQ1Warps - kQ1LowWarps) * kQ1WarpRing, "merge area fits above the table");
-constexpr float kQ1PScale = 1.0f / 256.0f;   // P' = p * n_v / 256 (undone in the combine)
+static_assert(kQ1MergeBytes <= (kQ1Bufs - kQ1LowBufs) * kQ1Buf, "merge area fits above the table");
+static_assert(kQ1DynBytes <= 227 * 1024, "fits the per-CTA shared memory");
+constexpr float kQ1PScale = 1.0f / 256.0f;   // P' = p * n_v / 256 (undone when the partial is written)
 constexpr float kQ1Lazy = 8.0f;              // rescale only when a row max grows by > 2^8 (log2 units)
+constexpr uint32_t kQ1SpinLimit = 1u << 24;  // bounded wait on a tile's arrival
 
 constexpr size_t decode_q1_smem_bytes() { return kQ1DynBytes; }
+
+// MMA row m (0..15) of an m-tile holds tile-local position sigma(m & 7) + (m & 8):
+// with the 128-B swizzle (16-B chunk index XOR row & 7) this makes the K-phase
+// and V-phase shared loads conflict-free.
+__host__ __device__ constexpr int q1_sigma(int m) {
+  return ((0x37156240u >> (4 * (m & 7))) & 7) + (m & 8);
+}
 
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
@@ -52,6 +70,15 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
+}
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void st_shared_f4(uint32_t a, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
   uint16_t v;
@@ -68,21 +95,54 @@ __device__ __forceinline__ uint32_t lut64k(uint32_t w, uint32_t lanebase) {
   return ld_shared_u32(__byte_perm(w, lanebase, sel));
 }
 
-__global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodeParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
+// ---- mbarrier and bulk-copy primitives (one CTA = its own cluster; no multicast)
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// The pool seen by the tensor map: rows of 128 B (32 u32), 2,080 rows per page:
+// K words (4 heads x 256 slots), V words, then 32 rows of norms.
+constexpr int kRowsPerPage = int(kPageBytes / 128);   // 2,080
+
+__global__ void __launch_bounds__(kQ1Threads, 1)
+    decode_q1_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int h = blockIdx.y;
-  if (base + kQ1LowBytes > kQ1Lut) {   // the layout needs the dynamic window to start low
+  const uint32_t low0 = (base + kQ1CtlBytes + 1023) & ~1023u;
+  if (low0 + kQ1LowBufs * kQ1Buf > kQ1Lut) {   // the layout needs the dynamic window to start low
     if (tid == 0) record_error(p.status, TQ4_ERR_CUDA);
     return;
   }
   int* s_item = reinterpret_cast<int*>(smem);
-  __half* qv_hi = reinterpret_cast<__half*>(smem + 128);
+  __half* qv_hi = reinterpret_cast<__half*>(smem + kQ1QvOff);
   __half* qv_lo = qv_hi + 8 * kQvStride;
-  const uint32_t ring = w < kQ1LowWarps ? base + 128 + 2 * 8 * kQvStride * 2 + w * kQ1WarpRing
-                                        : kQ1Hi + (w - kQ1LowWarps) * kQ1WarpRing;
+  auto buf_addr = [&](int b) { return b < kQ1LowBufs ? low0 + b * kQ1Buf : kQ1Hi + (b - kQ1LowBufs) * kQ1Buf; };
   const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 4u);
 
   if (w == 0) {
@@ -94,6 +154,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
       if (blockIdx.x == 0 && h == 0 && total > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
     }
   }
+  if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   __syncthreads();
   const int r = s_item[0];
   if (r < 0 || int(blockIdx.x) >= p.items_ub) return;
@@ -101,57 +163,34 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
   const int seq_len = __ldg(p.seq_lens + r);
   const int pos_b = split * p.split_len;
   const int pos_e = min(pos_b + p.split_len, seq_len);
-  const int n_tiles = (pos_e - pos_b + 15) >> 4;
+  const int n_tiles = (pos_e - pos_b + kQ1Tile - 1) / kQ1Tile;
   const int my_tiles = n_tiles > w ? (n_tiles - w + kQ1Warps - 1) / kQ1Warps : 0;
   const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
-  const uint8_t* pool = p.pool;
-  const int num_pages = p.num_pages;
-  const int64_t head_off = int64_t(h) * kPage * 128;        // head's first word row inside a region
 
-  // per-lane copy plan: 8 word segments (K then V) and, for lanes 0..3, one norm segment
-  int src_off[8];
-  uint32_t dst_off[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int e = lane + 32 * j;
-    const int kv = e >> 7, pl = (e >> 3) & 15, sg = e & 7;
-    src_off[j] = int(kv ? kVWords : kKWords) + pl * 128 + sg * 16;
-    dst_off[j] = uint32_t(kv * 2048 + pl * 128 + ((sg ^ seg_swz(pl)) << 4));
-  }
-  const int nrm_src = int((lane >> 1) ? kVNorms : kKNorms) + (lane & 1) * 16;
-  const uint32_t nrm_dst = 4096 + (lane >> 1) * 32 + (lane & 1) * 16;
-
-  auto tile_pos = [&](int k) { return pos_b + ((w + k * kQ1Warps) << 4); };
-  int page_next = my_tiles > 0 ? __ldg(table + (tile_pos(0) >> 8)) : 0;
+  // ---- lane 0 of each warp streams the warp's tiles: tile w + 8k -> buffer w*2 + k%2
+  auto tile_pos = [&](int k) { return pos_b + (w + k * kQ1Warps) * kQ1Tile; };
   auto issue_tile = [&](int k) {
-    if (k < my_tiles) {
+    if (lane == 0 && k < my_tiles) {
       const int c = tile_pos(k);
-      const int page = page_next;
-      if (k + 1 < my_tiles) page_next = __ldg(table + (tile_pos(k + 1) >> 8));
-      if (page < 0 || page >= num_pages) {
-        if (lane == 0) record_error(p.status, TQ4_ERR_PAGE_RANGE);
-      } else {
-        const int nvalid = min(16, pos_e - c);
-        const uint8_t* tb = pool + int64_t(page) * kPageBytes + head_off + (c & (kPage - 1)) * 128;
-        const uint32_t st = ring + (k % kQ1Stages) * kQ1TileBytes;
-        if (nvalid == 16) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) cp_async16(st + dst_off[j], tb + src_off[j]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (((lane + 32 * j) >> 3 & 15) < nvalid) cp_async16(st + dst_off[j], tb + src_off[j]);
-        }
-        // norms: K and V, 16 halves each (2 x 2 segments); slot offset = word offset / 64
-        if (lane < 4 && (lane & 1) * 8 < nvalid)
-          cp_async16(st + nrm_dst, pool + int64_t(page) * kPageBytes + nrm_src +
-                                       (head_off + (c & (kPage - 1)) * 128) / 64);
+      const int b = w * kQ1Stages + (k % kQ1Stages);
+      const uint32_t bar = base + kQ1BarOff + b * 8;
+      int page = __ldg(table + (c >> 8));
+      if (page < 0 || page >= p.num_pages) {
+        record_error(p.status, TQ4_ERR_PAGE_RANGE);
+        page = 0;   // still complete the barrier (reading page 0); the tile is masked below
       }
+      const int slot0 = h * kPage + (c & (kPage - 1));
+      const int row = page * kRowsPerPage + slot0;
+      const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
+      const uint32_t kdst = buf_addr(b), ndst = base + kQ1NrmOff + b * 128;
+      mbar_expect_tx(bar, kQ1TxBytes);
+      tma_load_2d(kdst, &tmap, 0, row, bar);                       // K words of 32 positions
+      tma_load_2d(kdst + kQ1KV, &tmap, 0, row + 4 * kPage, bar);   // V words
+      bulk_load(ndst, pg + kKNorms + slot0 * 2, kQ1Tile * 2, bar);
+      bulk_load(ndst + 64, pg + kVNorms + slot0 * 2, kQ1Tile * 2, bar);
     }
-    cp_async_commit();
   };
-#pragma unroll
-  for (int k = 0; k < kQ1Stages - 1; ++k) issue_tile(k);
+  issue_tile(0);
 
   // ---- q' = R q * scale for the 6 query heads of this KV head, split hi + lo, virtual order
   {
@@ -179,9 +218,9 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
       const int kk = 2 * wsel + (i >> 2);
       const int col = kk * 16 + ((i >> 1) & 1) * 8 + 2 * tt;
       const __half2 hi = __floats2half2_rn(v[i], v[i + 1]);
-      const float2 hf = __half22float2(hi);
+      const float2 hfl = __half22float2(hi);
       *reinterpret_cast<__half2*>(qv_hi + row * kQvStride + col) = hi;
-      *reinterpret_cast<__half2*>(qv_lo + row * kQvStride + col) = __floats2half2_rn(v[i] - hf.x, v[i + 1] - hf.y);
+      *reinterpret_cast<__half2*>(qv_lo + row * kQvStride + col) = __floats2half2_rn(v[i] - hfl.x, v[i + 1] - hfl.y);
     }
   }
   for (int e = tid; e < 256 * 32; e += kQ1Threads) {
@@ -200,9 +239,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
     ldmatrix_x4(ql[kk][0], ql[kk][1], ql[kk + 1][0], ql[kk + 1][1], smem_u32(qv_lo + off));
   }
 
-  // rows 2t, 2t+1 (query heads); only 6 are real
-  const bool row_ok0 = 2 * t < 6, row_ok1 = 2 * t + 1 < 6;
-  // m_ref: the reference the exponentials use (raised lazily); m_run: true running max
+  const bool row_ok0 = 2 * t < 6, row_ok1 = 2 * t + 1 < 6;   // query heads 2t, 2t+1
   float m_ref[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
   float o[16][4];
 #pragma unroll
@@ -210,59 +247,82 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
 #pragma unroll
     for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
 
-  const uint32_t k_off0 = g * 128 + ((t ^ seg_swz(g)) << 4);
-  const uint32_t k_off1 = g * 128 + (((4 + t) ^ seg_swz(g)) << 4);
-  const uint32_t v_off0 = 2048 + (2 * t) * 128 + ((g ^ seg_swz(2 * t)) << 4);      // words 4g..4g+3, pos 2t
-  const uint32_t v_off1 = 2048 + (2 * t + 1) * 128 + ((g ^ seg_swz(2 * t + 1)) << 4);  // pos 2t+1
+  // positions of this lane: K phase rows g, g+8 -> sigma; V phase k-indices 2t, 2t+1 (+8)
+  const int pk = q1_sigma(g);                        // and pk + 8 (same swizzle phase)
+  const int pv0 = q1_sigma(2 * t), pv1 = q1_sigma(2 * t + 1);
+  const uint32_t k_off0 = pk * 128 + ((t ^ (pk & 7)) << 4);          // words 4t..4t+3
+  const uint32_t k_off1 = pk * 128 + (((4 + t) ^ (pk & 7)) << 4);    // words 16+4t..16+4t+3
+  const uint32_t v_off0 = pv0 * 128 + ((g ^ (pv0 & 7)) << 4);        // words 4g..4g+3 of position pv0
+  const uint32_t v_off1 = pv1 * 128 + ((g ^ (pv1 & 7)) << 4);
+  bool timed_out = false;
+
   for (int k = 0; k < my_tiles; ++k) {
-    issue_tile(k + kQ1Stages - 1);
-    cp_async_wait<kQ1Stages - 1>();
-    __syncwarp();
-    const uint32_t st = ring + (k % kQ1Stages) * kQ1TileBytes;
+    issue_tile(k + 1);
+    const int b = w * kQ1Stages + (k % kQ1Stages);
+    const uint32_t bar = base + kQ1BarOff + b * 8;
+    {
+      uint32_t spins = 0;
+      while (!mbar_try_wait(bar, (k / kQ1Stages) & 1)) {
+        if (++spins > kQ1SpinLimit) { timed_out = true; break; }
+      }
+      if (__any_sync(0xffffffffu, timed_out)) {
+        if (lane == 0) record_error(p.status, TQ4_ERR_TIMEOUT);
+        break;
+      }
+    }
+    const uint32_t kst = buf_addr(b), vst = kst + kQ1KV;
+    const uint32_t nb = base + kQ1NrmOff + b * 128;
     const int c = tile_pos(k);
 
-    // ------------------------------------------------------------ K phase
-    const uint4 ka0 = ld_shared_v4(st + k_off0);
-    const uint4 ka1 = ld_shared_v4(st + k_off1);
-    const uint4 kb0 = ld_shared_v4(st + k_off0 + 8 * 128);
-    const uint4 kb1 = ld_shared_v4(st + k_off1 + 8 * 128);
-    float sh[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    float sl[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    // ------------------------------------------------------------ K phase, two m-tiles
+    uint4 ka[2], kb4[2], kc[2], kd[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t mrow = kst + j * 16 * 128;
+      ka[j] = ld_shared_v4(mrow + k_off0);
+      kb4[j] = ld_shared_v4(mrow + k_off1);
+      kc[j] = ld_shared_v4(mrow + 8 * 128 + k_off0);
+      kd[j] = ld_shared_v4(mrow + 8 * 128 + k_off1);
+    }
+    float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
-      const uint32_t wg = pick(ka0, ka1, kk >> 1);
-      const uint32_t wg8 = pick(kb0, kb1, kk >> 1);
-      uint32_t a0, a1, a2, a3;
-      if (kk & 1) {
-        a0 = lut64k<2>(wg, lanebase); a1 = lut64k<2>(wg8, lanebase);
-        a2 = lut64k<3>(wg, lanebase); a3 = lut64k<3>(wg8, lanebase);
-      } else {
-        a0 = lut64k<0>(wg, lanebase); a1 = lut64k<0>(wg8, lanebase);
-        a2 = lut64k<1>(wg, lanebase); a3 = lut64k<1>(wg8, lanebase);
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint32_t wg = pick(ka[j], kb4[j], kk >> 1);
+        const uint32_t wg8 = pick(kc[j], kd[j], kk >> 1);
+        uint32_t a0, a1, a2, a3;
+        if (kk & 1) {
+          a0 = lut64k<2>(wg, lanebase); a1 = lut64k<2>(wg8, lanebase);
+          a2 = lut64k<3>(wg, lanebase); a3 = lut64k<3>(wg8, lanebase);
+        } else {
+          a0 = lut64k<0>(wg, lanebase); a1 = lut64k<0>(wg8, lanebase);
+          a2 = lut64k<1>(wg, lanebase); a3 = lut64k<1>(wg8, lanebase);
+        }
+        mma_16816(sc[j], a0, a1, a2, a3, qh[kk][0], qh[kk][1]);
+        mma_16816(sd[j], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
       }
-      mma_16816(sh[kk & 1], a0, a1, a2, a3, qh[kk][0], qh[kk][1]);
-      mma_16816(sl[kk & 1], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
     }
 
-    // ------------------------------------------------------------ in-warp online softmax
-    const float kn0 = __half2float(__ushort_as_half(ld_shared_u16(st + 4096 + 2 * g)));
-    const float kn8 = __half2float(__ushort_as_half(ld_shared_u16(st + 4096 + 2 * g + 16)));
-    const float vn0 = __half2float(__ushort_as_half(ld_shared_u16(st + 4128 + 2 * g))) * kQ1PScale;
-    const float vn8 = __half2float(__ushort_as_half(ld_shared_u16(st + 4128 + 2 * g + 16))) * kQ1PScale;
-    const bool p0 = c + g < pos_e, p8 = c + g + 8 < pos_e;
-    float s[4];
-    s[0] = (p0 && row_ok0) ? ((sh[0][0] + sh[1][0]) + (sl[0][0] + sl[1][0])) * kn0 : -INFINITY;
-    s[1] = (p0 && row_ok1) ? ((sh[0][1] + sh[1][1]) + (sl[0][1] + sl[1][1])) * kn0 : -INFINITY;
-    s[2] = (p8 && row_ok0) ? ((sh[0][2] + sh[1][2]) + (sl[0][2] + sl[1][2])) * kn8 : -INFINITY;
-    s[3] = (p8 && row_ok1) ? ((sh[0][3] + sh[1][3]) + (sl[0][3] + sl[1][3])) * kn8 : -INFINITY;
-    // scores in log2 units from here on
+    // ------------------------------------------------------------ online softmax over 32 positions
+    float s[2][4], kn[2][2], vn[2][2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) s[j] *= kLog2e;
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int pos = 16 * j + pk + 8 * e;
+        kn[j][e] = __half2float(__ushort_as_half(ld_shared_u16(nb + 2 * pos)));
+        vn[j][e] = __half2float(__ushort_as_half(ld_shared_u16(nb + 64 + 2 * pos))) * kQ1PScale;
+        const bool ok = c + pos < pos_e;
+        s[j][2 * e] = (ok && row_ok0) ? (sc[j][2 * e] + sd[j][2 * e]) * kn[j][e] * kLog2e : -INFINITY;
+        s[j][2 * e + 1] = (ok && row_ok1) ? (sc[j][2 * e + 1] + sd[j][2 * e + 1]) * kn[j][e] * kLog2e : -INFINITY;
+      }
     bool raise = false;
     float alpha[2] = {1.f, 1.f};
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float v = fmaxf(s[e], s[e + 2]);
+    for (int e = 0; e < 2; ++e) {   // e: row 2t+e
+      float v = fmaxf(fmaxf(s[0][e], s[0][e + 2]), fmaxf(s[1][e], s[1][e + 2]));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
       v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
@@ -274,11 +334,6 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
     }
     const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
     const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
-    float pr[4];
-    pr[0] = fast_exp2(s[0] - mu0);
-    pr[1] = fast_exp2(s[1] - mu1);
-    pr[2] = fast_exp2(s[2] - mu0);
-    pr[3] = fast_exp2(s[3] - mu1);
     if (__any_sync(0xffffffffu, raise)) {
       l_part[0] *= alpha[0];
       l_part[1] *= alpha[1];
@@ -290,61 +345,82 @@ __global__ void __launch_bounds__(kQ1Threads, 1) decode_q1_kernel(const DecodePa
         o[mt][3] *= alpha[1];
       }
     }
-    l_part[0] += pr[0] + pr[2];
-    l_part[1] += pr[1] + pr[3];
-    // P' = p * n_v / 256 (exp2(-inf) = 0 where masked; stale norms are multiplied by 0
-    // only if finite, so select), f16 hi + lo, transposed into B fragments
-    const float w0 = s[0] == -INFINITY ? 0.f : pr[0] * vn0;
-    const float w1 = s[1] == -INFINITY ? 0.f : pr[1] * vn0;
-    const float w2 = s[2] == -INFINITY ? 0.f : pr[2] * vn8;
-    const float w3 = s[3] == -INFINITY ? 0.f : pr[3] * vn8;
-    const __half2 h01 = __floats2half2_rn(w0, w1), h23 = __floats2half2_rn(w2, w3);
-    const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-    const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
-    const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
-    const uint32_t bh0 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
-    const uint32_t bh1 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-    const uint32_t bl0 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l01));
-    const uint32_t bl1 = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l23));
+    uint32_t bh[2][2], bl[2][2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float pw[4];
+      pw[0] = fast_exp2(s[j][0] - mu0);
+      pw[1] = fast_exp2(s[j][1] - mu1);
+      pw[2] = fast_exp2(s[j][2] - mu0);
+      pw[3] = fast_exp2(s[j][3] - mu1);
+      l_part[0] += pw[0] + pw[2];
+      l_part[1] += pw[1] + pw[3];
+      // P' = p * n_v / 256 (zero where masked, so stale norms never enter), f16 hi + lo,
+      // transposed into B fragments (k index = mma row = position sigma(row))
+      const float w0 = s[j][0] == -INFINITY ? 0.f : pw[0] * vn[j][0];
+      const float w1 = s[j][1] == -INFINITY ? 0.f : pw[1] * vn[j][0];
+      const float w2 = s[j][2] == -INFINITY ? 0.f : pw[2] * vn[j][1];
+      const float w3 = s[j][3] == -INFINITY ? 0.f : pw[3] * vn[j][1];
+      const __half2 h01 = __floats2half2_rn(w0, w1), h23 = __floats2half2_rn(w2, w3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
+      const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
+      bh[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
+      bh[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
+      bl[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l01));
+      bl[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l23));
+    }
 
-    // ------------------------------------------------------------ V phase (all 256 dims)
-    const uint4 x0 = ld_shared_v4(st + v_off0);             // words 4g..4g+3 of position 2t
-    const uint4 x1 = ld_shared_v4(st + v_off1);             // position 2t+1
-    const uint4 y0 = ld_shared_v4(st + v_off0 + 8 * 128);   // position 2t+8 (same swizzle)
-    const uint4 y1 = ld_shared_v4(st + v_off1 + 8 * 128);   // position 2t+9
+    // ------------------------------------------------------------ V phase (all 256 dims), two k-steps
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      uint32_t lo01, hi01, lo89, hi89;
-      interleave_nibbles(pick(x0, x0, q), pick(x1, x1, q), lo01, hi01);
-      interleave_nibbles(pick(y0, y0, q), pick(y1, y1, q), lo89, hi89);
+    for (int j = 0; j < 2; ++j) {
+      const uint32_t vrow = vst + j * 16 * 128;
+      const uint4 x0 = ld_shared_v4(vrow + v_off0);              // position sigma(2t)
+      const uint4 x1 = ld_shared_v4(vrow + v_off1);              // position sigma(2t+1)
+      const uint4 y0 = ld_shared_v4(vrow + 8 * 128 + v_off0);    // +8
+      const uint4 y1 = ld_shared_v4(vrow + 8 * 128 + v_off1);
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        uint32_t a0, a1, a2, a3;
-        switch (kb) {
-          case 0:
-            a0 = lut64k<0>(lo01, lanebase); a1 = lut64k<0>(hi01, lanebase);
-            a2 = lut64k<0>(lo89, lanebase); a3 = lut64k<0>(hi89, lanebase);
-            break;
-          case 1:
-            a0 = lut64k<1>(lo01, lanebase); a1 = lut64k<1>(hi01, lanebase);
-            a2 = lut64k<1>(lo89, lanebase); a3 = lut64k<1>(hi89, lanebase);
-            break;
-          case 2:
-            a0 = lut64k<2>(lo01, lanebase); a1 = lut64k<2>(hi01, lanebase);
-            a2 = lut64k<2>(lo89, lanebase); a3 = lut64k<2>(hi89, lanebase);
-            break;
-          default:
-            a0 = lut64k<3>(lo01, lanebase); a1 = lut64k<3>(hi01, lanebase);
-            a2 = lut64k<3>(lo89, lanebase); a3 = lut64k<3>(hi89, lanebase);
-            break;
+      for (int q = 0; q < 4; ++q) {
+        uint32_t lo01, hi01, lo89, hi89;
+        interleave_nibbles(pick(x0, x0, q), pick(x1, x1, q), lo01, hi01);
+        interleave_nibbles(pick(y0, y0, q), pick(y1, y1, q), lo89, hi89);
+#pragma unroll
+        for (int kb_ = 0; kb_ < 4; ++kb_) {
+          uint32_t a0, a1, a2, a3;
+          switch (kb_) {
+            case 0:
+              a0 = lut64k<0>(lo01, lanebase); a1 = lut64k<0>(hi01, lanebase);
+              a2 = lut64k<0>(lo89, lanebase); a3 = lut64k<0>(hi89, lanebase);
+              break;
+            case 1:
+              a0 = lut64k<1>(lo01, lanebase); a1 = lut64k<1>(hi01, lanebase);
+              a2 = lut64k<1>(lo89, lanebase); a3 = lut64k<1>(hi89, lanebase);
+              break;
+            case 2:
+              a0 = lut64k<2>(lo01, lanebase); a1 = lut64k<2>(hi01, lanebase);
+              a2 = lut64k<2>(lo89, lanebase); a3 = lut64k<2>(hi89, lanebase);
+              break;
+            default:
+              a0 = lut64k<3>(lo01, lanebase); a1 = lut64k<3>(hi01, lanebase);
+              a2 = lut64k<3>(lo89, lanebase); a3 = lut64k<3>(hi89, lanebase);
+              break;
+          }
+          mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bh[j][0], bh[j][1]);
+          mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bl[j][0], bl[j][1]);
         }
-        mma_16816(o[4 * q + kb], a0, a1, a2, a3, bh0, bh1);
-        mma_16816(o[4 * q + kb], a0, a1, a2, a3, bl0, bl1);
       }
     }
-    __syncwarp();   // all lanes are done with this slot before it is refilled
+    __syncwarp();   // all lanes are done with this buffer before lane 0 refills it
   }
-  cp_async_wait<0>();
+
+  // drain: a warp that broke out early still has at most one tile in flight; wait for it (bounded)
+  if (my_tiles > 0) {
+    const int last = my_tiles - 1;
+    const int b = w * kQ1Stages + (last % kQ1Stages);
+    uint32_t spins = 0;
+    while (!mbar_try_wait(base + kQ1BarOff + b * 8, (last / kQ1Stages) & 1) && ++spins < kQ1SpinLimit) {
+    }
+  }
 
   // ---------------------------------------------------------------- merge the 8 warp states
   // (m in natural-log units, so the combine pass sees the same units from every kernel)

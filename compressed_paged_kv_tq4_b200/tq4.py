@@ -22,6 +22,7 @@ TQ4_ERR_PAGE_RANGE = -3
 TQ4_ERR_CUDA = -4
 TQ4_ERR_WORKSPACE = -5
 TQ4_ERR_SEQ = -6
+TQ4_ERR_TIMEOUT = -7
 
 HEAD_DIM = 256
 PAGE_POSITIONS = 256
