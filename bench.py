@@ -62,6 +62,22 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# ---------------------------------------------------------------------------- replicas (host side)
+def max_over_ranks(ms, dist, device):
+    """Step time of the whole job: the slowest rank's (every rank calls this, in the same order)."""
+    if dist is None:
+        return float(ms)
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_step, world, ms):
+    """Whole-job throughput: units processed by all ranks over the slowest rank's step time."""
+    return units_per_step * world / (ms * 1e-3)
+
+
 # ---------------------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML in a thread."""
@@ -462,14 +478,10 @@ def main():
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1) / args.steps
-    if dist:
-        t = torch.tensor([ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, device)
     if S.ctx.status() != tq4.TQ4_OK:
         raise RuntimeError("device status error during timing")
-    value = S.units_per_step() * world / (ms * 1e-3)
+    value = job_value(S.units_per_step(), world, ms)
     if args.profile:
         if rank == 0:
             print(json.dumps({"profile": True, "workload": args.workload, "layers": w.layers, "ms_per_step": ms}))
@@ -519,7 +531,8 @@ def main():
             e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
-        e2e = {"value": S.units_per_step() * world / (e2e_ms * 1e-3), "unit": UNIT,
+        e2e_ms = max_over_ranks(e2e_ms, dist, device)
+        e2e = {"value": job_value(S.units_per_step(), world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
                "path": "pinned H2D of the step's queries and new K/V, replay of the captured public C-ABI "
                        "calls, D2H of every layer's output"}
@@ -558,6 +571,7 @@ def main():
     del graph, g2
     if dist:
         dist.barrier()
+        dist.destroy_process_group()
         dist.destroy_process_group()
 
 

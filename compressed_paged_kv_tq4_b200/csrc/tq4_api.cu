@@ -15,6 +15,7 @@
 #include "tq4_decode.cuh"
 #include "tq4_decode_q1.cuh"
 #include "tq4_prefill.cuh"
+#include "tq4_prefill_tc.cuh"
 
 struct tq4_ctx {
   int device;
@@ -177,7 +178,7 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   if (e == cudaSuccess) e = set_decode_attrs<1>();
   if (e == cudaSuccess) e = set_decode_attrs<2>();
   if (e == cudaSuccess) e = set_decode_attrs<3>();
-  if (e == cudaSuccess) e = tq4::prefill_set_attrs();
+  if (e == cudaSuccess) e = tq4::prefill_tc_set_attrs();
   if (e == cudaSuccess) e = cudaMalloc(&ctx->d_status, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(ctx->d_status, 0, sizeof(int));
   if (e != cudaSuccess) {
@@ -315,10 +316,9 @@ int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, con
   const size_t need = tq4::prefill_workspace_bytes(n_tok);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
   if (int rc = check_device(ctx)) return rc;
-  return cuda_status(tq4::launch_prefill(static_cast<const uint8_t*>(pool), num_pages, page_table,
-                                         prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, workspace,
-                                         ctx->signs, ctx->d_status, ctx->num_sms,
-                                         static_cast<cudaStream_t>(stream)));
+  return cuda_status(tq4::launch_prefill_tc(static_cast<const uint8_t*>(pool), num_pages, page_table,
+                                            prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, workspace,
+                                            ctx->signs, ctx->d_status, static_cast<cudaStream_t>(stream)));
 }
 
 int tq4_get_status(tq4_ctx* ctx, void* stream) {

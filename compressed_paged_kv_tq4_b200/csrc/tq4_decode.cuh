@@ -36,7 +36,6 @@ constexpr int kStages = 3;                   // cp.async ring depth
 constexpr int kQvStride = kD + 8;            // halves per Q' row in smem (bank-conflict pad)
 constexpr int kPsStride = kChunk + 8;        // halves per P' row in smem
 constexpr int kStageBytes = 2 * kChunk * 128 + 2 * kChunk * 2;   // K words, V words, K norms, V norms
-constexpr float kLog2e = 1.4426950408889634f;
 
 struct DecodeParams {
   const uint8_t* pool;

@@ -96,9 +96,6 @@ __device__ __forceinline__ uint32_t lut64k(uint32_t w, uint32_t lanebase) {
 }
 
 // ---- mbarrier and bulk-copy primitives (one CTA = its own cluster; no multicast)
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
-}
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes) : "memory");
 }

@@ -106,6 +106,13 @@ __device__ __forceinline__ uint32_t lut_decode(uint32_t lut_s, uint32_t w, uint3
   return ld_shared_u32(lut_s + __byte_perm(w, lane4, sel));
 }
 
+constexpr float kLog2e = 1.4426950408889634f;
+
+// mbarrier initialisation (shared::cta address)
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+
 // 2^x on the special-function unit (max relative error about 2^-22), used for
 // softmax weights; -inf maps to +0.
 __device__ __forceinline__ float fast_exp2(float x) {

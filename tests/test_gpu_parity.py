@@ -201,14 +201,19 @@ def test_decode_page_table_permutation_invariance():
     assert torch.equal(outs[0], outs[1])
 
 
-@pytest.mark.parametrize("prefix_len,n_tok", [(300, 70), (0, 5), (512, 64), (1, 1), (777, 130)])
-def test_prefill_parity(codebook, prefix_len, n_tok):
+# (prefix_len, n_tok, outlier_frac): one or several 128-row blocks per KV head with a
+# ragged last block; prefixes that end inside a 64-position tile and cross pages;
+# 5% x8 outlier norms, whose large scores raise the softmax reference mid-walk
+@pytest.mark.parametrize("prefix_len,n_tok,outliers", [(300, 70, 0.0), (0, 5, 0.0), (512, 64, 0.0), (1, 1, 0.0),
+                                                       (777, 130, 0.0), (1000, 200, 0.0), (600, 43, 0.05),
+                                                       (2048, 22, 0.05)])
+def test_prefill_parity(codebook, prefix_len, n_tok, outliers):
     c, _ = codebook
     signs = I.signs(4)
     ctx = tq4.Context(signs)
     npg = max(1, (prefix_len + 255) // 256)
     table = I.page_table_scattered(4, npg, npg + 2)
-    k, v = I.kv_vectors(4, 0, prefix_len)
+    k, v = I.kv_vectors(4, 0, prefix_len, outlier_frac=outliers)
     pool = tq4.Context.new_pool(npg + 2)
     tt = torch.from_numpy(table).cuda()
     if prefix_len:
@@ -223,7 +228,7 @@ def test_prefill_parity(codebook, prefix_len, n_tok):
     assert ctx.status() == tq4.TQ4_OK
     exp = O.prefill_attention(opool, table, prefix_len, I.bf16_bits_to_f32(qb), I.bf16_bits_to_f32(kb),
                               I.bf16_bits_to_f32(vb), SCALE, signs, c)
-    H.assert_bf16_close(out.float().cpu().numpy(), exp, f"prefill {prefix_len}+{n_tok}")
+    H.assert_bf16_close(out.float().cpu().numpy(), exp, f"prefill {prefix_len}+{n_tok} outliers {outliers}")
 
 
 # ------------------------------------------------------------------ failure paths (no GPU fault)

@@ -1,0 +1,62 @@
+"""Multi-GPU runs of bench.py are independent replicas (the path has no exchange
+step). What is shared between ranks is host logic: the whole job's step time is
+the slowest rank's, the value counts the units of every rank, and the reference
+arm runs on rank 0 only. These tests run that logic as two gloo ranks on the CPU."""
+import json
+import os
+import socket
+import sys
+import types
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = 2.0 + 3.0 * rank                      # rank 1 is the slow one
+        slowest = bench.max_over_ranks(ms, dist, torch.device("cpu"))
+        e2e = bench.max_over_ranks(10.0 - rank, dist, torch.device("cpu"))   # rank 0 is slow here
+        value = bench.job_value(1000, world, slowest)
+        with open(os.path.join(out_dir, f"rank{rank}.json"), "w") as f:
+            json.dump({"slowest": slowest, "e2e": e2e, "value": value}, f)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_agree_on_the_slowest_rank(tmp_path):
+    world = 2
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    res = [json.load(open(tmp_path / f"rank{r}.json")) for r in range(world)]
+    for r in res:
+        assert r["slowest"] == 5.0          # max over ranks, seen identically by every rank
+        assert r["e2e"] == 10.0
+        assert r["value"] == pytest.approx(1000 * 2 / 5e-3)   # all ranks' units over the slowest time
+
+
+def test_single_process_needs_no_collective():
+    assert bench.max_over_ranks(3.5, None, None) == 3.5
+    assert bench.job_value(10, 1, 2.0) == pytest.approx(5000.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    args = types.SimpleNamespace(workload="decode_32k", steps=1, warmup=0, gpus=2)
+    bench.run_reference(args, rank=1)      # returns before building anything
+    assert capsys.readouterr().out == ""
