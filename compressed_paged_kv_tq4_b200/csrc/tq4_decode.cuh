@@ -122,12 +122,6 @@ __device__ __forceinline__ uint32_t pick(const uint4& a, const uint4& b, int i) 
 // (one word of positions 2t / 2t+1 per lane group) both hit 32 distinct banks.
 __device__ __forceinline__ int seg_swz(int pos) { return (((pos >> 1) & 3) << 1) ^ ((pos & 1) << 2); }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }

@@ -108,6 +108,14 @@ __device__ __forceinline__ uint32_t lut_decode(uint32_t lut_s, uint32_t w, uint3
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// 16-byte global -> shared copies that bypass registers (generic proxy; wait before use)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 // mbarrier initialisation (shared::cta address)
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");

@@ -24,8 +24,9 @@
 //               centroid table (32 KiB: row = one byte of indices, one 4-byte slot
 //               per lane) into f16 panels [4 dim blocks][64 positions][128 B]
 //               with the 128-byte swizzle; the chunk's own K/V are copied.
-//   warp 12     one thread issues tcgen05.mma: S = Q'hi K^T + Q'lo K^T (A = Q'hi in
-//               TMEM, then A = Q'lo in shared memory; B = K panels, K-major) and
+//   warp 12     one thread issues tcgen05.mma: S = Q'hi K^T (+ Q'lo K^T where the
+//               tile needs it; A = Q'hi in TMEM, A = Q'lo in shared memory; B = K
+//               panels, K-major) and
 //               O += P V (A = P in TMEM, B = V panels, MN-major), in the order
 //               QK(j), PV(j-1), so the tensor pipe holds the next score tile while
 //               the softmax runs.
@@ -59,7 +60,7 @@ constexpr uint32_t kTcQloOff = 2 * kTcStage;             // q' lo panels [4][128
 constexpr uint32_t kTcLutOff = kTcQloOff + 4 * kTcQloPanel;   // 32 KiB per-lane centroid table
 constexpr uint32_t kTcNormOff = kTcLutOff + kTcLutBytes; // [2 stages][K 64, V 64] fp32
 constexpr uint32_t kTcBarOff = kTcNormOff + 2 * 2 * kTcTile * 4;
-constexpr uint32_t kTcMiscOff = kTcBarOff + 128;
+constexpr uint32_t kTcMiscOff = kTcBarOff + 128;   // u32 [0] TMEM base, [1] abort; f32 [8 + 4 stage + warp] K norm max
 constexpr uint32_t kTcSmem = kTcMiscOff + 128 + 1024;    // + alignment slack
 constexpr int kTcOsStride = kD + 4;                      // epilogue rows (fp32), reuse the stages + q' lo
 static_assert(uint32_t(kTcRows * kTcOsStride * 4) <= kTcLutOff, "epilogue rows overlap the table");
@@ -70,6 +71,12 @@ static_assert(kTcGroupThreads * kTcUnits == 2 * kTcTile * 8, "units cover K and 
 constexpr uint32_t kTcSpin = 1u << 24;
 constexpr float kTcPScale = 1.0f / 256.0f;   // P carries 1/256, undone in the epilogue
 constexpr float kTcLazy = 8.0f;              // raise the row reference only when the max grows by > 2^8
+// The q' lo correction (Q'lo K^T) runs for a tile when it holds chunk positions or
+// a prefix key whose norm exceeds kTcLoNorm. Below it, the error the f16 q' puts
+// in a score is about 2.5e-5 * ||k|| in log2 units (std over the rounding), far
+// below what moves a bf16 output by the tolerance; the workloads' keys have norms
+// 16 s with s in [0.5, 2] (up to ~34), their 8x outliers start at 64.
+constexpr float kTcLoNorm = 48.0f;
 
 // TMEM columns
 constexpr uint32_t kTmQ = 0, kTmS0 = 128, kTmO = 256;
@@ -144,6 +151,13 @@ __device__ __forceinline__ void tm_st32(uint32_t taddr, const uint32_t (&r)[32])
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
       "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
       "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+__device__ __forceinline__ void tm_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
 __device__ __forceinline__ void tm_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
@@ -340,18 +354,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         }
       }
       l_sum += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      uint32_t pk[32];
+      // P hi (columns 0-31: positions 2k, 2k+1 in column k) and P lo = P - f16(P)
+      // (columns 32-63), written over the scores in halves of 32 positions
 #pragma unroll
-      for (int k = 0; k < 32; ++k)   // P hi: positions 2k, 2k+1
-        pk[k] = pack_half2(__uint_as_float(sr[k >> 4][(2 * k) & 31]), __uint_as_float(sr[k >> 4][(2 * k + 1) & 31]));
-      tm_st32(lane_addr + kTmS0 + 64 * b, pk);
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {   // P lo = P - f16(P)
-        const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
-        pk[k] = pack_half2(__uint_as_float(sr[k >> 4][(2 * k) & 31]) - hi.x,
-                           __uint_as_float(sr[k >> 4][(2 * k + 1) & 31]) - hi.y);
+        for (int k = 0; k < 16; ++k) pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]), __uint_as_float(sr[c][2 * k + 1]));
+        tm_st16(lane_addr + kTmS0 + 64 * b + 16 * c, pk);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
+          pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]) - hi.x, __uint_as_float(sr[c][2 * k + 1]) - hi.y);
+        }
+        tm_st16(lane_addr + kTmS0 + 64 * b + 32 + 16 * c, pk);
       }
-      tm_st32(lane_addr + kTmS0 + 64 * b + 32, pk);
       tm_wait_st();
       tc_fence_before();
       mbar_arrive(bar_p_full + 8 * b);
@@ -418,48 +435,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         }
       }
     };
-    // expand unit u of tile j into the stage; returns the unit's pre-scaled norm
+    // expand unit u of tile j into the stage: centroid values for a prefix position,
+    // an asynchronous copy of the prologue's f16 row for a chunk position, zeros past
+    // the CTA's last visible position. Returns the unit's norm (1 for chunk rows: the
+    // rotated row carries its own length; 0 past the end).
     auto expand = [&](int j, int u) -> float {
       const int q = (gt >> 5) + 4 * u;
       const int kv = q >> 4, pl = 4 * (q & 15) + pl_lo, pos = j * kTcTile + pl;
-      uint32_t out[16];   // dims 32 grp .. 32 grp + 31 as f16 pairs
-      float nrm;
+      // dims 32 grp .. +31 = panel grp / 2, 16-B chunks 4 (grp & 1) .. +3 of row pl, 128-byte swizzle
+      uint8_t* prow = st + kv * kTcKV + (grp >> 1) * kTcPanel + pl * 128;
+      const int sw = pl & 7, c0 = (grp & 1) * 4;
       if (pos < prefix_end) {
         const uint32_t ww[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          out[4 * k + 0] = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[k], lane8, 0x5504u) >> 1));
-          out[4 * k + 1] = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[k], lane8, 0x5514u) >> 1));
-          out[4 * k + 2] = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[k], lane8, 0x5524u) >> 1));
-          out[4 * k + 3] = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[k], lane8, 0x5534u) >> 1));
+        for (int c = 0; c < 4; ++c) {   // word c = dims 8c .. 8c + 7 of the span
+          const uint32_t a = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5504u) >> 1));
+          const uint32_t b = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5514u) >> 1));
+          const uint32_t d = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5524u) >> 1));
+          const uint32_t e = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5534u) >> 1));
+          *reinterpret_cast<uint4*>(prow + (((c0 + c) ^ sw) << 4)) = make_uint4(a, b, d, e);
         }
-        nrm = rawn[u];
-      } else if (pos < kv_end) {   // the chunk's own rotated K/V (f16)
-        const uint4* src = reinterpret_cast<const uint4*>((kv ? p.vr : p.kr) +
-                                                          (int64_t(pos - p.prefix_len) * kHkv + h) * kD + 32 * grp);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 v4 = __ldg(src + k);
-          out[4 * k] = v4.x;
-          out[4 * k + 1] = v4.y;
-          out[4 * k + 2] = v4.z;
-          out[4 * k + 3] = v4.w;
-        }
-        nrm = 1.f;
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) out[k] = 0u;
-        nrm = 0.f;
+        return rawn[u];
       }
-      // dims 32 grp .. +31 = panel grp / 2, 16-B chunks 4 (grp & 1) .. +3 of row pl, 128-byte swizzle
-      uint8_t* prow = st + kv * kTcKV + (grp >> 1) * kTcPanel + pl * 128;
+      if (pos < kv_end) {
+        const __half* src = (kv ? p.vr : p.kr) + (int64_t(pos - p.prefix_len) * kHkv + h) * kD + 32 * grp;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int chunk = ((grp & 1) * 4 + c) ^ (pl & 7);
-        *reinterpret_cast<uint4*>(prow + chunk * 16) =
-            make_uint4(out[4 * c], out[4 * c + 1], out[4 * c + 2], out[4 * c + 3]);
+        for (int c = 0; c < 4; ++c) cp_async16(smem_u32(prow + (((c0 + c) ^ sw) << 4)), src + 8 * c);
+        return 1.f;
       }
-      return nrm * (kv ? kTcPScale : kLog2e);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(prow + (((c0 + c) ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
+      return 0.f;
     };
     int32_t pg_next = 0;   // page of tile j + 2
     if (grp_id < n_tiles) {
@@ -468,30 +474,49 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
 #pragma unroll
       for (int u = 0; u < kTcUnits; ++u) fetch(grp_id, u, pg0);
     }
+    volatile float* kmax = reinterpret_cast<volatile float*>(misc) + 8 + 4 * grp_id;
     for (int j = grp_id; j < n_tiles; j += 2) {
       const int32_t pg_far = page_of(j + 4);
       const bool more = j + 2 < n_tiles;
-      float kn_keep[4];
+      const bool chunk_rows = (j + 1) * kTcTile > prefix_end;   // this tile reaches the chunk (or past it)
+      float kn[4];
       // ---- K half: free once QK(j - 2) has run
       if (j >= 2 && !bounded_wait(bar_k_empty + 8 * grp_id, ((j >> 1) - 1) & 1)) break;
+      float big = chunk_rows ? INFINITY : 0.f;   // largest K norm; chunk rows always take the q' lo pass
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        kn_keep[u] = expand(j, u);
-        if (more) fetch(j + 2, u, pg_next);
+        kn[u] = expand(j, u);
+        big = fmaxf(big, kn[u]);
       }
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic-proxy stores -> tensor-core reads
+      // chunk-row copies complete before the next tile's loads are issued (the wait
+      // would otherwise also cover those)
+      cp_async_commit();
+      cp_async_wait<0>();
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fetch(j + 2, u, pg_next);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) big = fmaxf(big, __shfl_xor_sync(0xffffffffu, big, o));
+      if (lane == 0) kmax[(w - kTcSoftWarps) & 3] = big;   // read by the MMA thread after k_full
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic-proxy writes -> tensor-core reads
       mbar_arrive(bar_k_full + 8 * grp_id);
-      // ---- V half (and both norms): free once PV(j - 2) has run
+      // ---- V half and both norms: free once PV(j - 2) has run
       if (j >= 2 && !bounded_wait(bar_v_empty + 8 * grp_id, ((j >> 1) - 1) & 1)) break;
 #pragma unroll
       for (int u = 4; u < 8; ++u) {
         const float vn = expand(j, u);
-        if (more) fetch(j + 2, u, pg_next);
         if (grp == 0) {
           const int pl = 4 * (((gt >> 5) + 4 * u) & 15) + pl_lo;
-          nb[pl] = kn_keep[u - 4];
-          nb[kTcTile + pl] = vn;
+          nb[pl] = kn[u - 4] * kLog2e;
+          nb[kTcTile + pl] = vn * kTcPScale;
         }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      if (more) {
+#pragma unroll
+        for (int u = 4; u < 8; ++u) fetch(j + 2, u, pg_next);
       }
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       mbar_arrive(bar_v_full + 8 * grp_id);
@@ -515,11 +540,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
             const uint64_t bd = tc_sdesc(kbase + (kk >> 2) * kTcPanel + (kk & 3) * 32, 16, 1024);
             tc_mma(tmem + kTmS0 + 64 * b, tmem + kTmQ + 8 * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
           }
+          const volatile float* km = reinterpret_cast<const volatile float*>(misc) + 8 + 4 * b;
+          if (fmaxf(fmaxf(km[0], km[1]), fmaxf(km[2], km[3])) > kTcLoNorm) {
 #pragma unroll
-          for (int kk = 0; kk < 16; ++kk) {
-            const uint64_t ad = tc_sdesc(sbase + kTcQloOff + (kk >> 2) * kTcQloPanel + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = tc_sdesc(kbase + (kk >> 2) * kTcPanel + (kk & 3) * 32, 16, 1024);
-            tc_mma_ss(tmem + kTmS0 + 64 * b, ad, bd, idesc_qk, 1u);
+            for (int kk = 0; kk < 16; ++kk) {
+              const uint64_t ad = tc_sdesc(sbase + kTcQloOff + (kk >> 2) * kTcQloPanel + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = tc_sdesc(kbase + (kk >> 2) * kTcPanel + (kk & 3) * 32, 16, 1024);
+              tc_mma_ss(tmem + kTmS0 + 64 * b, ad, bd, idesc_qk, 1u);
+            }
           }
           tc_commit(bar_s_full + 8 * b);
           tc_commit(bar_k_empty + 8 * b);

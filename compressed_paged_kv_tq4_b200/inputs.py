@@ -29,7 +29,7 @@ H_Q = 24
 POOL_PAGES = 229_376 // PAGE  # 896 pages
 
 # purposes (second SeedSequence word)
-_SIGNS, _KV, _OUTLIER, _Q, _TABLE, _NEWKV, _CHUNK = range(7)
+_SIGNS, _KV, _OUTLIER, _Q, _TABLE, _NEWKV, _CHUNK, _CODES, _NORMS = range(9)
 
 
 def _rng(config: int, purpose: int, layer: int = 0) -> np.random.Generator:
@@ -105,6 +105,24 @@ def chunk_kv(config: int, layer: int, n_tok: int):
     k = r.standard_normal((n_tok, H_KV, D), dtype=np.float32)
     v = r.standard_normal((n_tok, H_KV, D), dtype=np.float32)
     return to_bf16_bits(k), to_bf16_bits(v)
+
+
+def random_codes(config: int, layer: int, n_words: int) -> np.ndarray:
+    """n_words uniformly random uint32 words: every 4-bit field is uniform over 0..15."""
+    r = _rng(config, _CODES, layer)
+    return r.integers(0, 2 ** 32, size=n_words, dtype=np.uint64).astype(np.uint32)
+
+
+def random_norms(config: int, layer: int, n: int, *, outlier_frac: float = 0.0,
+                 outlier_scale: float = 8.0) -> np.ndarray:
+    """n positive fp32 magnitudes 16 s, s ~ U(0.5, 2) (the length of a 256-dim
+    N(0, s^2 I) vector is about 16 s); a seeded ``outlier_frac`` of them times
+    ``outlier_scale``. The scale mix of ``kv_vectors``, without the vectors."""
+    r = _rng(config, _NORMS, layer)
+    s = r.uniform(0.5, 2.0, size=n)
+    if outlier_frac > 0.0:
+        s[r.random(n) < outlier_frac] *= outlier_scale
+    return (16.0 * s).astype(np.float32)
 
 
 def page_table_scattered(config: int, n_pages: int, pool_pages: int = POOL_PAGES,
