@@ -62,6 +62,34 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+# ---------------------------------------------------------------------------- measured DRAM traffic
+# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
+# (summarised under profiles/), per unit of work. A figure counts only while the
+# kernel's source file hashes to the value it had when the counters were taken.
+MEASURED_TRAFFIC = {
+    # decode_q1_kernel, decode_32k capture: 34,146,048 B read + 74,240 B written for
+    # 32,768 positions; the kernel's traffic grows with the positions it streams
+    "decode_q1": ("tq4_decode_q1.cuh", "800114719a0281f06ec035d23001165314f238f5bc629e438f4f6a92f42810a3",
+                  (34_146_048 + 74_240) / 32_768),
+}
+
+
+def measured_traffic(key, units):
+    """Bytes per launch for ``units`` units of work, or None if the kernel changed since the capture."""
+    if key not in MEASURED_TRAFFIC:
+        return None
+    import hashlib
+    fname, digest, per_unit = MEASURED_TRAFFIC[key]
+    path = os.path.join(ROOT, "compressed_paged_kv_tq4_b200", "csrc", fname)
+    try:
+        with open(path, "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    except OSError:
+        return None
+    return per_unit * units
+
+
 # ---------------------------------------------------------------------------- replicas (host side)
 def max_over_ranks(ms, dist, device):
     """Step time of the whole job: the slowest rank's (every rank calls this, in the same order)."""
@@ -508,7 +536,8 @@ def main():
     if w.kind == "decode":
         ach = S.dominant_bytes() / (att_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": None, "kernel": "tq4_decode_attention (split-K kernel + combine)",
+                "traffic": measured_traffic("decode_q1", S.total) if w.n_q == 1 else None,
+                "kernel": "tq4_decode_attention (split-K kernel + combine)",
                 "launch_ms": att_ms, "peak_source": f"{peak_kind} hbm_gbs"}
     else:
         ach = S.dominant_flops() / (att_ms * 1e-3) / 1e12
