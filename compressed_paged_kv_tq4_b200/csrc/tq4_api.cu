@@ -278,21 +278,27 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, cons
   p.status = ctx->d_status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
+  cudaError_t e;
   switch (tq4::decode_nt(n_q)) {
     case 1: {
       CUtensorMap map;
       if (int rc = pool_tensor_map(pool, num_pages, &map)) return rc;
-      tq4::decode_q1_kernel<<<grid, tq4::kQ1Threads, tq4::decode_q1_smem_bytes(), st>>>(p, map);
+      e = tq4::launch_pdl(tq4::decode_q1_kernel, grid, dim3(tq4::kQ1Threads), tq4::decode_q1_smem_bytes(), st, p,
+                          map);
       break;
     }
-    case 2: tq4::decode_splitk_kernel<2><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<2>(), st>>>(p); break;
-    default: tq4::decode_splitk_kernel<3><<<grid, tq4::kDecThreads, tq4::decode_smem_bytes<3>(), st>>>(p); break;
+    case 2:
+      e = tq4::launch_pdl(tq4::decode_splitk_kernel<2>, grid, dim3(tq4::kDecThreads), tq4::decode_smem_bytes<2>(),
+                          st, p);
+      break;
+    default:
+      e = tq4::launch_pdl(tq4::decode_splitk_kernel<3>, grid, dim3(tq4::kDecThreads), tq4::decode_smem_bytes<3>(),
+                          st, p);
+      break;
   }
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return TQ4_ERR_CUDA;
   const int rows = n_req * n_q * tq4::kHq;
-  tq4::decode_combine_kernel<<<rows, 32 * tq4::kCombWarps, 0, st>>>(p);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(tq4::launch_pdl(tq4::decode_combine_kernel, dim3(rows), dim3(32 * tq4::kCombWarps), 0, st, p));
 }
 
 size_t tq4_prefill_workspace_bytes(int32_t n_tok) {

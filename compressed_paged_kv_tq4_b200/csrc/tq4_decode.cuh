@@ -143,6 +143,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   const int h = blockIdx.y;
   const uint32_t lane4 = uint32_t(lane) * 4u;
 
+  pdl_wait();   // every read of the call's inputs comes after the previous kernel
+  pdl_launch_dependents();
   if (w == 0) {
     int req = 0, split = 0, total = 0;
     const bool ok = find_item(p, blockIdx.x, req, split, total);
@@ -545,6 +547,8 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const D
   __shared__ int s_first;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row_id = blockIdx.x;
+  pdl_wait();   // the split partials come from the previous kernel
+  pdl_launch_dependents();
   const int qh = row_id % kHq;
   const int tok = (row_id / kHq) % p.n_q;
   const int r = row_id / (kHq * p.n_q);

@@ -142,6 +142,16 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   auto buf_addr = [&](int b) { return b < kQ1LowBufs ? low0 + b * kQ1Buf : kQ1Hi + (b - kQ1LowBufs) * kQ1Buf; };
   const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 4u);
 
+  // prologue that reads none of the call's inputs (overlaps the previous kernel)
+  if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  for (int e = tid; e < 256 * 32; e += kQ1Threads) {
+    const int b = e >> 5, l = e & 31;
+    st_shared_u32(kQ1Lut + b * 256 + l * 4,
+                  uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16));
+  }
+  pdl_wait();
+  pdl_launch_dependents();
   if (w == 0) {
     int req = 0, split = 0, total = 0;
     const bool ok = find_item(p, blockIdx.x, req, split, total);
@@ -151,8 +161,6 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       if (blockIdx.x == 0 && h == 0 && total > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
     }
   }
-  if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
-  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   __syncthreads();
   const int r = s_item[0];
   if (r < 0 || int(blockIdx.x) >= p.items_ub) return;
@@ -219,11 +227,6 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       *reinterpret_cast<__half2*>(qv_hi + row * kQvStride + col) = hi;
       *reinterpret_cast<__half2*>(qv_lo + row * kQvStride + col) = __floats2half2_rn(v[i] - hfl.x, v[i + 1] - hfl.y);
     }
-  }
-  for (int e = tid; e < 256 * 32; e += kQ1Threads) {
-    const int b = e >> 5, l = e & 31;
-    st_shared_u32(kQ1Lut + b * 256 + l * 4,
-                  uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16));
   }
   __syncthreads();
 

@@ -45,6 +45,8 @@ __global__ void __launch_bounds__(256) encode_append_kernel(
     Signs signs, int* status) {
   const int lane = threadIdx.x & 31;
   const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();   // inputs and the pool may come from the previous kernel
+  pdl_launch_dependents();
   if (vec >= int64_t(n_tok) * 2 * kHkv) return;
   const int tok = int(vec / (2 * kHkv));
   const int kv = int(vec / kHkv) & 1;       // 0 = K, 1 = V
@@ -103,6 +105,8 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
   if (vec >= int64_t(n) * 2 * kHkv) return;
   const int tok = int(vec / (2 * kHkv));
   const int kv = int(vec / kHkv) & 1;
@@ -141,14 +145,12 @@ cudaError_t launch_encode_append(uint8_t* pool, int32_t num_pages, const int32_t
   const int64_t vecs = int64_t(n_tok) * 2 * kHkv;
   const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
   if (dtype == TQ4_DTYPE_F32)
-    encode_append_kernel<float><<<blocks, threads, 0, stream>>>(
-        pool, num_pages, page_table, start_pos, n_tok, static_cast<const float*>(k_new),
-        static_cast<const float*>(v_new), signs, status);
-  else
-    encode_append_kernel<uint16_t><<<blocks, threads, 0, stream>>>(
-        pool, num_pages, page_table, start_pos, n_tok, static_cast<const uint16_t*>(k_new),
-        static_cast<const uint16_t*>(v_new), signs, status);
-  return cudaGetLastError();
+    return launch_pdl(encode_append_kernel<float>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                      page_table, start_pos, n_tok, static_cast<const float*>(k_new),
+                      static_cast<const float*>(v_new), signs, status);
+  return launch_pdl(encode_append_kernel<uint16_t>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                    page_table, start_pos, n_tok, static_cast<const uint16_t*>(k_new),
+                    static_cast<const uint16_t*>(v_new), signs, status);
 }
 
 cudaError_t launch_reconstruct(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,
@@ -157,9 +159,8 @@ cudaError_t launch_reconstruct(const uint8_t* pool, int32_t num_pages, const int
   const int threads = 256, wpb = threads / 32;
   const int64_t vecs = int64_t(n) * 2 * kHkv;
   const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
-  reconstruct_kernel<<<blocks, threads, 0, stream>>>(pool, num_pages, page_table, start, n, k_out,
-                                                      v_out, signs, status);
-  return cudaGetLastError();
+  return launch_pdl(reconstruct_kernel, dim3(blocks), dim3(threads), 0, stream, pool, num_pages, page_table, start,
+                    n, k_out, v_out, signs, status);
 }
 
 }  // namespace tq4

@@ -39,6 +39,8 @@ __global__ void __launch_bounds__(256) prefill_rotate_kernel(
   const int lane = threadIdx.x & 31;
   const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int64_t nq = int64_t(n_tok) * kHq, nk = int64_t(n_tok) * kHkv;
+  pdl_wait();   // inputs may come from the previous kernel
+  pdl_launch_dependents();
   if (vec >= nq + 2 * nk) return;
   const uint16_t* src;
   __half* dst;

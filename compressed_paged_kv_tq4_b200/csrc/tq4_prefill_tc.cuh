@@ -217,6 +217,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     reinterpret_cast<uint32_t*>(smem + kTcLutOff)[b * 32 + l] =
         uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16);
   }
+  pdl_wait();   // q', the chunk rows and the pool may come from the previous kernels
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -628,9 +630,8 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
   __half* kr = qlo + size_t(n_tok) * kHq * kD;
   __half* vr = kr + size_t(n_tok) * kHkv * kD;
   const int64_t vecs = int64_t(n_tok) * (kHq + 2 * kHkv);
-  prefill_rotate_kernel<<<unsigned((vecs + 7) / 8), 256, 0, stream>>>(q, kc, vc, n_tok, scale, qr, qlo, kr,
-                                                                        vr, signs);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(prefill_rotate_kernel, dim3(unsigned((vecs + 7) / 8)), dim3(256), 0, stream, q, kc, vc,
+                             n_tok, scale, qr, qlo, kr, vr, signs);
   if (e != cudaSuccess) return e;
   PrefillParams p{};
   p.pool = pool;
@@ -646,8 +647,7 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
   p.signs = signs;
   p.status = status;
   const dim3 grid(unsigned((6 * n_tok + kTcRows - 1) / kTcRows), kHkv);
-  prefill_tc_kernel<<<grid, kTcThreads, kTcSmem, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(prefill_tc_kernel, grid, dim3(kTcThreads), size_t(kTcSmem), stream, p);
 }
 
 }  // namespace tq4
