@@ -45,7 +45,11 @@ constexpr uint32_t kQ1NrmOff = kQ1BarOff + 128;                        // 16 x 1
 constexpr uint32_t kQ1CtlBytes = kQ1NrmOff + kQ1Bufs * 128;           // 10,752
 constexpr int kQ1LowBufs = 6;
 constexpr uint32_t kQ1DynBytes = kQ1Hi + (kQ1Bufs - kQ1LowBufs) * kQ1Buf;   // 212,992
-constexpr int kQ1MergeBytes = kQ1Warps * (8 * kD + 16) * 4;
+// merge area, per warp: 8 rows of o' with each 32-dim block padded to 36 floats and
+// rows 292 floats apart (conflict-free float4 stores of the mma fragments and reads
+// of row slices), then m[8], l[8]
+constexpr int kQ1MrgBlk = 36, kQ1MrgRow = 8 * kQ1MrgBlk + 4, kQ1MrgWarp = 8 * kQ1MrgRow + 16;
+constexpr int kQ1MergeBytes = kQ1Warps * kQ1MrgWarp * 4;
 static_assert(kQ1MergeBytes <= (kQ1Bufs - kQ1LowBufs) * kQ1Buf, "merge area fits above the table");
 static_assert(kQ1DynBytes <= 227 * 1024, "fits the per-CTA shared memory");
 constexpr float kQ1PScale = 1.0f / 256.0f;   // P' = p * n_v / 256 (undone when the partial is written)
@@ -145,32 +149,51 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   // prologue that reads none of the call's inputs (overlaps the previous kernel)
   if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  for (int e = tid; e < 256 * 32; e += kQ1Threads) {
-    const int b = e >> 5, l = e & 31;
-    st_shared_u32(kQ1Lut + b * 256 + l * 4,
-                  uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16));
+  {   // table rows through shuffles: lane l holds c[l & 15]
+    const uint32_t cl = g_codebook.c16[lane & 15];
+    for (int b = w; b < 256; b += kQ1Warps) {
+      const uint32_t lo = __shfl_sync(0xffffffffu, cl, b & 15), hi = __shfl_sync(0xffffffffu, cl, b >> 4);
+      st_shared_u32(kQ1Lut + b * 256 + lane * 4, lo | (hi << 16));
+    }
   }
   pdl_wait();
   pdl_launch_dependents();
-  if (w == 0) {
-    int req = 0, split = 0, total = 0;
-    const bool ok = find_item(p, blockIdx.x, req, split, total);
-    if (lane == 0) {
-      s_item[0] = ok ? req : -1;
-      s_item[1] = split;
-      if (blockIdx.x == 0 && h == 0 && total > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
+  // (request, split) of this CTA: with one request it is (0, blockIdx.x); otherwise
+  // warp 0 scans the lengths
+  int r = 0, split = int(blockIdx.x);
+  if (p.n_req > 1) {
+    if (w == 0) {
+      int req = 0, sp = 0, total = 0;
+      const bool ok = find_item(p, blockIdx.x, req, sp, total);
+      if (lane == 0) {
+        s_item[0] = ok ? req : -1;
+        s_item[1] = sp;
+        if (blockIdx.x == 0 && h == 0 && total > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
+      }
     }
+    __syncthreads();
+    r = s_item[0];
+    split = s_item[1];
+    if (r < 0 || int(blockIdx.x) >= p.items_ub) return;
   }
-  __syncthreads();
-  const int r = s_item[0];
-  if (r < 0 || int(blockIdx.x) >= p.items_ub) return;
-  const int split = s_item[1];
-  const int seq_len = __ldg(p.seq_lens + r);
+  const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
   const int pos_b = split * p.split_len;
+  // independent loads go out together: the length, this warp's first page id
+  // (speculative, inside the table) and this warp's query row
+  const int seq_len = __ldg(p.seq_lens + r);
+  const int c_first = pos_b + w * kQ1Tile;
+  const int32_t page_first = (c_first >> 8) < p.max_pages ? __ldg(table + (c_first >> 8)) : -1;
+  uint4 qraw = make_uint4(0, 0, 0, 0);
+  if (w < kGroup)
+    qraw = __ldg(reinterpret_cast<const uint4*>(p.q + (int64_t(r) * kHq + h * kGroup + w) * kD + lane * 8));
+  if (p.n_req == 1) {
+    const int S = seq_ok(seq_len, p.n_q, p.max_pages) ? (seq_len + p.split_len - 1) / p.split_len : 0;
+    if (tid == 0 && blockIdx.x == 0 && h == 0 && S > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
+    if (split >= S || split >= p.items_ub) return;   // the same decision in every thread of the CTA
+  }
   const int pos_e = min(pos_b + p.split_len, seq_len);
   const int n_tiles = (pos_e - pos_b + kQ1Tile - 1) / kQ1Tile;
   const int my_tiles = n_tiles > w ? (n_tiles - w + kQ1Warps - 1) / kQ1Warps : 0;
-  const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
 
   // ---- lane 0 of each warp streams the warp's tiles: tile w + 8k -> buffer w*2 + k%2
   auto tile_pos = [&](int k) { return pos_b + (w + k * kQ1Warps) * kQ1Tile; };
@@ -179,7 +202,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       const int c = tile_pos(k);
       const int b = w * kQ1Stages + (k % kQ1Stages);
       const uint32_t bar = base + kQ1BarOff + b * 8;
-      int page = __ldg(table + (c >> 8));
+      int page = k == 0 ? page_first : __ldg(table + (c >> 8));
       if (page < 0 || page >= p.num_pages) {
         record_error(p.status, TQ4_ERR_PAGE_RANGE);
         page = 0;   // still complete the barrier (reading page 0); the tile is masked below
@@ -202,9 +225,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     const int row = w;
     float v[8];
     if (row < 6) {
-      const uint16_t* src = p.q + (int64_t(r) * kHq + h * kGroup + row) * kD + lane * 8;
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
-      const uint32_t ww[4] = {raw.x, raw.y, raw.z, raw.w};
+      const uint32_t ww[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         v[2 * i] = __uint_as_float(ww[i] << 16) * sign_of(p.signs, lane * 8 + 2 * i);
@@ -426,7 +447,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   // (m in natural-log units, so the combine pass sees the same units from every kernel)
   __syncthreads();
   float* mrg = reinterpret_cast<float*>(smem + (kQ1Hi - base));   // per warp: o'[8 rows][256], m[8], l[8]
-  float* mine = mrg + w * (8 * kD + 16);
+  float* mine = mrg + w * kQ1MrgWarp;
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     float lv = l_part[e];
@@ -435,12 +456,12 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     lv += __shfl_xor_sync(0xffffffffu, lv, 16);
     const int row = 2 * t + e;
     if (g == 0) {
-      mine[8 * kD + row] = m_ref[e] == -INFINITY ? -INFINITY : m_ref[e] / kLog2e;
-      mine[8 * kD + 8 + row] = lv;
+      mine[8 * kQ1MrgRow + row] = m_ref[e] == -INFINITY ? -INFINITY : m_ref[e] / kLog2e;
+      mine[8 * kQ1MrgRow + 8 + row] = lv;
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {   // dims 32g + 8q + 0..7 of row 2t+e
-      float* d = mine + row * kD + 32 * g + 8 * q;
+      float* d = mine + row * kQ1MrgRow + g * kQ1MrgBlk + 8 * q;
       reinterpret_cast<float4*>(d)[0] =
           make_float4(o[4 * q][e], o[4 * q][e + 2], o[4 * q + 1][e], o[4 * q + 1][e + 2]);
       reinterpret_cast<float4*>(d)[1] =
@@ -452,18 +473,19 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     const int row = tid >> 5, d0 = (tid & 31) * 8;   // 8 rows x 32 lanes x 8 dims
     float M = -INFINITY;
 #pragma unroll
-    for (int ww = 0; ww < kQ1Warps; ++ww) M = fmaxf(M, mrg[ww * (8 * kD + 16) + 8 * kD + row]);
+    for (int ww = 0; ww < kQ1Warps; ++ww) M = fmaxf(M, mrg[ww * kQ1MrgWarp + 8 * kQ1MrgRow + row]);
     float L = 0.f, acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int ww = 0; ww < kQ1Warps; ++ww) {
-        const float* src = mrg + ww * (8 * kD + 16);
-        const float a = fast_exp2((src[8 * kD + row] - M) * kLog2e);
-        L = fmaf(a, src[8 * kD + 8 + row], L);
-        const float4 u0 = reinterpret_cast<const float4*>(src + row * kD + d0)[0];
-        const float4 u1 = reinterpret_cast<const float4*>(src + row * kD + d0)[1];
+        const float* src = mrg + ww * kQ1MrgWarp;
+        const float a = fast_exp2((src[8 * kQ1MrgRow + row] - M) * kLog2e);
+        L = fmaf(a, src[8 * kQ1MrgRow + 8 + row], L);
+        const float* sl = src + row * kQ1MrgRow + (d0 >> 5) * kQ1MrgBlk + (d0 & 31);
+        const float4 u0 = reinterpret_cast<const float4*>(sl)[0];
+        const float4 u1 = reinterpret_cast<const float4*>(sl)[1];
         acc[0] = fmaf(a, u0.x, acc[0]); acc[1] = fmaf(a, u0.y, acc[1]);
         acc[2] = fmaf(a, u0.z, acc[2]); acc[3] = fmaf(a, u0.w, acc[3]);
         acc[4] = fmaf(a, u1.x, acc[4]); acc[5] = fmaf(a, u1.y, acc[5]);
