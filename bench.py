@@ -4,9 +4,10 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
 One step = one pass of the whole hot path over one batch: for every layer,
-tq4_encode_append of the step's new K/V positions, then tq4_decode_attention
-(decode workloads) or tq4_prefill_attention followed by the append of the
-chunk (prefill workload). The step's launches are captured once in a CUDA
+tq4_decode_append_attention (the step's new K/V positions appended, then decode
+attention over the whole history; with one query token the append runs inside
+the decode kernel) for decode workloads, or tq4_prefill_attention followed by
+tq4_encode_append of the chunk (prefill workload). The step's launches are captured once in a CUDA
 graph through the public C ABI and replayed; the timed region is exactly K
 replays between CUDA events, after W warm-up replays.
 
@@ -221,7 +222,7 @@ class DecodeSetup:
         qi, ki, vi, oi = [], [], [], []
         for layer in range(w.layers):
             pool = tq4.Context.new_pool(w.pool_pages, device)
-            kr, vr = [], []
+            knew_l, vnew_l = [], []
             for r in range(w.n_req):
                 first = w.shared_prefix_pages * 256 if r > 0 else 0
                 s = int(self.seq_np[r])
@@ -232,21 +233,22 @@ class DecodeSetup:
                     e = min(a + 32768, hist)
                     self.ctx.encode_append(pool, tt, first + a, torch.from_numpy(k[a:e]).to(device),
                                            torch.from_numpy(v[a:e]).to(device))
-                kr.append(ain.add(np.ascontiguousarray(k[hist:]), torch.float32, (w.n_q, 4, 256)))
-                vr.append(ain.add(np.ascontiguousarray(v[hist:]), torch.float32, (w.n_q, 4, 256)))
+                knew_l.append(np.ascontiguousarray(k[hist:]))
+                vnew_l.append(np.ascontiguousarray(v[hist:]))
                 del k, v
+            # the step's new K/V of all requests: [n_req, n_q, 4, 256] fp32
+            ki.append(ain.add(np.stack(knew_l), torch.float32, (w.n_req, w.n_q, 4, 256)))
+            vi.append(ain.add(np.stack(vnew_l), torch.float32, (w.n_req, w.n_q, 4, 256)))
             qb = I.queries(w.config, layer, (w.n_req, w.n_q, 24, 256))
             qi.append(ain.add(qb, torch.bfloat16, (w.n_req, w.n_q, 24, 256)))
             oi.append(aout.add(np.zeros((w.n_req, w.n_q, 24, 256), np.uint16), torch.bfloat16,
                                (w.n_req, w.n_q, 24, 256)))
-            ki.append(kr)
-            vi.append(vr)
             self.pools.append(pool)
         vin, vout = ain.finalize(), aout.finalize()
         self.arena_in, self.arena_out = ain, aout
         self.qs = [vin[i] for i in qi]
-        self.knew = [[vin[i] for i in kr] for kr in ki]
-        self.vnew = [[vin[i] for i in vr] for vr in vi]
+        self.knew = [vin[i] for i in ki]
+        self.vnew = [vin[i] for i in vi]
         self.outs = [vout[i] for i in oi]
         torch.cuda.synchronize()
         st = self.ctx.status()
@@ -254,33 +256,25 @@ class DecodeSetup:
             raise RuntimeError(f"cache build failed with device status {st}")
 
     # raw ABI calls (no Python-side allocation) so that the step can be captured
-    def append(self, layer):
-        tq4, w = self.tq4, self.w
-        for r in range(w.n_req):
-            s = int(self.seq_np[r])
-            rc = tq4.tq4_encode_append(self.ctx.handle, self.pools[layer], w.pool_pages, self.tables[r],
-                                       self.tables.shape[1], s - w.n_q, w.n_q, self.knew[layer][r],
-                                       self.vnew[layer][r], tq4.DTYPE_F32)
-            assert rc == 0, rc
-
     def attend(self, layer):
+        """The step's append and decode of one layer, one call (the timed attention call)."""
         tq4, w = self.tq4, self.w
-        rc = tq4.tq4_decode_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.qs[layer],
-                                      self.tables, self.tables.shape[1], self.seq, w.n_req, w.n_q,
-                                      self.total, SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws,
-                                      self.ws.numel())
+        rc = tq4.tq4_decode_append_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.knew[layer],
+                                             self.vnew[layer], tq4.DTYPE_F32, self.qs[layer], self.tables,
+                                             self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total, SCALE,
+                                             self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
         assert rc == 0, rc
 
     def step(self):
         for layer in range(self.w.layers):
-            self.append(layer)
             self.attend(layer)
 
     def units_per_step(self):
         return self.total * self.w.layers  # attended KV positions x layers
 
     def kernels_per_step(self):
-        return self.w.layers * (self.w.n_req + 2)
+        # decode + combine per layer; with n_q > 1 a tail-encode kernel as well
+        return self.w.layers * (2 if self.w.n_q == 1 else 3)
 
     def dominant_bytes(self):
         """Algorithmic bytes of one decode launch: the packed history it must read."""
@@ -537,7 +531,8 @@ def main():
         ach = S.dominant_bytes() / (att_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                 "traffic": measured_traffic("decode_q1", S.total) if w.n_q == 1 else None,
-                "kernel": "tq4_decode_attention (split-K kernel + combine)",
+                "kernel": "tq4_decode_append_attention (split-K decode with the append inside it for one "
+                          "query token + combine)",
                 "launch_ms": att_ms, "peak_source": f"{peak_kind} hbm_gbs"}
     else:
         ach = S.dominant_flops() / (att_ms * 1e-3) / 1e12

@@ -239,10 +239,21 @@ size_t tq4_decode_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q
   return plan_decode(ctx, n_req, n_q, total_seq_len).total;
 }
 
-int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q,
-                         const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens,
-                         int32_t n_req, int32_t n_q, int64_t total_seq_len, float scale, void* out,
-                         int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+struct AppendArgs {   // the fused append of tq4_decode_append_attention
+  void* pool;
+  const void* k_new;
+  const void* v_new;
+  int dtype;
+};
+
+int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q, const int32_t* page_tables,
+                int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q, int64_t total_seq_len,
+                float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream,
+                const AppendArgs* app) {
   if (!ctx || n_req < 0) return TQ4_ERR_ARG;
   if (n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS) return TQ4_ERR_UNSUPPORTED;
   if (n_req == 0) return TQ4_OK;
@@ -253,6 +264,10 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, cons
   if (total_seq_len < int64_t(n_req) * n_q || total_seq_len > int64_t(n_req) * max_pages * tq4::kPage)
     return TQ4_ERR_ARG;
   if (!aligned(pool, 16) || !aligned(q, 16) || !aligned(out, 16)) return TQ4_ERR_ARG;
+  if (app) {
+    if (!app->k_new || !app->v_new || !aligned(app->k_new, 16) || !aligned(app->v_new, 16)) return TQ4_ERR_ARG;
+    if (app->dtype != TQ4_DTYPE_F32 && app->dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
+  }
   const DecodePlan pl = plan_decode(ctx, n_req, n_q, total_seq_len);
   if (!workspace || workspace_bytes < pl.total || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
   if (int rc = check_device(ctx)) return rc;
@@ -277,8 +292,18 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, cons
   p.signs = ctx->signs;
   p.status = ctx->d_status;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   cudaError_t e;
+  if (app && n_q == 1) {   // appended inside the decode kernel
+    p.pool_w = static_cast<uint8_t*>(app->pool);
+    p.k_new = app->k_new;
+    p.v_new = app->v_new;
+    p.new_dtype = app->dtype;
+  } else if (app) {        // a tail-encode kernel ahead of the decode
+    e = tq4::launch_encode_tail(static_cast<uint8_t*>(app->pool), num_pages, page_tables, max_pages, seq_lens,
+                                n_req, n_q, app->k_new, app->v_new, app->dtype, ctx->signs, ctx->d_status, st);
+    if (e != cudaSuccess) return TQ4_ERR_CUDA;
+  }
+  const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   switch (tq4::decode_nt(n_q)) {
     case 1: {
       CUtensorMap map;
@@ -299,6 +324,28 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, cons
   if (e != cudaSuccess) return TQ4_ERR_CUDA;
   const int rows = n_req * n_q * tq4::kHq;
   return cuda_status(tq4::launch_pdl(tq4::decode_combine_kernel, dim3(rows), dim3(32 * tq4::kCombWarps), 0, st, p));
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q,
+                         const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens,
+                         int32_t n_req, int32_t n_q, int64_t total_seq_len, float scale, void* out,
+                         int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, nullptr);
+}
+
+int tq4_decode_append_attention(tq4_ctx* ctx, void* pool, int32_t num_pages, const void* k_new, const void* v_new,
+                                int new_dtype, const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                const int32_t* seq_lens, int32_t n_req, int32_t n_q, int64_t total_seq_len,
+                                float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes,
+                                void* stream) {
+  const AppendArgs app{pool, k_new, v_new, new_dtype};
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, &app);
 }
 
 size_t tq4_prefill_workspace_bytes(int32_t n_tok) {

@@ -56,6 +56,13 @@ struct DecodeParams {
   int out_dtype;
   Signs signs;
   int* status;
+  // fused append (n_q == 1): the new position of each request, [n_req][4][256] of
+  // new_dtype, is encoded into pool_w at position seq_len - 1 before it is attended;
+  // pool_w == nullptr means the positions are already in the pool
+  uint8_t* pool_w;
+  const void* k_new;
+  const void* v_new;
+  int new_dtype;
 };
 
 __host__ __device__ constexpr int decode_nt(int n_q) { return (6 * n_q + 7) / 8; }

@@ -19,9 +19,15 @@
 //   * V phase: O'^T += C_v^T P'^T over all 256 dims (M = dims, K = positions);
 //   * at the end the 8 warp states (m, l, o') are merged through shared memory
 //     and written as one split-K partial for the combine pass.
+//   * fused append: in the CTA that owns a request's last position, warps 6 and 7
+//     encode the new K and V vectors of this KV head (the append kernel's
+//     arithmetic), store them in the pool and fence them for the tensor-copy
+//     proxy; the warp whose tile holds that position issues that tile's TMA only
+//     after both have arrived on an mbarrier (normally long before it gets there).
 #pragma once
 #include <cuda.h>
 #include "tq4_decode.cuh"
+#include "tq4_encode.cuh"
 
 namespace tq4 {
 
@@ -112,6 +118,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return done != 0;
 }
+__device__ __forceinline__ void mbar_arrive_q1(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int c0, int c1, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n"
@@ -147,7 +156,9 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 4u);
 
   // prologue that reads none of the call's inputs (overlaps the previous kernel)
+  const uint32_t bar_new = base + 8;   // the fused append's new position is in the pool (count 2)
   if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
+  if (tid == kQ1Bufs) mbar_init(bar_new, 2);
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   {   // table rows through shuffles: lane l holds c[l & 15]
     const uint32_t cl = g_codebook.c16[lane & 15];
@@ -156,6 +167,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       st_shared_u32(kQ1Lut + b * 256 + lane * 4, lo | (hi << 16));
     }
   }
+  __syncthreads();   // barriers initialised before any warp arms one
   pdl_wait();
   pdl_launch_dependents();
   // (request, split) of this CTA: with one request it is (0, blockIdx.x); otherwise
@@ -194,6 +206,34 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   const int pos_e = min(pos_b + p.split_len, seq_len);
   const int n_tiles = (pos_e - pos_b + kQ1Tile - 1) / kQ1Tile;
   const int my_tiles = n_tiles > w ? (n_tiles - w + kQ1Warps - 1) / kQ1Warps : 0;
+  // fused append: this CTA holds the request's last position (seq_len - 1)
+  const bool append_here = p.pool_w != nullptr && pos_e == seq_len && pos_b < pos_e;
+  // warp 6: K, warp 7: V of KV head h. The input row is loaded early (fused_load);
+  // the encode, the store and the release to the tile's TMA follow (fused_encode).
+  float x_new[8];
+  auto fused_load = [&]() {
+    const int kv = w - (kQ1Warps - 2);
+    const void* src = kv ? p.v_new : p.k_new;
+    if (p.new_dtype == TQ4_DTYPE_F32)
+      load8<float>(static_cast<const float*>(src) + (int64_t(r) * kHkv + h) * kD + lane * 8, x_new);
+    else
+      load8<uint16_t>(static_cast<const uint16_t*>(src) + (int64_t(r) * kHkv + h) * kD + lane * 8, x_new);
+  };
+  auto fused_encode = [&]() {
+    const int kv = w - (kQ1Warps - 2);
+    float nrm;
+    const uint32_t word = encode_vector_warp(x_new, p.signs, nrm);
+    store_packed_warp(p.pool_w, p.num_pages, table, seq_len - 1, h, kv, word, nrm, p.status);
+    asm volatile("fence.proxy.async.global;\n" ::: "memory");   // generic stores -> the TMA reads below
+    __syncwarp();
+    if (lane == 0) mbar_arrive_q1(bar_new);
+  };
+  const int last_w = (n_tiles - 1) % kQ1Warps, last_k = (n_tiles - 1) / kQ1Warps;
+  const bool encoder = append_here && w >= kQ1Warps - 2;
+  // When the tile with the new position is its owner's first tile, its TMA is issued
+  // before the block-wide barrier below, so the encode must precede that barrier;
+  // otherwise it follows it and delays no warp.
+  const bool encode_first = encoder && last_k == 0;
 
   // ---- lane 0 of each warp streams the warp's tiles: tile w + 8k -> buffer w*2 + k%2
   auto tile_pos = [&](int k) { return pos_b + (w + k * kQ1Warps) * kQ1Tile; };
@@ -202,6 +242,12 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       const int c = tile_pos(k);
       const int b = w * kQ1Stages + (k % kQ1Stages);
       const uint32_t bar = base + kQ1BarOff + b * 8;
+      if (append_here && w == last_w && k == last_k) {   // the tile with the appended position
+        uint32_t spins = 0;
+        while (!mbar_try_wait(bar_new, 0) && ++spins < kQ1SpinLimit) {
+        }
+        if (spins >= kQ1SpinLimit) record_error(p.status, TQ4_ERR_TIMEOUT);
+      }
       int page = k == 0 ? page_first : __ldg(table + (c >> 8));
       if (page < 0 || page >= p.num_pages) {
         record_error(p.status, TQ4_ERR_PAGE_RANGE);
@@ -218,6 +264,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       bulk_load(ndst + 64, pg + kVNorms + slot0 * 2, kQ1Tile * 2, bar);
     }
   };
+  if (encoder) fused_load();
+  if (encode_first) fused_encode();
   issue_tile(0);
 
   // ---- q' = R q * scale for the 6 query heads of this KV head, split hi + lo, virtual order
@@ -250,6 +298,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     }
   }
   __syncthreads();
+  if (encoder && !encode_first) fused_encode();   // after the block-wide barrier: no warp waits for it
 
   uint32_t qh[16][2], ql[16][2];
 #pragma unroll

@@ -76,6 +76,25 @@ __device__ __forceinline__ void warp_fwht256(float v[8]) {
   }
 }
 
+// The 8 sign bits of coordinates 8*lane .. 8*lane + 7 (bit i = coordinate 8*lane + i).
+// Word lane / 4 is picked with constant indices behind an empty asm, so a Signs
+// held in kernel parameters is not copied to local memory for an indexed read.
+__device__ __forceinline__ uint32_t lane_sign_bits(const Signs& s) {
+  const int lane = threadIdx.x & 31;
+  uint32_t w = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t wk = s.bits[k];
+    asm("" : "+r"(wk));
+    w = ((lane >> 2) == k) ? wk : w;
+  }
+  return (w >> (8 * (lane & 3))) & 0xFFu;
+}
+// flip the sign of x when bit i of sb is set
+__device__ __forceinline__ float apply_sign(float x, uint32_t sb, int i) {
+  return __uint_as_float(__float_as_uint(x) ^ (((sb >> i) & 1u) << 31));
+}
+
 // sign of coordinate 8*lane + i as a float multiplier
 __device__ __forceinline__ float sign_of(const Signs& s, int coord) {
   return ((s.bits[coord >> 5] >> (coord & 31)) & 1u) ? -1.0f : 1.0f;

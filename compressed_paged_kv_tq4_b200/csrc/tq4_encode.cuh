@@ -37,6 +37,56 @@ __device__ __forceinline__ void load8<uint16_t>(const uint16_t* src, float v[8])
   }
 }
 
+// Quantise one head vector held by a warp (lane l: coordinates 8l..8l+7 in x).
+// Returns lane l's packed word (word l of the vector); n receives ||x||_2.
+__device__ __forceinline__ uint32_t encode_vector_warp(const float x[8], const Signs& signs, float& n) {
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  n = sqrtf(ss);
+  uint32_t word = 0;
+  if (n > 0.f) {
+    const uint32_t sb = lane_sign_bits(signs);
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = apply_sign(x[i] / n, sb, i);
+    warp_fwht256(y);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float yi = y[i] * 0.0625f;  // 1/16, exact
+      uint32_t idx = 0;
+#pragma unroll
+      for (int j = 0; j < 15; ++j) idx += (yi > g_codebook.b[j]) ? 1u : 0u;
+      word |= idx << (4 * i);
+    }
+  }
+  return word;
+}
+
+// Store a packed vector (word of this lane, fp16 norm by lane 0) at position pos of
+// a request (page table `table`), head `head`, K (kv = 0) or V. A page id outside
+// [0, num_pages) records TQ4_ERR_PAGE_RANGE and writes nothing; returns false then.
+__device__ __forceinline__ bool store_packed_warp(uint8_t* pool, int32_t num_pages, const int32_t* table, int32_t pos,
+                                                  int head, int kv, uint32_t word, float n, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int32_t page = __ldg(table + (pos >> 8));
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+    return false;
+  }
+  const int slot = pos & (kPage - 1);
+  uint8_t* base = pool + int64_t(page) * kPageBytes;
+  uint32_t* words = reinterpret_cast<uint32_t*>(base + (kv ? kVWords : kKWords)) + (head * kPage + slot) * kWords;
+  words[lane] = word;
+  if (lane == 0) {
+    __half* norms = reinterpret_cast<__half*>(base + (kv ? kVNorms : kKNorms));
+    norms[head * kPage + slot] = __float2half_rn(n);
+  }
+  return true;
+}
+
 // grid: ceil(n_tok * 8 / warps_per_block); warp -> (token, kv, head)
 template <typename T>
 __global__ void __launch_bounds__(256) encode_append_kernel(
@@ -51,48 +101,39 @@ __global__ void __launch_bounds__(256) encode_append_kernel(
   const int tok = int(vec / (2 * kHkv));
   const int kv = int(vec / kHkv) & 1;       // 0 = K, 1 = V
   const int head = int(vec % kHkv);
-  const T* src = (kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8;
-
   float x[8];
-  load8<T>(src, x);
-  float ss = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
-#pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-  const float n = sqrtf(ss);
+  load8<T>((kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8, x);
+  float n;
+  const uint32_t word = encode_vector_warp(x, signs, n);
+  store_packed_warp(pool, num_pages, page_table, start_pos + tok, head, kv, word, n, status);
+}
 
-  uint32_t word = 0;
-  if (n > 0.f) {
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = (x[i] / n) * sign_of(signs, lane * 8 + i);
-    warp_fwht256(y);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float yi = y[i] * 0.0625f;  // 1/16, exact
-      uint32_t idx = 0;
-#pragma unroll
-      for (int j = 0; j < 15; ++j) idx += (yi > g_codebook.b[j]) ? 1u : 0u;
-      word |= idx << (4 * i);
-    }
-  }
-
-  const int32_t p = start_pos + tok;
-  const int32_t page = __ldg(page_table + (p >> 8));
-  if (page < 0 || page >= num_pages) {
-    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+// The last n_q positions of every request, with positions taken from the device
+// lengths: new token t of request r goes to position seq_lens[r] - n_q + t.
+// grid: ceil(n_req * n_q * 8 / warps_per_block); inputs [n_req][n_q][4][256].
+template <typename T>
+__global__ void __launch_bounds__(256) encode_tail_kernel(
+    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_tables, int32_t max_pages,
+    const int32_t* __restrict__ seq_lens, int32_t n_req, int32_t n_q, const T* __restrict__ k_new,
+    const T* __restrict__ v_new, Signs signs, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (vec >= int64_t(n_req) * n_q * 2 * kHkv) return;
+  const int64_t tok = vec / (2 * kHkv);       // request-major token index
+  const int r = int(tok / n_q), t = int(tok % n_q);
+  const int kv = int(vec / kHkv) & 1;
+  const int head = int(vec % kHkv);
+  const int32_t len = __ldg(seq_lens + r);
+  if (len < n_q || len > max_pages * kPage) {   // the decode kernels record TQ4_ERR_SEQ for it
     return;
   }
-  const int slot = p & (kPage - 1);
-  uint8_t* base = pool + int64_t(page) * kPageBytes;
-  uint32_t* words = reinterpret_cast<uint32_t*>(base + (kv ? kVWords : kKWords)) +
-                    (head * kPage + slot) * kWords;
-  words[lane] = word;
-  if (lane == 0) {
-    __half* norms = reinterpret_cast<__half*>(base + (kv ? kVNorms : kKNorms));
-    norms[head * kPage + slot] = __float2half_rn(n);
-  }
+  float x[8];
+  load8<T>((kv ? v_new : k_new) + (tok * kHkv + head) * kD + lane * 8, x);
+  float n;
+  const uint32_t word = encode_vector_warp(x, signs, n);
+  store_packed_warp(pool, num_pages, page_tables + int64_t(r) * max_pages, len - n_q + t, head, kv, word, n, status);
 }
 
 // grid: ceil(n * 8 / warps_per_block); writes fp32 [n][4][256] for K and V
@@ -150,6 +191,21 @@ cudaError_t launch_encode_append(uint8_t* pool, int32_t num_pages, const int32_t
                       static_cast<const float*>(v_new), signs, status);
   return launch_pdl(encode_append_kernel<uint16_t>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
                     page_table, start_pos, n_tok, static_cast<const uint16_t*>(k_new),
+                    static_cast<const uint16_t*>(v_new), signs, status);
+}
+
+cudaError_t launch_encode_tail(uint8_t* pool, int32_t num_pages, const int32_t* page_tables, int32_t max_pages,
+                               const int32_t* seq_lens, int32_t n_req, int32_t n_q, const void* k_new,
+                               const void* v_new, int dtype, const Signs& signs, int* status, cudaStream_t stream) {
+  const int threads = 256, wpb = threads / 32;
+  const int64_t vecs = int64_t(n_req) * n_q * 2 * kHkv;
+  const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
+  if (dtype == TQ4_DTYPE_F32)
+    return launch_pdl(encode_tail_kernel<float>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                      page_tables, max_pages, seq_lens, n_req, n_q, static_cast<const float*>(k_new),
+                      static_cast<const float*>(v_new), signs, status);
+  return launch_pdl(encode_tail_kernel<uint16_t>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                    page_tables, max_pages, seq_lens, n_req, n_q, static_cast<const uint16_t*>(k_new),
                     static_cast<const uint16_t*>(v_new), signs, status);
 }
 

@@ -38,6 +38,7 @@ EXPORTS = (
     "tq4_ctx_create", "tq4_ctx_destroy", "tq4_codebook", "tq4_encode_append", "tq4_reconstruct",
     "tq4_decode_workspace_bytes", "tq4_decode_attention", "tq4_prefill_workspace_bytes",
     "tq4_prefill_attention", "tq4_get_status", "tq4_status_string", "tq4_decode_attention_noalloc",
+    "tq4_decode_append_attention",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -73,6 +74,8 @@ _sig = {
     "tq4_decode_attention_noalloc": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int, _p],
                                      ctypes.c_int),
     "tq4_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "tq4_decode_append_attention": ([_p, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32, _i32, _i64, _f,
+                                     _p, ctypes.c_int, _p, _sz, _p], ctypes.c_int),
 }
 for _name, (_args, _res) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -154,6 +157,15 @@ def tq4_decode_attention(ctx, pool, num_pages, q, page_tables, max_pages, seq_le
     return _lib.tq4_decode_attention(ctx, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
                                      _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out),
                                      out_dtype, _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_decode_append_attention(ctx, pool, num_pages, k_new, v_new, new_dtype, q, page_tables, max_pages,
+                                seq_lens, n_req, n_q, total_seq_len, scale, out, out_dtype, workspace,
+                                workspace_bytes, stream=None) -> int:
+    return _lib.tq4_decode_append_attention(ctx, _ptr(pool), num_pages, _ptr(k_new), _ptr(v_new), new_dtype,
+                                            _ptr(q), _ptr(page_tables), max_pages, _ptr(seq_lens), n_req, n_q,
+                                            total_seq_len, scale, _ptr(out), out_dtype, _ptr(workspace),
+                                            workspace_bytes, _stream(stream))
 
 
 def tq4_prefill_workspace_bytes(n_tok) -> int:
@@ -252,6 +264,30 @@ class Context:
         _check(tq4_decode_attention(self.handle, pool, pool.numel() // PAGE_BYTES, q, page_tables,
                                     page_tables.shape[1], seq_lens, n_req, n_q, total_seq_len, scale, out,
                                     od, workspace, workspace.numel(), stream), "tq4_decode_attention")
+        return out
+
+    def decode_append_attention(self, pool, k_new, v_new, q, page_tables, seq_lens, total_seq_len, scale,
+                                out=None, out_dtype=torch.bfloat16, workspace=None, stream=None):
+        """Append k_new/v_new [n_req, n_q, 4, 256] (float32 or bfloat16) at the last n_q
+        positions of each request, then decode as decode_attention."""
+        _need_cuda(pool, k_new, v_new, q, page_tables, seq_lens)
+        if q.dtype != torch.bfloat16:
+            raise ValueError("q must be bfloat16")
+        nd = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(k_new.dtype)
+        if nd is None or v_new.dtype != k_new.dtype:
+            raise ValueError("k_new/v_new must both be float32 or bfloat16")
+        n_req, n_q = q.shape[0], q.shape[1]
+        if tuple(k_new.shape) != (n_req, n_q, KV_HEADS, HEAD_DIM) or k_new.shape != v_new.shape:
+            raise ValueError("k_new/v_new must be [n_req, n_q, 4, 256]")
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        if workspace is None:
+            workspace = self.decode_workspace(n_req, n_q, total_seq_len, q.device)
+        _check(tq4_decode_append_attention(self.handle, pool, pool.numel() // PAGE_BYTES, k_new, v_new, nd, q,
+                                           page_tables, page_tables.shape[1], seq_lens, n_req, n_q,
+                                           total_seq_len, scale, out, od, workspace, workspace.numel(), stream),
+               "tq4_decode_append_attention")
         return out
 
     def prefill_attention(self, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,

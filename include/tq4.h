@@ -150,6 +150,29 @@ int tq4_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                          void* out, int out_dtype,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode step with its append ([KVEXEC]: the step's new K/V are encoded into the
+ * request's TQ4 pages, then attention runs over the paged history including them):
+ * the same result as tq4_encode_append of each request's n_q new positions
+ * followed by tq4_decode_attention, in one call.
+ *   pool        device, written: the new positions are stored in it.
+ *   k_new,v_new device [n_req][n_q][4][256] of new_dtype (TQ4_DTYPE_F32 or
+ *               TQ4_DTYPE_BF16). Token t of request r is stored at position
+ *               seq_lens[r] - n_q + t of that request (seq_lens count the new
+ *               positions, as in tq4_decode_attention).
+ *   all other arguments, the workspace, outputs and errors: as tq4_decode_attention.
+ * With n_q == 1 the encode runs inside the decode kernel: the CTA that holds a
+ * request's last position encodes it (per KV head) and stores it before it loads
+ * that tile, so no separate append launch is made. With n_q > 1 a tail-encode
+ * kernel runs ahead of the decode. A new position whose page id is out of range
+ * records TQ4_ERR_PAGE_RANGE and is not written. */
+int tq4_decode_append_attention(tq4_ctx* ctx, void* pool, int32_t num_pages,
+                                const void* k_new, const void* v_new, int new_dtype,
+                                const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                int64_t total_seq_len, float scale,
+                                void* out, int out_dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Prefill attention: a causal chunk of n_tok query tokens against the request's
  * TQ4 prefix [0, prefix_len) plus the chunk itself, whose K/V are given at full
  * precision ([KVEXEC] multi-query prefill). The chunk is not appended; call
