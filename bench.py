@@ -68,10 +68,17 @@ def peaks():
 # (summarised under profiles/), per unit of work. A figure counts only while the
 # kernel's source file hashes to the value it had when the counters were taken.
 MEASURED_TRAFFIC = {
-    # decode_q1_kernel, decode_32k capture: 34,146,048 B read + 74,240 B written for
-    # 32,768 positions; the kernel's traffic grows with the positions it streams
-    "decode_q1": ("tq4_decode_q1.cuh", "800114719a0281f06ec035d23001165314f238f5bc629e438f4f6a92f42810a3",
-                  (34_146_048 + 74_240) / 32_768),
+    # decode_q1_kernel, decode_32k capture (append fused): 34,171,392 B read + 54,272 B
+    # written for 32,768 positions; its traffic grows with the positions it streams
+    "decode_q1": ("tq4_decode_q1.cuh", "8af3e5b1d6289ad4c18ebbde56ac38cca241bcb35dc300ebc496258bdf6e95f9",
+                  (34_171_392 + 54_272) / 32_768),
+    # decode_splitk_kernel<3>, verify_2req_229k capture: 221,719,808 B read + 6,663,168 B
+    # written for 229,376 positions (the 64 shared pages partly hit in L2: this workload only)
+    "decode_splitk": ("tq4_decode.cuh", "52fa5f2d3917b89d50f3893b4ed8c0bd0327a57a9259dd4152597a2f3febeebe",
+                      (221_719_808 + 6_663_168) / 229_376),
+    # prefill_tc_kernel, prefill_2k_on_32k capture: one launch
+    "prefill_tc": ("tq4_prefill_tc.cuh", "ba2e11002be6b5829d25210f8c5594dafcd611b563d84415a558b9f5d9701aeb",
+                   94_314_752 + 9_152_768),
 }
 
 
@@ -530,14 +537,16 @@ def main():
     if w.kind == "decode":
         ach = S.dominant_bytes() / (att_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": measured_traffic("decode_q1", S.total) if w.n_q == 1 else None,
+                "traffic": (measured_traffic("decode_q1", S.total) if w.n_q == 1 else
+                            measured_traffic("decode_splitk", S.total) if w.name == "verify_2req_229k" else None),
                 "kernel": "tq4_decode_append_attention (split-K decode with the append inside it for one "
                           "query token + combine)",
                 "launch_ms": att_ms, "peak_source": f"{peak_kind} hbm_gbs"}
     else:
         ach = S.dominant_flops() / (att_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s", "frac": ach / bf16,
-                "traffic": None, "kernel": "tq4_prefill_attention (rotate prologue + attention kernel)",
+                "traffic": measured_traffic("prefill_tc", 1) if w.name == "prefill_2k_on_32k" else None,
+                "kernel": "tq4_prefill_attention (rotate prologue + attention kernel)",
                 "launch_ms": att_ms, "peak_source": f"{peak_kind} bf16_tflops (f16 operands: same nominal rate)"}
 
     # end to end: pinned host inputs in, results out, every step
