@@ -486,19 +486,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         kn[u] = expand(j, u);
         big = fmaxf(big, kn[u]);
       }
-      // chunk-row copies complete before the next tile's loads are issued (the wait
-      // would otherwise also cover those)
       cp_async_commit();
       cp_async_wait<0>();
-      if (more) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) fetch(j + 2, u, pg_next);
-      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) big = fmaxf(big, __shfl_xor_sync(0xffffffffu, big, o));
       if (lane == 0) kmax[(w - kTcSoftWarps) & 3] = big;   // read by the MMA thread after k_full
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic-proxy writes -> tensor-core reads
       mbar_arrive(bar_k_full + 8 * grp_id);
+      // the next tile's loads go out only now: the wait and the proxy fence above
+      // would otherwise wait for them as well
+      if (more) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fetch(j + 2, u, pg_next);
+      }
       // ---- V half and both norms: free once PV(j - 2) has run
       if (j >= 2 && !bounded_wait(bar_v_empty + 8 * grp_id, ((j >> 1) - 1) & 1)) break;
 #pragma unroll
@@ -512,12 +512,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       }
       cp_async_commit();
       cp_async_wait<0>();
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      mbar_arrive(bar_v_full + 8 * grp_id);
       if (more) {
 #pragma unroll
         for (int u = 4; u < 8; ++u) fetch(j + 2, u, pg_next);
       }
-      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      mbar_arrive(bar_v_full + 8 * grp_id);
       pg_next = pg_far;
     }
   } else {
