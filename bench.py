@@ -63,6 +63,26 @@ def peaks():
         return 6650.0, 1590.0, 1400.0, "fallback"
 
 
+WORKLOAD_DESC = {
+    "decode_32k": "16 layers x 32,768 TQ4 positions, 1 request, 1 bf16 query token, 24 Q / 4 KV heads x 256",
+    "decode_213k_outliers": "16 layers x 212,992 TQ4 positions (5% x8 outliers), 1 request, 1 query token",
+    "verify_2req_229k": "2 requests (163,840 + 65,536 positions, 64 shared pages), 4 causal query tokens each, "
+                        "16 layers",
+    "prefill_2k_on_32k": "2,048 causal bf16 query tokens on a 32,768-position TQ4 prefix + the chunk, 16 layers",
+    "single_layer_2k": "1 layer, 2,048 TQ4 positions, 1 query token",
+}
+
+
+def workload_config(name, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    w = I.WORKLOADS[name]
+    return {"workload": f"{name}: {WORKLOAD_DESC[name]}", "append_per_layer": w.append_per_step,
+            "pool_pages": w.pool_pages, "page_positions": 256,
+            "l2": "inputs larger than L2: packed KV read per step is "
+                  f"{w.layers * sum(w.seq_lens) * 1040 / 1e6:.0f} MB vs 126 MB L2",
+            "parallelism": f"replicas x{world}"}
+
+
 # ---------------------------------------------------------------------------- measured DRAM traffic
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
 # (summarised under profiles/), per unit of work. A figure counts only while the
@@ -77,8 +97,8 @@ MEASURED_TRAFFIC = {
     "decode_splitk": ("tq4_decode.cuh", "52fa5f2d3917b89d50f3893b4ed8c0bd0327a57a9259dd4152597a2f3febeebe",
                       (221_719_808 + 6_663_168) / 229_376),
     # prefill_tc_kernel, prefill_2k_on_32k capture: one launch
-    "prefill_tc": ("tq4_prefill_tc.cuh", "ba2e11002be6b5829d25210f8c5594dafcd611b563d84415a558b9f5d9701aeb",
-                   94_314_752 + 9_152_768),
+    "prefill_tc": ("tq4_prefill_tc.cuh", "f290435adb0de7f5ccb086652cf386f89fbab4a08afeb143fa73615e1aa92529",
+                   93_480_960 + 9_271_552),
 }
 
 
@@ -441,7 +461,7 @@ def run_reference(args, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(args.steps, 1) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded Gaussian K/V and queries)",
-            "config": {"workload": args.workload, "sample": orc.sample},
+            "config": dict(workload_config(args.workload, args.gpus), sample=orc.sample),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
                              "sample": orc.sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -578,23 +598,13 @@ def main():
                "seconds": el}
 
     if rank == 0:
-        desc = {
-            "decode_32k": "16 layers x 32,768 TQ4 positions, 1 request, 1 bf16 query token, 24 Q / 4 KV heads x 256",
-            "decode_213k_outliers": "16 layers x 212,992 TQ4 positions (5% x8 outliers), 1 request, 1 query token",
-            "verify_2req_229k": "2 requests (163,840 + 65,536 positions, 64 shared pages), 4 causal query tokens each, 16 layers",
-            "prefill_2k_on_32k": "2,048 causal bf16 query tokens on a 32,768-position TQ4 prefix + the chunk, 16 layers",
-            "single_layer_2k": "1 layer, 2,048 TQ4 positions, 1 query token",
-        }[args.workload]
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "u4 codes, f16 tensor-core operands, f32 accumulate",
             "data": "synthetic (seeded Gaussian K/V and queries)",
-            "config": {"workload": f"{args.workload}: {desc}", "append_per_layer": w.append_per_step,
-                       "pool_pages": w.pool_pages, "page_positions": 256,
-                       "l2": "inputs larger than L2: packed KV read per step is "
-                             f"{w.layers * sum(w.seq_lens) * 1040 / 1e6:.0f} MB vs 126 MB L2",
-                       "parallelism": f"replicas x{world}", "graph": graph is not None},
+            "config": workload_config(args.workload, world),
+            "graph": graph is not None,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": S.kernels_per_step() * args.steps,
             "clocks": clk.summary(),
