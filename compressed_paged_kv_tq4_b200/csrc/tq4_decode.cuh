@@ -525,11 +525,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
 }
 
 // One CTA of 8 warps per output row (request, token, query head). Warp w
-// merges items first + w, first + w + 8, ... four at a time (all loads of a
+// merges items first + w, first + w + 8, ... kCombBatch (8) at a time (all loads of a
 // group are issued before any is used, so the L2 round trips overlap), then
 // the 8 warp results are merged through shared memory, rotated back by R^T
 // and written out.
 constexpr int kCombWarps = 8;
+constexpr int kCombBatch = 8;   // splits each warp loads before using any (one L2 round for up to 64 splits)
 
 __device__ __forceinline__ int request_first_item(const DecodeParams& p, int r) {
   const int lane = threadIdx.x & 31;
@@ -577,11 +578,11 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const D
   float m = -INFINITY, l = 0.f, acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int x0 = first + w; x0 < first + n_split; x0 += 4 * kCombWarps) {
-    float2 ml[4];
-    float4 u[4][2];
+  for (int x0 = first + w; x0 < first + n_split; x0 += kCombBatch * kCombWarps) {
+    float2 ml[kCombBatch];
+    float4 u[kCombBatch][2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kCombBatch; ++j) {
       const int x = x0 + j * kCombWarps;
       if (x < first + n_split) {
         const int64_t rec = (int64_t(x) * kHkv + h) * p.rows_pad + row;
@@ -596,14 +597,14 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const D
     }
     float mn = m;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) mn = fmaxf(mn, ml[j].x);
+    for (int j = 0; j < kCombBatch; ++j) mn = fmaxf(mn, ml[j].x);
     if (mn == -INFINITY) continue;
     const float a = fast_exp2((m - mn) * kLog2e);
     l *= a;
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] *= a;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < kCombBatch; ++j) {
       const float wj = fast_exp2((ml[j].x - mn) * kLog2e);   // 0 for empty slots (m = -inf)
       l = fmaf(wj, ml[j].y, l);
       acc[0] = fmaf(wj, u[j][0].x, acc[0]); acc[1] = fmaf(wj, u[j][0].y, acc[1]);
