@@ -88,14 +88,14 @@ def workload_config(name, world):
 # (summarised under profiles/), per unit of work. A figure counts only while the
 # kernel's source file hashes to the value it had when the counters were taken.
 MEASURED_TRAFFIC = {
-    # decode_q1_kernel, decode_32k capture (append fused): 34,171,392 B read + 54,272 B
+    # decode_q1_kernel, decode_32k capture (append fused): 34,171,904 B read + 43,520 B
     # written for 32,768 positions; its traffic grows with the positions it streams
-    "decode_q1": ("tq4_decode_q1.cuh", "8af3e5b1d6289ad4c18ebbde56ac38cca241bcb35dc300ebc496258bdf6e95f9",
-                  (34_171_392 + 54_272) / 32_768),
-    # decode_splitk_kernel<3>, verify_2req_229k capture: 221,719,808 B read + 6,663,168 B
+    "decode_q1": ("tq4_decode_q1.cuh", "99ff80eec990bddce18158282a5942b25660898fc25e8a57af5a602a0198e6a7",
+                  (34_171_904 + 43_520) / 32_768),
+    # decode_splitk_kernel<3>, verify_2req_229k capture: 221,675,264 B read + 3,709,696 B
     # written for 229,376 positions (the 64 shared pages partly hit in L2: this workload only)
-    "decode_splitk": ("tq4_decode.cuh", "52fa5f2d3917b89d50f3893b4ed8c0bd0327a57a9259dd4152597a2f3febeebe",
-                      (221_719_808 + 6_663_168) / 229_376),
+    "decode_splitk": ("tq4_decode.cuh", "d27dcffa6032aeb25c0c742e6ca77347597bf628fd34c9a1f3d0b6a41afc0340",
+                      (221_675_264 + 3_709_696) / 229_376),
     # prefill_tc_kernel, prefill_2k_on_32k capture: one launch
     "prefill_tc": ("tq4_prefill_tc.cuh", "f290435adb0de7f5ccb086652cf386f89fbab4a08afeb143fa73615e1aa92529",
                    93_480_960 + 9_271_552),

@@ -563,13 +563,16 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const D
   const int h = qh / kGroup;
   const int row = tok * kGroup + qh % kGroup;
 
-  if (w == 0) {
-    const int f = request_first_item(p, r);
-    if (lane == 0) s_first = f;
+  const int s_len = __ldg(p.seq_lens + r);   // issued before the scan below needs anything
+  int first = 0;   // a single request's splits start at item 0
+  if (p.n_req > 1) {
+    if (w == 0) {
+      const int f = request_first_item(p, r);
+      if (lane == 0) s_first = f;
+    }
+    __syncthreads();
+    first = s_first;
   }
-  __syncthreads();
-  const int first = s_first;
-  const int s_len = __ldg(p.seq_lens + r);
   const bool ok = seq_ok(s_len, p.n_q, p.max_pages);
   int n_split = ok ? (s_len + p.split_len - 1) / p.split_len : 0;
   if (first + n_split > p.items_ub) n_split = 0;

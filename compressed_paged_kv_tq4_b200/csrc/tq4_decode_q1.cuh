@@ -81,15 +81,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];\n" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
-__device__ __forceinline__ float4 ld_shared_f4(uint32_t a) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];\n" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
-  return v;
-}
-__device__ __forceinline__ void st_shared_f4(uint32_t a, float4 v) {
-  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};\n" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
-               : "memory");
-}
 __device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
   uint16_t v;
   asm volatile("ld.shared.b16 %0, [%1];\n" : "=h"(v) : "r"(a));
