@@ -379,23 +379,29 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         s[j][2 * e] = (ok && row_ok0) ? (sc[j][2 * e] + sd[j][2 * e]) * kn[j][e] * kLog2e : -INFINITY;
         s[j][2 * e + 1] = (ok && row_ok1) ? (sc[j][2 * e + 1] + sd[j][2 * e + 1]) * kn[j][e] * kLog2e : -INFINITY;
       }
-    bool raise = false;
-    float alpha[2] = {1.f, 1.f};
+    // Lazy reference: a row's reference is raised only when the row max exceeds it by
+    // more than 2^8. Each lane first tests its own scores; the row maxima (shuffles)
+    // are formed only in the rare tiles where some lane needs a raise.
+    float lmax[2];
+    bool need = false;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {   // e: row 2t+e
-      float v = fmaxf(fmaxf(s[0][e], s[0][e + 2]), fmaxf(s[1][e], s[1][e + 2]));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-      v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-      if (v > m_ref[e] + kQ1Lazy) {       // raise the reference: weights would exceed 2^8
-        alpha[e] = fast_exp2(m_ref[e] - v);   // 0 on the first raise (m_ref = -inf)
-        m_ref[e] = v;
-        raise = true;
-      }
+      lmax[e] = fmaxf(fmaxf(s[0][e], s[0][e + 2]), fmaxf(s[1][e], s[1][e + 2]));
+      need |= lmax[e] > m_ref[e] + kQ1Lazy;
     }
-    const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
-    const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
-    if (__any_sync(0xffffffffu, raise)) {
+    if (__any_sync(0xffffffffu, need)) {
+      float alpha[2] = {1.f, 1.f};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = lmax[e];
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        if (v > m_ref[e] + kQ1Lazy) {           // weights would exceed 2^8
+          alpha[e] = fast_exp2(m_ref[e] - v);   // 0 on the first raise (m_ref = -inf)
+          m_ref[e] = v;
+        }
+      }
       l_part[0] *= alpha[0];
       l_part[1] *= alpha[1];
 #pragma unroll
@@ -406,6 +412,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         o[mt][3] *= alpha[1];
       }
     }
+    const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
+    const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
     uint32_t bh[2][2], bl[2][2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
