@@ -60,6 +60,8 @@ def _setup(config, seq_lens, n_q, dtype):
     (1, [4096], torch.bfloat16),          # new position in slot 255
     (1, [700, 1300], torch.float32),      # two requests
     (1, [33], torch.bfloat16),            # one short split
+    (1, [20000], torch.float32),          # last split: a partial round of 32-position tiles
+    (1, [32556], torch.bfloat16),         # last split: a full round, then 16-position tiles
     (2, [1500, 257], torch.float32),
     (4, [2048, 333], torch.bfloat16),
 ])

@@ -174,6 +174,9 @@ def test_decode_single_layer_2k_parity():
     ([1], 1, 0), ([17], 1, 0), ([255], 1, 0), ([256], 1, 0), ([257], 1, 0),
     ([1000, 63, 2047], 1, 0), ([300], 2, 0), ([513, 40], 3, 0), ([2048, 700], 4, 2),
     ([4], 4, 0), ([5000], 4, 0),
+    # one query token, longer splits: full rounds of 32-position tiles, then 16-position
+    # tail tiles (remainder <= 128) or a partial round of 32-position tiles (remainder > 128)
+    ([20000], 1, 0), ([9000, 3100], 1, 0),
 ])
 def test_decode_variants_parity(seq_lens, n_q, shared):
     case = Case(7, seq_lens, n_q, shared_pages=shared, outliers=0.05, chunks=(333,))
