@@ -2,8 +2,9 @@
 
     python -m compressed_paged_kv_tq4_b200.build [--force] [--verbose]
 
-The library is one translation unit (csrc/tq4_api.cu includes the kernel
-headers). The shared object lands next to this file so that it travels with
+The library is two translation units: csrc/tq4_api.cu (the C ABI of the
+kernels, which includes the kernel headers) and csrc/tq4_pages.cpp (the host
+page pool). The shared object lands next to this file so that it travels with
 the source tree; it is rebuilt when any source or the public header is newer.
 """
 from __future__ import annotations
@@ -18,7 +19,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libtq4.so")
-SOURCES = [os.path.join(HERE, "csrc", "tq4_api.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "tq4_api.cu"), os.path.join(HERE, "csrc", "tq4_pages.cpp")]
 ARCH = "-gencode=arch=compute_100a,code=sm_100a"
 
 
@@ -30,8 +31,8 @@ def _nvcc() -> str:
 
 
 def _inputs():
-    return (glob.glob(os.path.join(HERE, "csrc", "*")) +
-            [os.path.join(ROOT, "include", "tq4.h"), os.path.abspath(__file__)])
+    return (glob.glob(os.path.join(HERE, "csrc", "*")) + glob.glob(os.path.join(ROOT, "include", "*.h")) +
+            [os.path.abspath(__file__)])
 
 
 def needs_build() -> bool:

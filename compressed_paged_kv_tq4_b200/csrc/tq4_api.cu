@@ -394,6 +394,7 @@ const char* tq4_status_string(int status) {
     case TQ4_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
     case TQ4_ERR_SEQ: return "sequence length inconsistent with page table or plan";
     case TQ4_ERR_TIMEOUT: return "a bounded device-side wait gave up";
+    case TQ4_ERR_NO_PAGES: return "not enough page-pool capacity";
     default: return "unknown status";
   }
 }

@@ -23,6 +23,7 @@ TQ4_ERR_CUDA = -4
 TQ4_ERR_WORKSPACE = -5
 TQ4_ERR_SEQ = -6
 TQ4_ERR_TIMEOUT = -7
+TQ4_ERR_NO_PAGES = -8
 
 HEAD_DIM = 256
 PAGE_POSITIONS = 256
@@ -39,6 +40,10 @@ EXPORTS = (
     "tq4_decode_workspace_bytes", "tq4_decode_attention", "tq4_prefill_workspace_bytes",
     "tq4_prefill_attention", "tq4_get_status", "tq4_status_string", "tq4_decode_attention_noalloc",
     "tq4_decode_append_attention",
+    # host page pool (include/tq4_pages.h)
+    "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
+    "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
+    "tq4_pages_available", "tq4_pages_refcount", "tq4_pages_free_list",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -76,6 +81,19 @@ _sig = {
     "tq4_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "tq4_decode_append_attention": ([_p, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32, _i32, _i64, _f,
                                      _p, ctypes.c_int, _p, _sz, _p], ctypes.c_int),
+    "tq4_pages_create": ([_i32, ctypes.POINTER(_p)], ctypes.c_int),
+    "tq4_pages_destroy": ([_p], ctypes.c_int),
+    "tq4_pages_reservation": ([_i64, _i64], _i64),
+    "tq4_pages_admit": ([_p, _i64, _i64, _i32, _i64, ctypes.POINTER(_i32), ctypes.POINTER(_i32),
+                         ctypes.POINTER(_i32)], ctypes.c_int),
+    "tq4_pages_grow": ([_p, _i32, _i64], ctypes.c_int),
+    "tq4_pages_finish": ([_p, _i32], ctypes.c_int),
+    "tq4_pages_step_boundary": ([_p], ctypes.c_int),
+    "tq4_pages_table": ([_p, _i32, _p, _i32, ctypes.POINTER(_i32), ctypes.POINTER(_i64)], ctypes.c_int),
+    "tq4_pages_free_count": ([_p], _i32),
+    "tq4_pages_available": ([_p], _i32),
+    "tq4_pages_refcount": ([_p, _i32], _i32),
+    "tq4_pages_free_list": ([_p, _p, _i32], _i32),
 }
 for _name, (_args, _res) in _sig.items():
     _fn = getattr(_lib, _name)
@@ -190,6 +208,108 @@ def tq4_decode_attention_noalloc(ctx, pool, num_pages, q, page_tables, max_pages
 
 def tq4_get_status(ctx, stream=None) -> int:
     return _lib.tq4_get_status(ctx, _stream(stream))
+
+
+# ---------------------------------------------------------------- host page pool (include/tq4_pages.h)
+def tq4_pages_create(num_pages: int) -> int:
+    out = _p()
+    _check(_lib.tq4_pages_create(num_pages, ctypes.byref(out)), "tq4_pages_create")
+    return out.value
+
+
+def tq4_pages_destroy(pp: int) -> None:
+    _check(_lib.tq4_pages_destroy(pp), "tq4_pages_destroy")
+
+
+def tq4_pages_reservation(prompt_len: int, out_budget: int) -> int:
+    return _lib.tq4_pages_reservation(prompt_len, out_budget)
+
+
+def tq4_pages_admit(pp, prompt_len, out_budget, src_req=-1, prefix_len=0):
+    """Returns (status, request id, copy_src, copy_dst); the id is -1 unless status is TQ4_OK."""
+    req, cs, cd = _i32(-1), _i32(-1), _i32(-1)
+    rc = _lib.tq4_pages_admit(pp, prompt_len, out_budget, src_req, prefix_len, ctypes.byref(req),
+                              ctypes.byref(cs), ctypes.byref(cd))
+    return rc, (req.value if rc == TQ4_OK else -1), cs.value, cd.value
+
+
+def tq4_pages_grow(pp, req, new_len) -> int:
+    return _lib.tq4_pages_grow(pp, req, new_len)
+
+
+def tq4_pages_finish(pp, req) -> int:
+    return _lib.tq4_pages_finish(pp, req)
+
+
+def tq4_pages_step_boundary(pp) -> int:
+    return _lib.tq4_pages_step_boundary(pp)
+
+
+def tq4_pages_table(pp, req, max_pages):
+    """Returns (status, page-table row as a list of max_pages ids padded with -1, length)."""
+    row = (_i32 * max(max_pages, 1))()
+    n, ln = _i32(0), _i64(0)
+    rc = _lib.tq4_pages_table(pp, req, ctypes.cast(row, _p), max_pages, ctypes.byref(n), ctypes.byref(ln))
+    return rc, list(row)[:max_pages], ln.value
+
+
+def tq4_pages_free_count(pp) -> int:
+    return _lib.tq4_pages_free_count(pp)
+
+
+def tq4_pages_available(pp) -> int:
+    return _lib.tq4_pages_available(pp)
+
+
+def tq4_pages_refcount(pp, page) -> int:
+    return _lib.tq4_pages_refcount(pp, page)
+
+
+def tq4_pages_free_list(pp):
+    n = _lib.tq4_pages_free_list(pp, None, 0)
+    buf = (_i32 * max(n, 1))()
+    _lib.tq4_pages_free_list(pp, ctypes.cast(buf, _p), n)
+    return list(buf)[:n]
+
+
+class PagePool:
+    """Owns a tq4_pages handle (host page pool; no GPU involved)."""
+
+    def __init__(self, num_pages: int):
+        self.num_pages = num_pages
+        self.handle = tq4_pages_create(num_pages)
+
+    def __del__(self, _destroy=_lib.tq4_pages_destroy):   # bound early: safe at interpreter exit
+        if getattr(self, "handle", None):
+            _destroy(self.handle)
+            self.handle = None
+
+    def admit(self, prompt_len, out_budget, src_req=-1, prefix_len=0):
+        return tq4_pages_admit(self.handle, prompt_len, out_budget, src_req, prefix_len)
+
+    def grow(self, req, new_len):
+        return tq4_pages_grow(self.handle, req, new_len)
+
+    def finish(self, req):
+        return tq4_pages_finish(self.handle, req)
+
+    def step_boundary(self):
+        return tq4_pages_step_boundary(self.handle)
+
+    def table(self, req, max_pages):
+        return tq4_pages_table(self.handle, req, max_pages)
+
+    def free_count(self):
+        return tq4_pages_free_count(self.handle)
+
+    def available(self):
+        return tq4_pages_available(self.handle)
+
+    def refcount(self, page):
+        return tq4_pages_refcount(self.handle, page)
+
+    def free_list(self):
+        return tq4_pages_free_list(self.handle)
 
 
 # ---------------------------------------------------------------- tensor-level helpers

@@ -69,6 +69,7 @@ extern "C" {
 #define TQ4_ERR_WORKSPACE     -5  /* workspace missing or smaller than required    */
 #define TQ4_ERR_SEQ           -6  /* device-side sequence length check failed      */
 #define TQ4_ERR_TIMEOUT       -7  /* a bounded device-side wait gave up            */
+#define TQ4_ERR_NO_PAGES      -8  /* page pool: not enough capacity (tq4_pages.h)  */
 
 #define TQ4_HEAD_DIM        256
 #define TQ4_PAGE_POSITIONS  256

@@ -1,8 +1,9 @@
-"""The C ABI without a GPU: libtq4.so loads, exports every function include/tq4.h
-declares, the Python binding names exactly those, and the host-only parts
+"""The C ABI without a GPU: libtq4.so loads, exports every function the headers in
+include/ declare, the Python binding names exactly those, and the host-only parts
 (status strings, workspace sizes, argument checks that return before any CUDA
 call) behave as the header states."""
 import ctypes
+import glob
 import os
 import re
 
@@ -10,14 +11,17 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "tq4.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 tq4 = pytest.importorskip("compressed_paged_kv_tq4_b200.tq4")
 
 
 def header_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)   # drop comments
-    return sorted(set(re.findall(r"\b(tq4_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", " ", open(h).read(), flags=re.S)   # drop comments
+        names |= set(re.findall(r"\b(tq4_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 def header_defines():
@@ -26,6 +30,7 @@ def header_defines():
 
 
 def test_header_declares_the_calls():
+    assert [os.path.basename(h) for h in HEADERS] == ["tq4.h", "tq4_pages.h"]
     names = header_functions()
     for required in ("tq4_encode_append", "tq4_decode_attention", "tq4_prefill_attention",
                      "tq4_decode_append_attention", "tq4_reconstruct", "tq4_get_status"):
@@ -50,7 +55,7 @@ def test_constants_match_header():
     assert d["TQ4_POSITION_BYTES"] == tq4.POSITION_BYTES == 1040
     assert d["TQ4_DTYPE_F32"] == tq4.DTYPE_F32 and d["TQ4_DTYPE_BF16"] == tq4.DTYPE_BF16
     for name in ("TQ4_OK", "TQ4_ERR_ARG", "TQ4_ERR_PAGE_RANGE", "TQ4_ERR_WORKSPACE", "TQ4_ERR_SEQ",
-                 "TQ4_ERR_TIMEOUT"):
+                 "TQ4_ERR_TIMEOUT", "TQ4_ERR_NO_PAGES"):
         assert getattr(tq4, name) == d[name]
 
 
