@@ -32,7 +32,8 @@
  *                [262144, 264192)  K norms  [4 heads][256 slots] fp16
  *                [264192, 266240)  V norms  [4 heads][256 slots] fp16
  *              Position p of a request lives in page page_table[p / 256],
- *              slot p % 256. Page tables are int32 physical page ids.
+ *              slot p % 256. Page tables are int32 physical page ids; the
+ *              host page pool of tq4_pages.h can supply them.
  *
  * Memory: the caller owns every buffer. Pointers documented as "device" must be
  * device memory (or managed memory) of the current device; "host" pointers are
