@@ -228,7 +228,13 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
 
   // ---- lane 0 of each warp streams the warp's tiles: tile w + 8k -> buffer w*2 + k%2
   auto tile_pos = [&](int k) { return pos_b + (w + k * kQ1Warps) * kQ1Tile; };
-  auto issue_tile = [&](int k) {
+  // page id of tile k of this warp, loaded one iteration before its copy is issued
+  // (a warp's consecutive tiles are one page apart); -1 past the table
+  auto tile_page = [&](int k) -> int32_t {
+    const int c = tile_pos(k);
+    return (k < my_tiles && (c >> 8) < p.max_pages) ? __ldg(table + (c >> 8)) : -1;
+  };
+  auto issue_tile = [&](int k, int32_t page) {
     if (lane == 0 && k < my_tiles) {
       const int c = tile_pos(k);
       const int b = w * kQ1Stages + (k % kQ1Stages);
@@ -239,7 +245,6 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         }
         if (spins >= kQ1SpinLimit) record_error(p.status, TQ4_ERR_TIMEOUT);
       }
-      int page = k == 0 ? page_first : __ldg(table + (c >> 8));
       if (page < 0 || page >= p.num_pages) {
         record_error(p.status, TQ4_ERR_PAGE_RANGE);
         page = 0;   // still complete the barrier (reading page 0); the tile is masked below
@@ -257,7 +262,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   };
   if (encoder) fused_load();
   if (encode_first) fused_encode();
-  issue_tile(0);
+  issue_tile(0, page_first);
+  int32_t page_next = tile_page(1);
 
   // ---- q' = R q * scale for the 6 query heads of this KV head, split hi + lo, virtual order
   {
@@ -318,7 +324,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   bool timed_out = false;
 
   for (int k = 0; k < my_tiles; ++k) {
-    issue_tile(k + 1);
+    issue_tile(k + 1, page_next);
+    page_next = tile_page(k + 2);   // used by the next iteration's copy
     const int b = w * kQ1Stages + (k % kQ1Stages);
     const uint32_t bar = base + kQ1BarOff + b * 8;
     {
