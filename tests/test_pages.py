@@ -214,3 +214,38 @@ def test_host_throughput():
         out[name] = len(ops) / (time.perf_counter() - t0)
     print(f"page pool ops/s through the Python binding: library {out['library']:.3g}, model {out['model']:.3g}")
     assert np.isfinite(out["library"]) and out["library"] > 0
+
+
+def test_concurrent_callers_keep_the_invariants():
+    """Four threads admit, grow and finish their own requests on one pool; the lock
+    keeps every page either free or referenced exactly as often as tables hold it."""
+    import threading
+
+    pool = tq4.PagePool(64)
+    errors = []
+
+    def worker(seed):
+        rng = random.Random(seed)
+        try:
+            for _ in range(300):
+                rc, req, _, _ = pool.admit(rng.randrange(1, 700), rng.randrange(0, 300))
+                if rc != 0:
+                    continue
+                for _ in range(rng.randrange(1, 4)):
+                    pool.grow(req, rng.randrange(0, 900))
+                assert pool.finish(req) == 0
+                if rng.random() < 0.5:
+                    pool.step_boundary()
+        except Exception as e:   # reported below; a thread cannot fail the test directly
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(s,)) for s in range(4)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+    pool.step_boundary()
+    assert pool.free_count() == 64 and pool.available() == 64
+    assert sorted(pool.free_list()) == list(range(64))
+    assert all(pool.refcount(p) == 0 for p in range(64))
