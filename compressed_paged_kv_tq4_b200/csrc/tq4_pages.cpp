@@ -10,6 +10,7 @@
 // request its page table, length, reservation and the pages it took itself.
 // Every call validates first and then mutates, so a failed call changes nothing.
 #include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <deque>
 #include <map>
@@ -114,6 +115,7 @@ int tq4_pages_admit(tq4_pages* pp, int64_t prompt_len, int64_t out_budget, int32
   // (or, if the reservation is zero, out of unreserved capacity)
   const int64_t need = std::max<int64_t>(reserve, copied);
   if (need > pp->available()) return TQ4_ERR_NO_PAGES;
+  if (pp->next_id == INT32_MAX) return TQ4_ERR_ARG;   // request ids are never reused
 
   Request r;
   r.reserve = reserve;

@@ -78,7 +78,8 @@ int64_t tq4_pages_reservation(int64_t prompt_len, int64_t out_budget);
  * full pages are shared, a partial last page is copied. *copy_src and *copy_dst
  * (both may be NULL when src_req < 0) receive the page copy to perform, or -1.
  * prompt_len counts the restored positions too (prefix_len <= prompt_len).
- * TQ4_ERR_NO_PAGES if the reservation does not fit the available capacity. */
+ * TQ4_ERR_NO_PAGES if the reservation does not fit the available capacity;
+ * TQ4_ERR_ARG once 2^31 - 1 ids have been handed out. */
 int tq4_pages_admit(tq4_pages* pp, int64_t prompt_len, int64_t out_budget, int32_t src_req, int64_t prefix_len,
                     int32_t* req_out, int32_t* copy_src, int32_t* copy_dst);
 
