@@ -60,3 +60,24 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     args = types.SimpleNamespace(workload="decode_32k", steps=1, warmup=0, gpus=2)
     bench.run_reference(args, rank=1)      # returns before building anything
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_the_contract_line(capsys):
+    """Rank 0 times the oracle on a bounded sample and prints one JSON line with the
+    arm's keys and the same workload config as the CUDA arm."""
+    import json
+
+    args = types.SimpleNamespace(workload="single_layer_2k", steps=1, warmup=0, gpus=1)
+    bench.run_reference(args, rank=0)
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["value"] > 0 and line["higher_is_better"] is True and line["n_gpus"] == 1
+    cfg = dict(line["config"])
+    cfg.pop("sample")
+    assert cfg == bench.workload_config("single_layer_2k", 1)
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
