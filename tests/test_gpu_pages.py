@@ -1,7 +1,8 @@
 """Page tables from the host page pool drive the CUDA path: two requests, the
 second restoring a prefix of the first (full pages shared by reference, the
-partial page copied on the device), appended and decoded in one call, against
-the fp64 oracle built on the same tables and the same page copy."""
+partial page copied on the device) and appending its own positions, then both
+decoded in one call, against the fp64 oracle built on the same tables and the
+same page copy."""
 import numpy as np
 import pytest
 
