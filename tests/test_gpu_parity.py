@@ -186,6 +186,32 @@ def test_decode_variants_parity(seq_lens, n_q, shared):
     H.assert_bf16_close(got, exp, f"decode {seq_lens} n_q={n_q}")
 
 
+@pytest.mark.parametrize("n_q", [1, 4])
+def test_decode_split_count_invariance(n_q):
+    """The host bound total_seq_len sets the split length: a looser bound gives fewer,
+    longer splits. Both plans must give the same attention (fp32 outputs, to the fp32
+    tolerance), and both must match the oracle."""
+    case = Case(11, [5000], n_q, outliers=0.05, chunks=(777,))
+    q = I.queries(11, 0, (1, n_q, 24, 256))
+    qt = _bf16_tensor(q)
+    pool = torch.from_numpy(case.opool).cuda()
+    width = 160                                  # table wider than the request: room for a loose bound
+    tab = np.full((1, width), -1, np.int32)
+    tab[0, :case.tab.shape[1]] = case.tab[0]
+    tt, seq = torch.from_numpy(tab).cuda(), torch.from_numpy(case.seq_lens).cuda()
+    outs = []
+    for total in (5000, width * 256):            # 20 splits of 256 positions, then 5 of 1,152
+        outs.append(case.ctx.decode_attention(pool, qt, tt, seq, total, SCALE, out_dtype=torch.float32)
+                    .cpu().numpy())
+    torch.cuda.synchronize()
+    assert case.ctx.status() == tq4.TQ4_OK
+    exp = case.oracle_decode(q)
+    tol = H.F32_ABS_TOL * max(1.0, np.abs(exp).max())
+    assert np.abs(outs[0] - outs[1]).max() <= tol
+    for got in outs:
+        assert np.abs(got - exp).max() <= tol
+
+
 def test_decode_page_table_permutation_invariance():
     """The same logical history through two different page tables gives identical GPU output."""
     ctx = tq4.Context(I.signs(8))
