@@ -212,6 +212,25 @@ def test_decode_split_count_invariance(n_q):
         assert np.abs(got - exp).max() <= tol
 
 
+def test_decode_first_of_four_tokens_equals_one_token_decode():
+    """Causal verify: query token 0 of an n_q = 4 call at length T sees [0, T-4], the
+    same history as a one-token call at length T-3 with the same query (fp32 outputs,
+    identical pool bytes; the two calls run different kernels)."""
+    case = Case(12, [3001], 4, outliers=0.05)
+    q4 = I.queries(12, 0, (1, 4, 24, 256))
+    pool = torch.from_numpy(case.opool).cuda()
+    tt = torch.from_numpy(case.tab).cuda()
+    out4 = case.ctx.decode_attention(pool, _bf16_tensor(q4), tt, torch.tensor([3001], dtype=torch.int32,
+                                     device="cuda"), 3001, SCALE, out_dtype=torch.float32).cpu().numpy()
+    out1 = case.ctx.decode_attention(pool, _bf16_tensor(np.ascontiguousarray(q4[:, :1])), tt,
+                                     torch.tensor([2998], dtype=torch.int32, device="cuda"), 2998, SCALE,
+                                     out_dtype=torch.float32).cpu().numpy()
+    torch.cuda.synchronize()
+    assert case.ctx.status() == tq4.TQ4_OK
+    tol = H.F32_ABS_TOL * max(1.0, np.abs(out1).max())
+    assert np.abs(out4[:, 0] - out1[:, 0]).max() <= tol
+
+
 def test_decode_page_table_permutation_invariance():
     """The same logical history through two different page tables gives identical GPU output."""
     ctx = tq4.Context(I.signs(8))
