@@ -391,7 +391,7 @@ class OracleSample:
         from oracle import tq4_oracle as O
         self.O, self.w = O, w
         self.signs = I.signs(w.config)
-        self.c, _ = O.stored_codebook()
+        self.c, _ = O.codebook()
         self.tables = I.request_tables(w)
         if w.kind == "decode":
             T = min(int(w.seq_lens[0]), 8192)

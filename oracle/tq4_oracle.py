@@ -24,10 +24,11 @@ What it computes, and where each step comes from (JustFit pages):
           a 24 GB Mac", mechanism table, row KVExec: rotated-domain attention.
 
 Readings where the pages are silent (each one is a choice, stated here):
- * codebook: 16-level Lloyd-Max quantiser for N(0, 1/256) coordinates, solved in
-   fp64 and stored as a table of 16 FP16 values (round to nearest even), the one
-   scalar type the format names (the norm is FP16); encode picks the nearest
-   stored centroid and decode looks the stored value up;
+ * codebook: 16-level Lloyd-Max quantiser for N(0, 1/256) coordinates, solved and
+   used in fp64: encode picks the nearest fp64 centroid (the decision boundaries
+   are the midpoints of adjacent centroids) and decode looks the fp64 value up.
+   How an implementation stores the table is its own affair; the oracle is the
+   definition;
  * rotation: R = H diag(s) / 16 with H the 256x256 Sylvester Hadamard matrix and
    s the seeded +-1 sign diagonal (signs applied first when rotating); the
    inverse is R^T = diag(s) H / 16;
@@ -100,13 +101,11 @@ def lloyd_max_gaussian(levels: int = LEVELS, sigma: float = 1.0 / 16.0,
     return c, 0.5 * (c[:-1] + c[1:])
 
 
-def stored_codebook(levels: int = LEVELS, sigma: float = 1.0 / 16.0):
-    """The codebook as stored by the format: fp16 (round to nearest even) of the
-    fp64 Lloyd-Max centroids, returned as float64 values, with the midpoints of
-    adjacent stored centroids as the nearest-centroid decision boundaries."""
-    c, _ = lloyd_max_gaussian(levels, sigma)
-    c16 = c.astype(np.float16).astype(np.float64)
-    return c16, 0.5 * (c16[:-1] + c16[1:])
+def codebook(levels: int = LEVELS, sigma: float = 1.0 / 16.0):
+    """The codebook encode and decode use: the fp64 Lloyd-Max centroids for
+    N(0, sigma^2) and, as nearest-centroid decision boundaries, the midpoints of
+    adjacent centroids (both float64)."""
+    return lloyd_max_gaussian(levels, sigma)
 
 
 def quantiser_mse(centroids, boundaries, sigma: float = 1.0 / 16.0) -> float:

@@ -39,7 +39,7 @@ def assert_bf16_close(got, expect, what=""):
 
 
 def oracle_codebook():
-    c, _ = O.stored_codebook()
+    c, _ = O.codebook()
     return c
 
 

@@ -85,7 +85,7 @@ def test_fused_append_against_oracle():
     out = ctx.decode_append_attention(pool, k_new, v_new, q, tabs, seq, 3000, SCALE, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert ctx.status() == tq4.TQ4_OK
-    c, _ = O.stored_codebook()
+    c, _ = O.codebook()
     # the oracle reads the GPU's pool bytes (history and the fused append alike)
     exp = O.decode_attention(pool.cpu().numpy(), tab, np.array(seq_lens),
                              I.bf16_bits_to_f32(qb).astype(np.float64), SCALE, signs, c)
@@ -97,7 +97,7 @@ def test_fused_append_against_oracle():
     gk, gv, gkn, gvn = O._regions(pool.cpu().numpy())
     ok_, ov_, okn, ovn = O._regions(opool)
     pg, sl = tab[0][2999 // 256], 2999 % 256
-    _, b = O.stored_codebook()
+    _, b = O.codebook()
     H.check_words_against_oracle(gk[pg, :, sl][None], ok_[pg, :, sl][None], yk, b, "K words")
     H.check_words_against_oracle(gv[pg, :, sl][None], ov_[pg, :, sl][None], yv, b, "V words")
 

@@ -44,7 +44,7 @@ def _random_pool(w, layer=0):
 
 @pytest.fixture(scope="module")
 def codebook():
-    return O.stored_codebook()
+    return O.codebook()
 
 
 @pytest.mark.parametrize("name", ["decode_32k", "decode_213k_outliers", "verify_2req_229k"])

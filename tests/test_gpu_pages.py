@@ -24,7 +24,7 @@ CFG = 21
 
 def test_decode_over_pool_tables_with_restored_prefix():
     signs = I.signs(CFG)
-    c, _ = O.stored_codebook()
+    c, _ = O.codebook()
     ctx = tq4.Context(signs)
     n_pages, max_pages = 12, 6
     pp = tq4.PagePool(n_pages)

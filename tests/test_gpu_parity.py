@@ -33,7 +33,7 @@ def _pool_view(pool_bytes):
 
 @pytest.fixture(scope="module")
 def codebook():
-    return O.stored_codebook()
+    return O.codebook()
 
 
 class Case:
@@ -42,7 +42,7 @@ class Case:
     def __init__(self, config, seq_lens, n_q, shared_pages=0, outliers=0.0, chunks=(1000,)):
         self.signs = I.signs(config)
         self.ctx = tq4.Context(self.signs)
-        self.c, self.b = O.stored_codebook()
+        self.c, self.b = O.codebook()
         npg = [(s + 255) // 256 for s in seq_lens]
         total_pages = npg[0] + sum(n - shared_pages for n in npg[1:]) + 3
         ids = I.page_table_scattered(config, total_pages, total_pages)

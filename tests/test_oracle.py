@@ -30,8 +30,8 @@ def solution():
 
 @pytest.fixture(scope="module")
 def codebook():
-    """The stored (fp16) codebook that encode/decode use."""
-    return O.stored_codebook()
+    """The codebook that encode/decode use (fp64 centroids, midpoint boundaries)."""
+    return O.codebook()
 
 
 @pytest.fixture(scope="module")
@@ -100,16 +100,16 @@ def test_codebook_symmetric_and_midpoints(solution):
     assert np.allclose(b, 0.5 * (c[1:] + c[:-1]), atol=0, rtol=0)
 
 
-def test_stored_codebook_is_fp16_of_solution(solution, codebook):
-    c, _ = solution
-    c16, b16 = codebook
-    for x, y in zip(c, c16):
-        assert np.float16(x) == y                       # round to nearest even of the fp64 value
-        assert abs(y - x) <= abs(x) * 2.0 ** -11        # within half an fp16 ulp (relative)
-    assert np.array_equal(c16, -c16[::-1])              # symmetric exactly after rounding
-    assert np.array_equal(b16, 0.5 * (c16[1:] + c16[:-1]))
-    # rounding the table costs nothing measurable in distortion
-    assert abs(O.quantiser_mse(c16 * 16, b16 * 16, 1.0) - O.quantiser_mse(c * 16, 0.5 * (c[1:] + c[:-1]) * 16, 1.0)) < 1e-6
+def test_codebook_used_is_the_fp64_solution(solution, codebook):
+    """Encode and decode use the fp64 Lloyd-Max centroids themselves (no rounding
+    of the table) and the midpoints of adjacent centroids as boundaries."""
+    c, b = solution
+    cu, bu = codebook
+    assert cu.dtype == np.float64 and bu.dtype == np.float64
+    assert np.array_equal(cu, c) and np.array_equal(bu, b)
+    # a table rounded to fp16 (or bf16) is a different table: it fails this pin
+    assert not np.array_equal(cu, c.astype(np.float16).astype(np.float64))
+    assert np.max(np.abs(cu - c.astype(np.float16).astype(np.float64))) > 1e-5
 
 
 def test_codebook_centroids_are_monte_carlo_conditional_means(solution):
