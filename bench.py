@@ -1,15 +1,21 @@
 #!/usr/bin/env python
 """Benchmark of the TQ4 paged-KV attention path on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--extra LIST]
+                    [--impl ours|reference]
 
 One step = one pass of the whole hot path over one batch: for every layer,
 tq4_decode_append_attention (the step's new K/V positions appended, then decode
 attention over the whole history; with one query token the append runs inside
 the decode kernel) for decode workloads, or tq4_prefill_attention followed by
-tq4_encode_append of the chunk (prefill workload). The step's launches are captured once in a CUDA
-graph through the public C ABI and replayed; the timed region is exactly K
-replays between CUDA events, after W warm-up replays.
+tq4_encode_append of the chunk (prefill workload). The step's launches are
+captured once in a CUDA graph through the public C ABI and replayed; the timed
+region is exactly K replays between CUDA events, after W warm-up replays.
+
+The headline line is the `--workload` (decode_32k by default, 16 layers of
+32,768 positions). The other workloads (`--extra`: the three others and the INT8 arm by default) are
+measured in the same run the same way, with as many timed steps as fit in about
+two seconds (at most K), and reported under "workloads" in the same JSON line.
 
 Prints one JSON line. Multi-GPU runs (torchrun) are independent replicas: the
 path has no exchange step, every rank runs the same workload on its own GPU
@@ -18,7 +24,6 @@ and the value is the units of all ranks over the slowest rank's time.
 from __future__ import annotations
 
 import argparse
-import concurrent.futures as cf
 import json
 import os
 import statistics
@@ -36,29 +41,35 @@ from compressed_paged_kv_tq4_b200 import inputs as I  # noqa: E402
 METRIC = "TQ4 fused attention KV positions/s & HBM GB/s (% of roofline) at 32K–229K ctx"
 UNIT = "KV positions/s"
 SCALE = 1.0 / 16.0
+EXTRA_DEFAULT = "decode_213k_outliers,verify_2req_229k,prefill_2k_on_32k,int8_decode_32k"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="decode_32k", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--extra", default=EXTRA_DEFAULT,
+                    help="comma-separated workloads measured after the headline one ('none' for none)")
+    ap.add_argument("--extra-seconds", type=float, default=2.0, help="timed seconds per extra workload (about)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch without a CUDA graph (profiling)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
     ap.add_argument("--profile", action="store_true",
-                    help="eager steps only: no roofline replay, e2e or CPU leg (for ncu captures)")
-    return ap.parse_args()
+                    help="eager steps of the one workload only: no roofline replay, e2e or CPU leg (ncu captures)")
+    return ap.parse_args(argv)
 
 
 def peaks():
+    """(hbm GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", 0)), "measured"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained") or d["bf16_tflops"]), "measured")
     except Exception:
         return 6650.0, 1590.0, 1400.0, "fallback"
 
@@ -70,16 +81,19 @@ WORKLOAD_DESC = {
                         "16 layers",
     "prefill_2k_on_32k": "2,048 causal bf16 query tokens on a 32,768-position TQ4 prefix + the chunk, 16 layers",
     "single_layer_2k": "1 layer, 2,048 TQ4 positions, 1 query token",
+    "int8_decode_32k": "uniform INT8 comparison arm: 16 layers x 32,768 INT8 positions (2,064 B per "
+                       "layer-position), 1 request, 1 bf16 query token, append of 1 position per layer",
 }
 
 
 def workload_config(name, world):
     """The `config` object of the JSON line (the same for both arms)."""
     w = I.WORKLOADS[name]
+    per_pos = 2064 if w.kind == "decode_int8" else 1040
     return {"workload": f"{name}: {WORKLOAD_DESC[name]}", "append_per_layer": w.append_per_step,
             "pool_pages": w.pool_pages, "page_positions": 256,
             "l2": "inputs larger than L2: packed KV read per step is "
-                  f"{w.layers * sum(w.seq_lens) * 1040 / 1e6:.0f} MB vs 126 MB L2",
+                  f"{w.layers * sum(w.seq_lens) * per_pos / 1e6:.0f} MB vs 126 MB L2",
             "parallelism": f"replicas x{world}"}
 
 
@@ -87,19 +101,7 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
 # (summarised under profiles/), per unit of work. A figure counts only while the
 # kernel's source file hashes to the value it had when the counters were taken.
-MEASURED_TRAFFIC = {
-    # decode_q1_kernel, decode_32k capture (append fused): 34,172,160 B read + 77,312 B
-    # written for 32,768 positions; its traffic grows with the positions it streams
-    "decode_q1": ("tq4_decode_q1.cuh", "a1aa9c992fe1114efe87749225ea10ca9eca128a3d97914e4c08bafae57d9706",
-                  (34_172_160 + 77_312) / 32_768),
-    # decode_splitk_kernel<3>, verify_2req_229k capture: 221,675,264 B read + 3,709,696 B
-    # written for 229,376 positions (the 64 shared pages partly hit in L2: this workload only)
-    "decode_splitk": ("tq4_decode.cuh", "d27dcffa6032aeb25c0c742e6ca77347597bf628fd34c9a1f3d0b6a41afc0340",
-                      (221_675_264 + 3_709_696) / 229_376),
-    # prefill_tc_kernel, prefill_2k_on_32k capture: one launch
-    "prefill_tc": ("tq4_prefill_tc.cuh", "f290435adb0de7f5ccb086652cf386f89fbab4a08afeb143fa73615e1aa92529",
-                   93_480_960 + 9_271_552),
-}
+MEASURED_TRAFFIC = {}
 
 
 def measured_traffic(key, units):
@@ -184,27 +186,7 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
-# ---------------------------------------------------------------------------- host data
-def gen_kv_parallel(config, layer, n, first_pos, request, outliers, workers=16):
-    """Same values as inputs.kv_vectors, generated in page-aligned blocks on several threads."""
-    k = np.empty((n, 4, 256), np.float32)
-    v = np.empty((n, 4, 256), np.float32)
-    if n == 0:
-        return k, v
-    blk = 64 * 256
-    starts = list(range(first_pos - first_pos % 256, first_pos + n, blk))
-
-    def job(s):
-        lo, hi = max(s, first_pos), min(s + blk, first_pos + n)
-        kk, vv = I.kv_vectors(config, layer, hi - lo, first_pos=lo, request=request, outlier_frac=outliers)
-        k[lo - first_pos:hi - first_pos] = kk
-        v[lo - first_pos:hi - first_pos] = vv
-
-    with cf.ThreadPoolExecutor(workers) as ex:
-        list(ex.map(job, starts))
-    return k, v
-
-
+# ---------------------------------------------------------------------------- device data
 class Arena:
     """One contiguous device buffer carved into aligned tensors, with a pinned host mirror."""
 
@@ -233,6 +215,11 @@ class Arena:
 
 
 class DecodeSetup:
+    """One decode workload on the device: every layer's pool (history encoded by
+    tq4_encode_append from K/V drawn on the device with the workload's law), page
+    tables, lengths, and the step's inputs (queries, new K/V) and outputs in one
+    arena with a pinned host mirror."""
+
     def __init__(self, w, torch, tq4, device):
         self.w, self.torch, self.tq4 = w, torch, tq4
         self.signs = I.signs(w.config)
@@ -253,15 +240,12 @@ class DecodeSetup:
             for r in range(w.n_req):
                 first = w.shared_prefix_pages * 256 if r > 0 else 0
                 s = int(self.seq_np[r])
-                k, v = gen_kv_parallel(w.config, layer, s - first, first, r, w.outlier_frac)
-                tt = self.tables[r]
+                k, v = I.kv_vectors_device(w.config, layer, s - first, request=r, outlier_frac=w.outlier_frac,
+                                           device=device)
                 hist = s - w.n_q - first  # history already in the cache; the last n_q are the step's appends
-                for a in range(0, hist, 32768):
-                    e = min(a + 32768, hist)
-                    self.ctx.encode_append(pool, tt, first + a, torch.from_numpy(k[a:e]).to(device),
-                                           torch.from_numpy(v[a:e]).to(device))
-                knew_l.append(np.ascontiguousarray(k[hist:]))
-                vnew_l.append(np.ascontiguousarray(v[hist:]))
+                self.ctx.encode_append(pool, self.tables[r], first, k[:hist], v[:hist])
+                knew_l.append(k[hist:].cpu().numpy())
+                vnew_l.append(v[hist:].cpu().numpy())
                 del k, v
             # the step's new K/V of all requests: [n_req, n_q, 4, 256] fp32
             ki.append(ain.add(np.stack(knew_l), torch.float32, (w.n_req, w.n_q, 4, 256)))
@@ -303,15 +287,98 @@ class DecodeSetup:
         # decode + combine per layer; with n_q > 1 a tail-encode kernel as well
         return self.w.layers * (2 if self.w.n_q == 1 else 3)
 
-    def dominant_bytes(self):
-        """Algorithmic bytes of one decode launch: the packed history it must read."""
-        return self.total * I.H_KV * 2 * 130
+    def roofline(self, att_ms, peaks_):
+        """Dominant call: one layer's tq4_decode_append_attention; algorithmic bytes =
+        the packed history it must read (1,040 B per attended layer-position)."""
+        hbm = peaks_[0]
+        nbytes = self.total * I.H_KV * 2 * 130
+        ach = nbytes / (att_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": measured_traffic("decode_q1" if self.w.n_q == 1 else "decode_splitk", self.total),
+                "kernel": "tq4_decode_append_attention (split-K decode with the append inside it for one "
+                          "query token + combine)",
+                "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms,
+                "peak_source": f"{peaks_[3]} hbm_gbs"}
 
     def h2d_d2h(self):
         return self.arena_in.nbytes, self.arena_out.nbytes
 
+    def tokens_per_step(self):
+        return self.w.n_req * self.w.n_q
+
+
+class Int8DecodeSetup(DecodeSetup):
+    """The uniform INT8 comparison arm on a decode workload: each layer's pool holds
+    the INT8-encoded history; a step appends the new position with
+    tq4_int8_encode_append and runs tq4_int8_decode_attention, per layer."""
+
+    def __init__(self, w, torch, tq4, device):
+        self.w, self.torch, self.tq4 = w, torch, tq4
+        self.ctx = tq4.Context(I.signs(w.config))
+        self.tables_np = I.request_tables(w)
+        self.tables = torch.from_numpy(self.tables_np).to(device)
+        self.seq_np = np.array(w.seq_lens, np.int32)
+        self.seq = torch.from_numpy(self.seq_np).to(device)
+        self.total = int(self.seq_np.sum())
+        self.start = int(self.seq_np[0]) - w.n_q
+        if w.n_req != 1:
+            raise ValueError("the INT8 arm's bench workload has one request")
+        self.pools = []
+        self.ws = self.ctx.decode_workspace(w.n_req, w.n_q, self.total, device)
+        ain, aout = Arena(torch, device), Arena(torch, device)
+        qi, ki, vi, oi = [], [], [], []
+        for layer in range(w.layers):
+            pool = tq4.Context.new_int8_pool(w.pool_pages, device)
+            k, v = I.kv_vectors_device(w.config, layer, self.total, outlier_frac=w.outlier_frac, device=device)
+            self.ctx.int8_encode_append(pool, self.tables[0], 0, k[:self.start], v[:self.start])
+            ki.append(ain.add(k[self.start:].cpu().numpy(), torch.float32, (w.n_q, 4, 256)))
+            vi.append(ain.add(v[self.start:].cpu().numpy(), torch.float32, (w.n_q, 4, 256)))
+            del k, v
+            qb = I.queries(w.config, layer, (1, w.n_q, 24, 256))
+            qi.append(ain.add(qb, torch.bfloat16, (1, w.n_q, 24, 256)))
+            oi.append(aout.add(np.zeros((1, w.n_q, 24, 256), np.uint16), torch.bfloat16, (1, w.n_q, 24, 256)))
+            self.pools.append(pool)
+        vin, vout = ain.finalize(), aout.finalize()
+        self.arena_in, self.arena_out = ain, aout
+        self.qs = [vin[i] for i in qi]
+        self.knew = [vin[i] for i in ki]
+        self.vnew = [vin[i] for i in vi]
+        self.outs = [vout[i] for i in oi]
+        torch.cuda.synchronize()
+        if self.ctx.status() != tq4.TQ4_OK:
+            raise RuntimeError("INT8 cache build failed")
+
+    def attend(self, layer):
+        """The step's append and decode of one layer: two calls on the INT8 arm."""
+        tq4, w = self.tq4, self.w
+        rc = tq4.tq4_int8_encode_append(self.ctx.handle, self.pools[layer], w.pool_pages, self.tables[0],
+                                        self.tables.shape[1], self.start, w.n_q, self.knew[layer], self.vnew[layer],
+                                        tq4.DTYPE_F32)
+        assert rc == 0, rc
+        rc = tq4.tq4_int8_decode_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.qs[layer],
+                                           self.tables, self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total,
+                                           SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
+        assert rc == 0, rc
+
+    def kernels_per_step(self):
+        return self.w.layers * 3   # encode, decode, combine
+
+    def roofline(self, att_ms, peaks_):
+        """Dominant call: one layer's append + INT8 decode; algorithmic bytes = the INT8
+        history it must read (2,064 B per attended layer-position)."""
+        hbm = peaks_[0]
+        nbytes = self.total * I.H_KV * 2 * 258
+        ach = nbytes / (att_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": None, "kernel": "tq4_int8_encode_append + tq4_int8_decode_attention (split-K + combine)",
+                "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms, "peak_source": f"{peaks_[3]} hbm_gbs"}
+
 
 class PrefillSetup:
+    """The prefill workload on the device: every layer's pool holds the TQ4 prefix
+    (encoded from K/V drawn on the device); the chunk's queries and K/V are seeded
+    bf16 inputs in an arena with a pinned host mirror."""
+
     def __init__(self, w, torch, tq4, device):
         self.w, self.torch, self.tq4 = w, torch, tq4
         self.signs = I.signs(w.config)
@@ -325,11 +392,8 @@ class PrefillSetup:
         idx = []
         for layer in range(w.layers):
             pool = tq4.Context.new_pool(w.pool_pages, device)
-            k, v = gen_kv_parallel(w.config, layer, self.P, 0, 0, w.outlier_frac)
-            for a in range(0, self.P, 32768):
-                e = min(a + 32768, self.P)
-                self.ctx.encode_append(pool, self.table, a, torch.from_numpy(k[a:e]).to(device),
-                                       torch.from_numpy(v[a:e]).to(device))
+            k, v = I.kv_vectors_device(w.config, layer, self.P, outlier_frac=w.outlier_frac, device=device)
+            self.ctx.encode_append(pool, self.table, 0, k, v)
             del k, v
             qb = I.queries(w.config, layer, (self.n, 24, 256))
             kb, vb = I.chunk_kv(w.config, layer, self.n)
@@ -352,7 +416,7 @@ class PrefillSetup:
         tq4, w = self.tq4, self.w
         rc = tq4.tq4_prefill_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.table,
                                        self.table.numel(), self.P, self.q[layer], self.kc[layer], self.vc[layer],
-                                       self.n, SCALE, self.outs[layer], self.ws, self.ws.numel())
+                                       self.n, SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
         assert rc == 0, rc
 
     def append(self, layer):
@@ -374,29 +438,62 @@ class PrefillSetup:
     def kernels_per_step(self):
         return self.w.layers * 3
 
-    def dominant_flops(self):
-        """Algorithmic FLOPs of one prefill launch (QK^T and PV, causal part only)."""
+    def roofline(self, att_ms, peaks_):
+        """Dominant call: one layer's tq4_prefill_attention; algorithmic FLOPs =
+        2 * 2 * 256 per visible (query row, position) pair (QK^T and PV, causal part
+        only). The attention launches are timed back to back for tens of ms, so the
+        sustained bf16 figure is the peak."""
         att = self.n * self.P + self.n * (self.n + 1) // 2
-        return 2 * 2 * 24 * 256 * att
+        flops = 2 * 2 * 24 * 256 * att
+        ach = flops / (att_ms * 1e-3) / 1e12
+        sus, burst = peaks_[2], peaks_[1]
+        return {"bound": "tensor", "achieved": ach, "peak": sus, "unit": "TFLOP/s", "frac": ach / sus,
+                "frac_of_burst_peak": ach / burst, "peak_burst": burst,
+                "traffic": measured_traffic("prefill_tc", 1) if self.w.name == "prefill_2k_on_32k" else None,
+                "kernel": "tq4_prefill_attention (rotate prologue + tcgen05 attention kernel)",
+                "algorithmic_flops_per_launch": flops, "launch_ms": att_ms,
+                "peak_source": f"{peaks_[3]} bf16_tflops_sustained (f16 operands: same nominal rate)"}
 
     def h2d_d2h(self):
         return self.arena_in.nbytes, self.arena_out.nbytes
 
+    def tokens_per_step(self):
+        return self.n
+
 
 # ---------------------------------------------------------------------------- CPU oracle legs
+def _oracle_kv(config, n, outliers):
+    """The workload's K/V for positions [0, n) from the numpy generator, a page-aligned
+    block at a time on a few threads (same values as inputs.kv_vectors)."""
+    import concurrent.futures as cf
+    k = np.empty((n, 4, 256), np.float32)
+    v = np.empty((n, 4, 256), np.float32)
+    blk = 64 * 256
+
+    def job(s):
+        e = min(s + blk, n)
+        k[s:e], v[s:e] = I.kv_vectors(config, 0, e - s, first_pos=s, outlier_frac=outliers)
+
+    with cf.ThreadPoolExecutor(8) as ex:
+        list(ex.map(job, range(0, n, blk)))
+    return k, v
+
+
 class OracleSample:
     """The oracle on one layer of the workload (a bounded sample); state is built once."""
 
-    def __init__(self, w):
+    def __init__(self, w, decode_positions=8192):
         from oracle import tq4_oracle as O
         self.O, self.w = O, w
         self.signs = I.signs(w.config)
         self.c, _ = O.codebook()
         self.tables = I.request_tables(w)
+        if w.kind == "decode_int8":
+            raise ValueError("the oracle leg times the TQ4 workloads")
         if w.kind == "decode":
-            T = min(int(w.seq_lens[0]), 8192)
+            T = min(int(w.seq_lens[0]), decode_positions)
             self.T = T
-            self.k, self.v = gen_kv_parallel(w.config, 0, T, 0, 0, w.outlier_frac)
+            self.k, self.v = _oracle_kv(w.config, T, w.outlier_frac)
             self.pool = O.new_pool(w.pool_pages)
             O.encode_append(self.pool, self.tables[0], 0, self.k[:T - w.n_q], self.v[:T - w.n_q],
                             self.signs, self.c)
@@ -406,7 +503,7 @@ class OracleSample:
         else:
             P = min(w.prefix_len, 4096)
             self.P = P
-            k, v = gen_kv_parallel(w.config, 0, P, 0, 0, 0.0)
+            k, v = _oracle_kv(w.config, P, 0.0)
             self.pool = O.new_pool(w.pool_pages)
             O.encode_append(self.pool, self.tables[0], 0, k, v, self.signs, self.c)
             qb = I.queries(w.config, 0, (w.n_q, 24, 256))
@@ -428,10 +525,15 @@ class OracleSample:
         return int(sum(self.P + i + 1 for i in self.rows))
 
     @staticmethod
-    def threads():
+    def cores():
+        """Threads the oracle ran on: its fp64 matrix products use the BLAS pool; the
+        per-head attention loop is Python on one thread."""
         import threadpoolctl
         info = threadpoolctl.threadpool_info()
-        return max([d.get("num_threads", 1) for d in info] or [1])
+        blas = max([d.get("num_threads", 1) for d in info] or [1])
+        return {"cores": blas, "host_cores": os.cpu_count(),
+                "threads_note": f"{blas} BLAS threads for the fp64 matrix products (rotation, K q); the per-head "
+                                "attention loop runs on one Python thread"}
 
     def timed(self, seconds=10.0):
         self.one()
@@ -448,7 +550,9 @@ def run_reference(args, rank):
     if rank != 0:
         return
     w = I.WORKLOADS[args.workload]
-    orc = OracleSample(w)
+    # a decode step's sample shrinks with the step count so that the run stays within minutes
+    T = max(1024, min(8192, (8192 * 400 // max(1, args.steps + args.warmup)) // 256 * 256))
+    orc = OracleSample(w, decode_positions=T)
     for _ in range(args.warmup):
         orc.one()
     units, t0 = 0, time.perf_counter()
@@ -456,49 +560,27 @@ def run_reference(args, rank):
         units += orc.one()
     el = time.perf_counter() - t0
     value = units / el
-    threads = orc.threads()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / max(args.steps, 1) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded Gaussian K/V and queries)",
             "config": dict(workload_config(args.workload, args.gpus), sample=orc.sample),
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": orc.sample},
+            "cpu_baseline": dict({"value": value, "unit": UNIT, "kind": "oracle", "sample": orc.sample},
+                                 **orc.cores()),
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-# ---------------------------------------------------------------------------- main
-def main():
-    args = parse()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        run_reference(args, rank)
-        return
-
-    import torch
-    from compressed_paged_kv_tq4_b200 import tq4
-
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-
-    w = I.WORKLOADS[args.workload]
+# ---------------------------------------------------------------------------- GPU measurement
+def measure_workload(name, args, torch, tq4, device, dist, world, steps, headline):
+    """Build one workload, capture its step as a CUDA graph, time `steps` replays,
+    then the dominant attention call alone and the end-to-end path (graphed and eager)."""
+    w = I.WORKLOADS[name]
     if args.layers:
         import dataclasses
         w = dataclasses.replace(w, layers=args.layers)
-    if args.profile:
-        args.eager = True
-    S = DecodeSetup(w, torch, tq4, device) if w.kind == "decode" else PrefillSetup(w, torch, tq4, device)
+    S = {"decode": DecodeSetup, "decode_int8": Int8DecodeSetup, "prefill": PrefillSetup}[w.kind](w, torch, tq4, device)
     stream = torch.cuda.Stream(device)
-
-    # capture one step through the public ABI
     graph = None
     with torch.cuda.stream(stream):
         S.step()  # eager once (also the first warm-up)
@@ -509,35 +591,42 @@ def main():
                 S.step()
     torch.cuda.synchronize()
     run = graph.replay if graph is not None else S.step
-
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         for _ in range(max(args.warmup, 3)):
             run()
+        ev0.record(stream)
+        run()
+        ev1.record(stream)
     torch.cuda.synchronize()
+    if not headline:   # as many steps as fit in about --extra-seconds, at most K, at least 3
+        est = ev0.elapsed_time(ev1)
+        steps = int(max(3, min(steps, args.extra_seconds * 1e3 / max(est, 1e-3))))
     if dist:
+        t = torch.tensor([steps], dtype=torch.int64, device=device)   # every rank times the same steps
+        dist.all_reduce(t, op=dist.ReduceOp.MIN)
+        steps = int(t.item())
         dist.barrier()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
+    with ClockSampler(device.index) as clk:
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             ev0.record(stream)
-            for _ in range(args.steps):
+            for _ in range(steps):
                 run()
             ev1.record(stream)
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, device)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps, dist, device)
     if S.ctx.status() != tq4.TQ4_OK:
-        raise RuntimeError("device status error during timing")
-    value = job_value(S.units_per_step(), world, ms)
+        raise RuntimeError(f"{name}: device status error during timing")
+    res = {"value": job_value(S.units_per_step(), world, ms), "unit": UNIT, "ms_per_step": ms, "steps": steps,
+           "tokens_per_s": S.tokens_per_step() * world / (ms * 1e-3),
+           "gpu_launches": S.kernels_per_step() * steps, "clocks": clk.summary(), "graph": graph is not None}
     if args.profile:
-        if rank == 0:
-            print(json.dumps({"profile": True, "workload": args.workload, "layers": w.layers, "ms_per_step": ms}))
-        return
+        return res
 
-    # dominant kernel: the attention call, timed alone (graph of the attention launches of all layers)
-    hbm, bf16, bf16_sus, peak_kind = peaks()
+    # dominant call: the attention call alone (a graph of the attention launches of all layers)
     g2 = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         torch.cuda.synchronize()
@@ -546,76 +635,117 @@ def main():
                 S.attend(layer)
         for _ in range(5):
             g2.replay()
-        reps = max(20, min(200, args.steps))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        reps = max(10, min(200, steps))
+        ev0.record(stream)
         for _ in range(reps):
             g2.replay()
-        e1.record(stream)
+        ev1.record(stream)
     torch.cuda.synchronize()
-    att_ms = e0.elapsed_time(e1) / (reps * w.layers)
-    if w.kind == "decode":
-        ach = S.dominant_bytes() / (att_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": (measured_traffic("decode_q1", S.total) if w.n_q == 1 else
-                            measured_traffic("decode_splitk", S.total) if w.name == "verify_2req_229k" else None),
-                "kernel": "tq4_decode_append_attention (split-K decode with the append inside it for one "
-                          "query token + combine)",
-                "launch_ms": att_ms, "peak_source": f"{peak_kind} hbm_gbs"}
-    else:
-        ach = S.dominant_flops() / (att_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": ach, "peak": bf16, "unit": "TFLOP/s", "frac": ach / bf16,
-                "traffic": measured_traffic("prefill_tc", 1) if w.name == "prefill_2k_on_32k" else None,
-                "kernel": "tq4_prefill_attention (rotate prologue + attention kernel)",
-                "launch_ms": att_ms, "peak_source": f"{peak_kind} bf16_tflops (f16 operands: same nominal rate)"}
+    att_ms = ev0.elapsed_time(ev1) / (reps * w.layers)
+    res["roofline"] = S.roofline(att_ms, peaks())
 
-    # end to end: pinned host inputs in, results out, every step
+    # end to end through the public API: pinned host inputs in, every layer's output out, each step
     h2d, d2h = S.h2d_d2h()
-    e2e = None
-    if graph is not None:
-        ain, aout = S.arena_in, S.arena_out
-        n_e2e = max(10, min(args.steps, 200))
+    ain, aout = S.arena_in, S.arena_out
+    e2e = {"unit": UNIT, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    for label, fn in (("graph", graph.replay if graph is not None else None), ("eager", S.step)):
+        if fn is None:
+            continue
+        n = max(3, min(steps, 200 if label == "graph" else 50))
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(n_e2e):
+            ev0.record(stream)
+            for _ in range(n):
                 ain.dev.copy_(ain.host, non_blocking=True)     # this step's queries and new K/V
-                graph.replay()
+                fn()
                 aout.host.copy_(aout.dev, non_blocking=True)   # every layer's attention output
-            e1.record(stream)
+            ev1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        e2e_ms = max_over_ranks(e2e_ms, dist, device)
-        e2e = {"value": job_value(S.units_per_step(), world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
-               "path": "pinned H2D of the step's queries and new K/V, replay of the captured public C-ABI "
-                       "calls, D2H of every layer's output"}
+        e_ms = max_over_ranks(ev0.elapsed_time(ev1) / n, dist, device)
+        if label == "graph":
+            e2e.update(value=job_value(S.units_per_step(), world, e_ms), ms_per_step=e_ms,
+                       path="pinned H2D of the step's queries and new K/V, replay of the captured public C-ABI "
+                            "calls, D2H of every layer's output")
+        else:
+            e2e["eager"] = {"value": job_value(S.units_per_step(), world, e_ms), "ms_per_step": e_ms,
+                            "path": "the same copies around the calls made one by one through the ctypes binding "
+                                    "(argument checks, planning and tensor-map encoding on every call)"}
+    if "value" not in e2e:   # eager-only runs
+        e2e.update(value=e2e["eager"]["value"], ms_per_step=e2e["eager"]["ms_per_step"])
+    res["e2e"] = e2e
+    if S.ctx.status() != tq4.TQ4_OK:
+        raise RuntimeError(f"{name}: device status error")
+    del graph, g2, S
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
 
-    cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        orc = OracleSample(w)
-        v, el = orc.timed(10.0)
-        cpu = {"value": v, "unit": UNIT, "cores": orc.threads(), "kind": "oracle", "sample": orc.sample,
-               "seconds": el}
 
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "u4 codes, f16 tensor-core operands, f32 accumulate",
-            "data": "synthetic (seeded Gaussian K/V and queries)",
-            "config": workload_config(args.workload, world),
-            "graph": graph is not None,
-            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": S.kernels_per_step() * args.steps,
-            "clocks": clk.summary(),
-            "tokens_per_s": (w.n_req * w.n_q if w.kind == "decode" else w.n_q) * world / (ms * 1e-3),
-        }
+def finish(line, dist):
+    """Print the line (rank 0) and leave the process group once."""
+    if line is not None:
         print(json.dumps(line), flush=True)
-    del graph, g2
     if dist:
         dist.barrier()
         dist.destroy_process_group()
-        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------- main
+def main(argv=None, measure=None):
+    """`measure(name, args, dist, world, steps, headline) -> dict` replaces the GPU
+    measurement when given (the multi-rank path is tested on CPU ranks that way)."""
+    args = parse(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one process per GPU "
+                         "with torchrun (python -m torch.distributed.run --nproc-per-node N ... --gpus N)")
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    dist = None
+    if measure is None:
+        from compressed_paged_kv_tq4_b200 import tq4
+        torch.cuda.set_device(local)
+        device = torch.device("cuda", local)
+        backend = "nccl"
+    else:
+        tq4, device, backend = None, torch.device("cpu"), "gloo"
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+    def run(name, steps, headline):
+        if measure is not None:
+            return measure(name, args, dist, world, steps, headline)
+        return measure_workload(name, args, torch, tq4, device, dist, world, steps, headline)
+
+    head = run(args.workload, args.steps, True)
+    extras = {}
+    if not args.profile:
+        for name in [x for x in args.extra.split(",") if x and x != "none" and x != args.workload]:
+            extras[name] = dict(run(name, args.steps, False), config=workload_config(name, world))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile and measure is None:
+        orc = OracleSample(I.WORKLOADS[args.workload])
+        v, el = orc.timed(10.0)
+        cpu = dict({"value": v, "unit": UNIT, "kind": "oracle", "sample": orc.sample, "seconds": el}, **orc.cores())
+
+    line = None
+    if rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": head["steps"],
+                "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "u4 codes, f16 tensor-core operands, f32 accumulate",
+                "data": "synthetic (seeded Gaussian K/V and queries)",
+                "config": workload_config(args.workload, world),
+                "graph": head.get("graph"), "roofline": head.get("roofline"), "cpu_baseline": cpu,
+                "e2e": head.get("e2e"), "gpu_launches": head.get("gpu_launches"), "clocks": head.get("clocks"),
+                "tokens_per_s": head.get("tokens_per_s"), "workloads": extras}
+    finish(line, dist)
 
 
 if __name__ == "__main__":

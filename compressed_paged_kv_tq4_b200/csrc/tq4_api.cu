@@ -3,7 +3,6 @@
 // translation unit (the kernel headers are included below).
 #include <cmath>
 #include <cstring>
-#include <mutex>
 #include <new>
 
 #include <cuda.h>
@@ -24,6 +23,9 @@ struct tq4_ctx {
   double centroids[16];
   double boundaries[15];
   int* d_status;
+  uint32_t wait_polls;   // bounded device waits give up after this many polls
+  int withhold;          // test hook: kernels withhold one producer signal (see tq4_ctx_set_wait_limit)
+  void* noalloc_scratch; // device address of the library's fixed split-K array on this device
 };
 
 namespace {
@@ -74,10 +76,25 @@ int check_device(const tq4_ctx* ctx) {
   return dev == ctx->device ? TQ4_OK : TQ4_ERR_ARG;
 }
 
-template <int NT>
+template <int NT, bool kI8>
 cudaError_t set_decode_attrs() {
-  return cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              int(tq4::decode_smem_bytes<NT>()));
+  cudaError_t e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, kI8, false>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(tq4::decode_smem_bytes<NT, kI8>()));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, kI8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(tq4::decode_smem_bytes<NT, kI8>()));
+  return e;
+}
+
+// one split-K decode launch with the output precision chosen at run time
+template <int NT, bool kI8>
+cudaError_t launch_splitk(dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  if (p.out_dtype == TQ4_DTYPE_F32)
+    return tq4::launch_pdl(tq4::decode_splitk_kernel<NT, kI8, true>, grid, dim3(tq4::kDecThreads),
+                           tq4::decode_smem_bytes<NT, kI8>(), st, p);
+  return tq4::launch_pdl(tq4::decode_splitk_kernel<NT, kI8, false>, grid, dim3(tq4::kDecThreads),
+                         tq4::decode_smem_bytes<NT, kI8>(), st, p);
 }
 
 struct DecodePlan {
@@ -141,6 +158,22 @@ DecodePlan plan_decode(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t t
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Decode attention without any allocation by the caller or the library.
+//
+// Some callers cannot allocate device memory: plugin code running inside a host
+// program that owns the whole device-memory budget (a raw cudaMalloc would
+// bypass its accounting), and serving processes that reserve all device memory
+// up front and run under a hard memory guard. For them the split-K partial
+// results live in this fixed array instead of a caller-provided workspace.
+// The array is part of the library image: every GPU that loads the library
+// holds TQ4_NOALLOC_SCRATCH_BYTES of it until the process exits. In host code
+// its name is only a host-side stand-in, so tq4_ctx_create asks the runtime for
+// the array's device address on the context's device (with that device current)
+// and keeps it in the context.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[TQ4_NOALLOC_SCRATCH_BYTES];
+
 extern "C" {
 
 int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
@@ -154,31 +187,38 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   tq4_ctx* ctx = new (std::nothrow) tq4_ctx();
   if (!ctx) return TQ4_ERR_ARG;
   ctx->signs = sb;
-  // the format stores the 16 centroids as fp16; boundaries are midpoints of the stored values
-  double sol[16], sol_b[15];
-  lloyd_max_16(1.0 / 16.0, sol, sol_b);
+  ctx->wait_polls = TQ4_DEFAULT_WAIT_POLLS;
+  // the fp64 Lloyd-Max solution is the codebook: encode compares against its
+  // midpoints (rounded to fp32), reconstruction reads the centroids rounded to
+  // fp32, and the attention kernels read each centroid as an f16 hi + lo pair
   tq4::Codebook cb{};
+  lloyd_max_16(1.0 / 16.0, ctx->centroids, ctx->boundaries);
   for (int j = 0; j < 16; ++j) {
-    cb.c16[j] = half_bits(sol[j]);
+    cb.c[j] = float(ctx->centroids[j]);
+    cb.c16[j] = half_bits(ctx->centroids[j]);
     __half hh;
     std::memcpy(&hh, &cb.c16[j], 2);
-    ctx->centroids[j] = double(__half2float(hh));
-    cb.c[j] = __half2float(hh);
+    cb.r16[j] = half_bits(ctx->centroids[j] - double(__half2float(hh)));
   }
-  for (int j = 0; j < 15; ++j) {
-    ctx->boundaries[j] = 0.5 * (ctx->centroids[j] + ctx->centroids[j + 1]);
-    cb.b[j] = float(ctx->boundaries[j]);  // exact: the sum of two fp16 values fits in fp32
-  }
+  for (int j = 0; j < 15; ++j) cb.b[j] = float(ctx->boundaries[j]);
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(tq4::g_codebook, &cb, sizeof(cb));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(tq4::decode_q1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(tq4::decode_q1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(tq4::decode_q1_smem_bytes()));
-  if (e == cudaSuccess) e = set_decode_attrs<1>();
-  if (e == cudaSuccess) e = set_decode_attrs<2>();
-  if (e == cudaSuccess) e = set_decode_attrs<3>();
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tq4::decode_q1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(tq4::decode_q1_smem_bytes()));
+  if (e == cudaSuccess) e = set_decode_attrs<1, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<2, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<3, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<1, true>();
+  if (e == cudaSuccess) e = set_decode_attrs<2, true>();
+  if (e == cudaSuccess) e = set_decode_attrs<3, true>();
   if (e == cudaSuccess) e = tq4::prefill_tc_set_attrs();
+  if (e == cudaSuccess) e = cudaGetSymbolAddress(&ctx->noalloc_scratch, g_noalloc_scratch);
+  if (e == cudaSuccess && !ctx->noalloc_scratch) e = cudaErrorInvalidSymbol;
   if (e == cudaSuccess) e = cudaMalloc(&ctx->d_status, sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(ctx->d_status, 0, sizeof(int));
   if (e != cudaSuccess) {
@@ -196,6 +236,13 @@ int tq4_ctx_destroy(tq4_ctx* ctx) {
   const cudaError_t e = cudaFree(ctx->d_status);
   delete ctx;
   return cuda_status(e);
+}
+
+int tq4_ctx_set_wait_limit(tq4_ctx* ctx, uint32_t polls, int withhold_signal) {
+  if (!ctx) return TQ4_ERR_ARG;
+  ctx->wait_polls = polls ? polls : TQ4_DEFAULT_WAIT_POLLS;
+  ctx->withhold = withhold_signal ? 1 : 0;
+  return TQ4_OK;
 }
 
 int tq4_codebook(const tq4_ctx* ctx, double* centroids, double* boundaries) {
@@ -253,7 +300,7 @@ struct AppendArgs {   // the fused append of tq4_decode_append_attention
 int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q, const int32_t* page_tables,
                 int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q, int64_t total_seq_len,
                 float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream,
-                const AppendArgs* app) {
+                const AppendArgs* app, bool int8 = false) {
   if (!ctx || n_req < 0) return TQ4_ERR_ARG;
   if (n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS) return TQ4_ERR_UNSUPPORTED;
   if (n_req == 0) return TQ4_OK;
@@ -291,6 +338,9 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
   p.out_dtype = out_dtype;
   p.signs = ctx->signs;
   p.status = ctx->d_status;
+  p.spin_limit = ctx->wait_polls;
+  p.test_withhold = ctx->withhold;
+  p.rotate = int8 ? 0 : 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (app && n_q == 1) {   // appended inside the decode kernel
@@ -304,22 +354,28 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
     if (e != cudaSuccess) return TQ4_ERR_CUDA;
   }
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
-  switch (tq4::decode_nt(n_q)) {
-    case 1: {
-      CUtensorMap map;
-      if (int rc = pool_tensor_map(pool, num_pages, &map)) return rc;
-      e = tq4::launch_pdl(tq4::decode_q1_kernel, grid, dim3(tq4::kQ1Threads), tq4::decode_q1_smem_bytes(), st, p,
-                          map);
-      break;
+  if (int8) {
+    switch (tq4::decode_nt(n_q)) {
+      case 1: e = launch_splitk<1, true>(grid, st, p); break;
+      case 2: e = launch_splitk<2, true>(grid, st, p); break;
+      default: e = launch_splitk<3, true>(grid, st, p); break;
     }
-    case 2:
-      e = tq4::launch_pdl(tq4::decode_splitk_kernel<2>, grid, dim3(tq4::kDecThreads), tq4::decode_smem_bytes<2>(),
-                          st, p);
-      break;
-    default:
-      e = tq4::launch_pdl(tq4::decode_splitk_kernel<3>, grid, dim3(tq4::kDecThreads), tq4::decode_smem_bytes<3>(),
-                          st, p);
-      break;
+  } else {
+    switch (tq4::decode_nt(n_q)) {
+      case 1: {
+        CUtensorMap map;
+        if (int rc = pool_tensor_map(pool, num_pages, &map)) return rc;
+        if (out_dtype == TQ4_DTYPE_F32)
+          e = tq4::launch_pdl(tq4::decode_q1_kernel<true>, grid, dim3(tq4::kQ1Threads), tq4::decode_q1_smem_bytes(),
+                              st, p, map);
+        else
+          e = tq4::launch_pdl(tq4::decode_q1_kernel<false>, grid, dim3(tq4::kQ1Threads),
+                              tq4::decode_q1_smem_bytes(), st, p, map);
+        break;
+      }
+      case 2: e = launch_splitk<2, false>(grid, st, p); break;
+      default: e = launch_splitk<3, false>(grid, st, p); break;
+    }
   }
   if (e != cudaSuccess) return TQ4_ERR_CUDA;
   const int rows = n_req * n_q * tq4::kHq;
@@ -348,6 +404,29 @@ int tq4_decode_append_attention(tq4_ctx* ctx, void* pool, int32_t num_pages, con
                      out, out_dtype, workspace, workspace_bytes, stream, &app);
 }
 
+int tq4_int8_encode_append(tq4_ctx* ctx, void* pool, int32_t num_pages, const int32_t* page_table,
+                           int32_t table_len, int32_t start_pos, int32_t n_tok, const void* k_new,
+                           const void* v_new, int dtype, void* stream) {
+  if (!ctx || n_tok < 0 || start_pos < 0) return TQ4_ERR_ARG;
+  if (n_tok == 0) return TQ4_OK;
+  if (!pool || !page_table || !k_new || !v_new || num_pages <= 0 || table_len <= 0) return TQ4_ERR_ARG;
+  if (dtype != TQ4_DTYPE_F32 && dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
+  if ((int64_t(start_pos) + n_tok + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
+  if (!aligned(pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16)) return TQ4_ERR_ARG;
+  if (int rc = check_device(ctx)) return rc;
+  return cuda_status(tq4::launch_int8_encode_append(static_cast<uint8_t*>(pool), num_pages, page_table, start_pos,
+                                                    n_tok, k_new, v_new, dtype, ctx->d_status,
+                                                    static_cast<cudaStream_t>(stream)));
+}
+
+int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q,
+                              const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens,
+                              int32_t n_req, int32_t n_q, int64_t total_seq_len, float scale, void* out,
+                              int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, nullptr, true);
+}
+
 size_t tq4_prefill_workspace_bytes(int32_t n_tok) {
   if (n_tok <= 0) return 0;
   return tq4::prefill_workspace_bytes(n_tok);
@@ -356,10 +435,11 @@ size_t tq4_prefill_workspace_bytes(int32_t n_tok) {
 int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int32_t* page_table,
                           int32_t table_len, int32_t prefix_len, const uint16_t* q,
                           const uint16_t* k_chunk, const uint16_t* v_chunk, int32_t n_tok, float scale,
-                          uint16_t* out, void* workspace, size_t workspace_bytes, void* stream) {
+                          void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
   if (!ctx || n_tok < 0 || prefix_len < 0) return TQ4_ERR_ARG;
   if (n_tok == 0) return TQ4_OK;
   if (!q || !k_chunk || !v_chunk || !out) return TQ4_ERR_ARG;
+  if (out_dtype != TQ4_DTYPE_F32 && out_dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
   if (prefix_len > 0 && (!pool || !page_table || num_pages <= 0 || table_len <= 0)) return TQ4_ERR_ARG;
   if (prefix_len > 0 && (int64_t(prefix_len) + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
   if (!std::isfinite(scale)) return TQ4_ERR_ARG;
@@ -370,8 +450,9 @@ int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages, con
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
   if (int rc = check_device(ctx)) return rc;
   return cuda_status(tq4::launch_prefill_tc(static_cast<const uint8_t*>(pool), num_pages, page_table,
-                                            prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, workspace,
-                                            ctx->signs, ctx->d_status, static_cast<cudaStream_t>(stream)));
+                                            prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, out_dtype,
+                                            workspace, ctx->signs, ctx->d_status, ctx->wait_polls,
+                                            ctx->withhold, static_cast<cudaStream_t>(stream)));
 }
 
 int tq4_get_status(tq4_ctx* ctx, void* stream) {
@@ -399,40 +480,6 @@ const char* tq4_status_string(int status) {
   }
 }
 
-// ---------------------------------------------------------------------------
-// Decode attention without any allocation by the caller or the library.
-//
-// Some callers cannot allocate device memory: plugin code running inside a host
-// program that owns the whole device-memory budget (a raw cudaMalloc would
-// bypass its accounting), and serving processes that reserve all device memory
-// up front and run under a hard memory guard. For them the split-K partial
-// results live in this fixed array instead of a caller-provided workspace.
-// The array is part of the library image: every GPU that loads the library
-// holds TQ4_NOALLOC_SCRATCH_BYTES of it until the process exits.
-// ---------------------------------------------------------------------------
-static __device__ __align__(256) unsigned char g_noalloc_scratch[TQ4_NOALLOC_SCRATCH_BYTES];
-
-namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device. In host code the
-// array's name is only a host-side stand-in, so the address is asked from the
-// runtime once per device (with that device current) and cached.
-int noalloc_scratch(int device, void** out) {
-  if (device < 0 || device >= kMaxDevices) return TQ4_ERR_ARG;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[device]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return TQ4_ERR_CUDA;
-    g_noalloc_ptr[device] = ptr;
-  }
-  *out = g_noalloc_ptr[device];
-  return TQ4_OK;
-}
-}  // namespace
-
 int tq4_decode_attention_noalloc(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q,
                                  const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens,
                                  int32_t n_req, int32_t n_q, int64_t total_seq_len, float scale, void* out,
@@ -443,11 +490,9 @@ int tq4_decode_attention_noalloc(tq4_ctx* ctx, const void* pool, int32_t num_pag
   if (n_req < 0 || total_seq_len <= 0) return TQ4_ERR_ARG;
   if (tq4_decode_workspace_bytes(ctx, n_req, n_q, total_seq_len) > TQ4_NOALLOC_SCRATCH_BYTES)
     return TQ4_ERR_WORKSPACE;
-  if (int rc = check_device(ctx)) return rc;
-  void* scratch = nullptr;
-  if (int rc = noalloc_scratch(ctx->device, &scratch)) return rc;
   return tq4_decode_attention(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
-                              total_seq_len, scale, out, out_dtype, scratch, TQ4_NOALLOC_SCRATCH_BYTES, stream);
+                              total_seq_len, scale, out, out_dtype, ctx->noalloc_scratch, TQ4_NOALLOC_SCRATCH_BYTES,
+                              stream);
 }
 
 }  // extern "C"

@@ -25,6 +25,8 @@
 // Per-split partial results (m, l, o') go to the workspace; the combine pass
 // merges them (log-sum-exp), rotates back and writes bf16/fp32.
 #pragma once
+#include <type_traits>
+
 #include "tq4_device.cuh"
 
 namespace tq4 {
@@ -36,6 +38,16 @@ constexpr int kStages = 3;                   // cp.async ring depth
 constexpr int kQvStride = kD + 8;            // halves per Q' row in smem (bank-conflict pad)
 constexpr int kPsStride = kChunk + 8;        // halves per P' row in smem
 constexpr int kStageBytes = 2 * kChunk * 128 + 2 * kChunk * 2;   // K words, V words, K norms, V norms
+
+// Uniform INT8 comparison arm: a page holds 256 positions of one layer as
+// K codes [4 heads][256 slots][256 int8], V codes, K scales [4][256] fp16, V scales.
+constexpr int64_t kI8PageBytes = TQ4_INT8_PAGE_BYTES;   // 528,384
+constexpr int64_t kI8KCodes = 0;
+constexpr int64_t kI8VCodes = int64_t(kHkv) * kPage * kD;          // 262,144
+constexpr int64_t kI8KScales = 2 * kI8VCodes;                       // 524,288
+constexpr int64_t kI8VScales = kI8KScales + int64_t(kHkv) * kPage * 2;   // 526,336
+constexpr int kI8Stages = 2;
+constexpr int kI8StageBytes = 2 * kChunk * 256 + 2 * kChunk * 2;   // K codes, V codes, K scales, V scales
 
 struct DecodeParams {
   const uint8_t* pool;
@@ -63,14 +75,17 @@ struct DecodeParams {
   const void* k_new;
   const void* v_new;
   int new_dtype;
+  uint32_t spin_limit;   // polls before a bounded wait gives up (TQ4_ERR_TIMEOUT)
+  int test_withhold;     // test hook: withhold the first tile copy of each warp (its wait runs out)
+  int rotate;            // 1: o = R^T o' (TQ4, rotated domain); 0: o = o' (the INT8 arm)
 };
 
 __host__ __device__ constexpr int decode_nt(int n_q) { return (6 * n_q + 7) / 8; }
 
-template <int NT>
+template <int NT, bool kI8>
 constexpr size_t decode_smem_bytes() {
-  return size_t(kLutBytes) + size_t(kStages) * kStageBytes + 2 * size_t(8 * NT) * kQvStride * 2 +
-         2 * size_t(8 * NT) * kPsStride * 2 + size_t(kDecWarps) * 8 * NT * 4;
+  return (kI8 ? size_t(kI8Stages) * kI8StageBytes : size_t(kLutBytes) + size_t(kStages) * kStageBytes) +
+         2 * size_t(8 * NT) * kQvStride * 2 + 2 * size_t(8 * NT) * kPsStride * 2 + size_t(kDecWarps) * 8 * NT * 4;
 }
 
 __device__ __forceinline__ int warp_incl_scan(int v) {
@@ -130,15 +145,40 @@ __device__ __forceinline__ uint32_t pick(const uint4& a, const uint4& b, int i) 
 __device__ __forceinline__ int seg_swz(int pos) { return (((pos >> 1) & 3) << 1) ^ ((pos & 1) << 2); }
 
 
+// INT8 rows are 256 B (16 segments of 16 B). The swizzle makes both the K phase
+// (segments 4m + t of positions g, g + 1 per quarter warp) and the V phase (8-byte
+// pieces of one segment pair from positions 2t, t = 0..3, per half warp) hit
+// distinct banks.
+__device__ __forceinline__ int i8_swz(int pos) { return (((pos >> 1) & 3) << 1) ^ ((pos & 1) << 2); }
+
+// int8 codes in bits 0-7 and 16-23 of t (the rest ignored) -> f16x2 holding them
+// exactly: the code plus 128 (its sign bit flipped) sits in the mantissa of 1024
+// (f16 0x6400), and 1152 is subtracted
+__device__ __forceinline__ uint32_t i8_pair_bytes(uint32_t t) {
+  uint32_t u;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;\n" : "=r"(u) : "r"(t), "r"(0x00FF00FFu), "r"(0x64806480u));   // (a & b) ^ c
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&u), __floats2half2_rn(1152.f, 1152.f));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+// int8 codes in bytes B0, B1 of w -> exact f16x2 (byte B0 in the low half)
+template <int B0, int B1>
+__device__ __forceinline__ uint32_t i8_pair(uint32_t w) {
+  return i8_pair_bytes(__byte_perm(w, 0u, uint32_t(B0) | (4u << 4) | (uint32_t(B1) << 8) | (4u << 12)));
+}
+
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
-template <int NT>
+template <int NT, bool kI8, bool kExact>   // kExact: fp32 outputs, every product (see kVloNorm)
 __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t lut = smem_u32(smem);
-  uint8_t* ring = smem + kLutBytes;
-  __half* qv_hi = reinterpret_cast<__half*>(ring + kStages * kStageBytes);
+  constexpr int kRB = kI8 ? 256 : 128;                 // bytes of one staged K or V row
+  constexpr int kNS = kI8 ? kI8Stages : kStages;       // ring stages; chunks prefetched kNS - 1 ahead
+  constexpr int kSB = kI8 ? kI8StageBytes : kStageBytes;
+  const uint32_t lut = smem_u32(smem);                 // the centroid table (TQ4 only)
+  uint8_t* ring = smem + (kI8 ? 0 : kLutBytes);
+  __half* qv_hi = reinterpret_cast<__half*>(ring + kNS * kSB);
   __half* qv_lo = qv_hi + 8 * NT * kQvStride;
   __half* ps_hi = qv_lo + 8 * NT * kQvStride;
   __half* ps_lo = ps_hi + 8 * NT * kPsStride;   // P' = hi + lo, both f16
@@ -148,7 +188,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int h = blockIdx.y;
-  const uint32_t lane4 = uint32_t(lane) * 4u;
+  const uint32_t lane8 = uint32_t(lane) * 8u;
 
   pdl_wait();   // every read of the call's inputs comes after the previous kernel
   pdl_launch_dependents();
@@ -181,34 +221,40 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       if (page < 0 || page >= p.num_pages) {
         if (tid == 0) record_error(p.status, TQ4_ERR_PAGE_RANGE);
       } else {
-        const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
+        constexpr int64_t kPB = kI8 ? kI8PageBytes : kPageBytes;
+        constexpr int64_t kKR = kI8 ? kI8KCodes : kKWords, kVR = kI8 ? kI8VCodes : kVWords;
+        constexpr int64_t kKN = kI8 ? kI8KScales : kKNorms, kVN = kI8 ? kI8VScales : kVNorms;
+        constexpr int kSeg = kRB / 16;   // 16-byte segments per row
+        const uint8_t* pg = p.pool + int64_t(page) * kPB;
         const int64_t slot0 = head_slot0 + (c & (kPage - 1));
-        uint8_t* st = ring + (i % kStages) * kStageBytes;
+        uint8_t* st = ring + (i % kNS) * kSB;
         const int nvalid = min(kChunk, pos_e - c);
-        // words: 2 x kChunk positions x 8 segments
-        for (int e = tid; e < 2 * kChunk * 8; e += kDecThreads) {
-          const int kv = e / (kChunk * 8), pl = (e >> 3) % kChunk, sg = e & 7;
+        // K and V rows: 2 x kChunk positions x kSeg segments
+        for (int e = tid; e < 2 * kChunk * kSeg; e += kDecThreads) {
+          const int kv = e / (kChunk * kSeg), pl = (e / kSeg) % kChunk, sg = e % kSeg;
           if (pl < nvalid) {
-            const uint8_t* src = pg + (kv ? kVWords : kKWords) + (slot0 + pl) * 128 + sg * 16;
-            cp_async16(smem_u32(st + kv * kChunk * 128 + pl * 128 + ((sg ^ seg_swz(pl)) << 4)), src);
+            const uint8_t* src = pg + (kv ? kVR : kKR) + (slot0 + pl) * kRB + sg * 16;
+            const int sw = kI8 ? i8_swz(pl) : seg_swz(pl);
+            cp_async16(smem_u32(st + kv * kChunk * kRB + pl * kRB + ((sg ^ sw) << 4)), src);
           }
         }
-        // norms: 2 x kChunk halves = 2 x (kChunk / 8) segments
+        // norms (scales): 2 x kChunk halves = 2 x (kChunk / 8) segments
         if (tid < 2 * (kChunk / 8)) {
           const int kv = tid / (kChunk / 8), sg = tid % (kChunk / 8);
           if (sg * 8 < nvalid) {
-            const uint8_t* src = pg + (kv ? kVNorms : kKNorms) + (slot0 + sg * 8) * 2;
-            cp_async16(smem_u32(st + 2 * kChunk * 128 + kv * kChunk * 2 + sg * 16), src);
+            const uint8_t* src = pg + (kv ? kVN : kKN) + (slot0 + sg * 8) * 2;
+            cp_async16(smem_u32(st + 2 * kChunk * kRB + kv * kChunk * 2 + sg * 16), src);
           }
         }
       }
     }
     cp_async_commit();
   };
-  issue_chunk(0);
-  issue_chunk(1);
+#pragma unroll
+  for (int i = 0; i < kNS - 1; ++i) issue_chunk(i);
 
-  // ---- rotate the queries of this (request, KV head): q' = R q * scale, split hi + lo f16, virtual order
+  // ---- the queries of this (request, KV head): q' = R q * scale (TQ4) or q * scale
+  // (INT8), split hi + lo f16, stored in the K phase's virtual dim order
   for (int row = w; row < 8 * NT; row += kDecWarps) {
     float v[8];
     if (row < NR) {
@@ -216,14 +262,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       const uint16_t* src = p.q + ((int64_t(r) * p.n_q + tok) * kHq + h * kGroup + j) * kD + lane * 8;
       const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
       const uint32_t ww[4] = {raw.x, raw.y, raw.z, raw.w};
+      if constexpr (kI8) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(ww[i] << 16) * sign_of(p.signs, lane * 8 + 2 * i);
-        v[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * sign_of(p.signs, lane * 8 + 2 * i + 1);
+        for (int i = 0; i < 4; ++i) {
+          v[2 * i] = __uint_as_float(ww[i] << 16) * p.scale;
+          v[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * p.scale;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[2 * i] = __uint_as_float(ww[i] << 16) * sign_of(p.signs, lane * 8 + 2 * i);
+          v[2 * i + 1] = __uint_as_float(ww[i] & 0xFFFF0000u) * sign_of(p.signs, lane * 8 + 2 * i + 1);
+        }
+        warp_fwht256(v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] *= p.scale * 0.0625f;
       }
-      warp_fwht256(v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] *= p.scale * 0.0625f;
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = 0.f;
@@ -231,23 +285,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
     // lane owns real dims 8*lane + i (word lane). Word lane is read in the K phase by
     // thread t = (lane & 15) >> 2 as its word index ws = (lane & 3) + 4*(lane >> 4);
     // k-step kk = 2*ws + (i >> 2), mma column 2t + (i & 1) + 8*((i >> 1) & 1).
+    // INT8: dim d = 8 lane + i is read in the K phase by thread t = (d >> 4) & 3 from
+    // its 16-byte segment 4m + t (m = d >> 6) as byte (d & 3) of word j = (d >> 2) & 3:
+    // k-step kk = 4m + j, mma column 2t + (d & 1) + 8 ((d >> 1) & 1).
     const int tt = (lane & 15) >> 2, wsel = (lane & 3) + 4 * (lane >> 4);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-      const int kk = 2 * wsel + (i >> 2);
-      const int col = kk * 16 + ((i >> 1) & 1) * 8 + 2 * tt;
+      const int kk = kI8 ? 4 * (lane >> 3) + ((2 * lane + (i >> 2)) & 3) : 2 * wsel + (i >> 2);
+      const int col = kI8 ? kk * 16 + 2 * ((lane >> 1) & 3) + 8 * ((i >> 1) & 1)
+                          : kk * 16 + ((i >> 1) & 1) * 8 + 2 * tt;
       const __half2 hi = __floats2half2_rn(v[i], v[i + 1]);
       const float2 hf = __half22float2(hi);
       *reinterpret_cast<__half2*>(qv_hi + row * kQvStride + col) = hi;
       *reinterpret_cast<__half2*>(qv_lo + row * kQvStride + col) = __floats2half2_rn(v[i] - hf.x, v[i + 1] - hf.y);
     }
   }
-  // centroid table: row b holds f16x2 {c[b & 15], c[b >> 4]} at +4*lane (the stored fp16 codebook)
-  for (int e = tid; e < 256 * 32; e += kDecThreads) {
-    const int b = e >> 5, l = e & 31;
-    reinterpret_cast<uint32_t*>(smem)[b * 64 + l] =
-        uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16);
-  }
+  // centroid table: row b holds each lane's 8-byte slot {c16 pair, r16 pair} at +8*lane
+  if constexpr (!kI8)
+    for (int e = tid; e < 256 * 32; e += kDecThreads) reinterpret_cast<uint2*>(smem)[e] = lut_row(e >> 5);
   __syncthreads();
 
   // ---- B fragments of Q' (hi, lo) for the K phase, in registers when they fit
@@ -287,26 +342,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   const int dg = w & 3, ph = w >> 2;   // V phase: 64-dim group, 64-position half
 
   for (int i = 0; i < n_chunks; ++i) {
-    cp_async_wait<1>();
+    cp_async_wait<kNS - 2>();
     __syncthreads();            // chunk i visible to all; everyone is done with chunk i-1
-    issue_chunk(i + 2);
+    issue_chunk(i + kNS - 1);
     const int c = pos_b + i * kChunk;
-    const uint8_t* st = ring + (i % kStages) * kStageBytes;
+    const uint8_t* st = ring + (i % kNS) * kSB;
     const uint8_t* kst = st;
-    const uint8_t* vst = st + kChunk * 128;
-    const __half* knr = reinterpret_cast<const __half*>(st + 2 * kChunk * 128);
+    const uint8_t* vst = st + kChunk * kRB;
+    const __half* knr = reinterpret_cast<const __half*>(st + 2 * kChunk * kRB);
     const __half* vnr = knr + kChunk;
 
     // ---------------------------------------------------------- K phase: S = C_k Q'^T (fp32-grade)
     const int pg0 = 16 * w + g;   // chunk-local positions pg0, pg0 + 8
-    const int sz = seg_swz(pg0);  // same for pg0 + 8
-    const uint4 ka0 = lds128(kst + pg0 * 128 + ((t ^ sz) << 4));
-    const uint4 ka1 = lds128(kst + pg0 * 128 + (((4 + t) ^ sz) << 4));
-    const uint4 kb0 = lds128(kst + (pg0 + 8) * 128 + ((t ^ sz) << 4));
-    const uint4 kb1 = lds128(kst + (pg0 + 8) * 128 + (((4 + t) ^ sz) << 4));
-    // scores = C_k (q'_hi + q'_lo): the centroid values are exact in f16, so two products
-    // with fp32 accumulation carry the scores to fp32 precision; even/odd k-steps use
-    // separate accumulators to halve the dependent mma chains
+    // scores = (C_hi + C_lo)(q'_hi + q'_lo) to fp32 precision: C_hi q'_hi + [C_hi q'_lo + C_lo q'_hi]
+    // (the two small terms share one accumulator; C_lo q'_lo is below fp32 resolution);
+    // INT8 codes are exact f16 values, so there C_lo = 0. Even/odd k-steps use
+    // separate accumulators to halve the dependent mma chains.
     float shh[2][NT][4], sx[2][NT][4];
 #pragma unroll
     for (int a = 0; a < 2; ++a)
@@ -314,42 +365,76 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < 4; ++j) shh[a][nt][j] = sx[a][nt][j] = 0.f;
+    // B fragments of q' hi / lo for k-step kk and n-tile nt
+    auto qfrag = [&](int kk, int nt, uint32_t& bh0, uint32_t& bh1, uint32_t& bl0, uint32_t& bl1) {
+      if constexpr (kQReg) {
+        bh0 = qh[kk][0]; bh1 = qh[kk][1]; bl0 = ql[kk][0]; bl1 = ql[kk][1];
+      } else {
+        const int m = (lane >> 3) & 1;
+        const int off = (nt * 8 + (lane & 7)) * kQvStride + kk * 16 + m * 8;
+        ldmatrix_x2(bh0, bh1, smem_u32(qv_hi + off));
+        ldmatrix_x2(bl0, bl1, smem_u32(qv_lo + off));
+      }
+    };
+    if constexpr (kI8) {
+      const int sz = i8_swz(pg0);   // same for pg0 + 8
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {   // k-steps 4m .. 4m + 3: one 16-byte segment per position
+        const uint4 ka = lds128(kst + pg0 * 256 + (((4 * m + t) ^ sz) << 4));
+        const uint4 kb = lds128(kst + (pg0 + 8) * 256 + (((4 * m + t) ^ sz) << 4));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int kk = 4 * m + j;
+          const uint32_t wa = pick(ka, ka, j), wb = pick(kb, kb, j);
+          const uint32_t a0 = i8_pair<0, 1>(wa), a1 = i8_pair<0, 1>(wb);
+          const uint32_t a2 = i8_pair<2, 3>(wa), a3 = i8_pair<2, 3>(wb);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            uint32_t bh0, bh1, bl0, bl1;
+            qfrag(kk, nt, bh0, bh1, bl0, bl1);
+            mma_16816(shh[kk & 1][nt], a0, a1, a2, a3, bh0, bh1);
+            mma_16816(sx[kk & 1][nt], a0, a1, a2, a3, bl0, bl1);
+          }
+        }
+      }
+    } else {
+    const int sz = seg_swz(pg0);  // same for pg0 + 8
+    const uint4 ka0 = lds128(kst + pg0 * 128 + ((t ^ sz) << 4));
+    const uint4 ka1 = lds128(kst + pg0 * 128 + (((4 + t) ^ sz) << 4));
+    const uint4 kb0 = lds128(kst + (pg0 + 8) * 128 + ((t ^ sz) << 4));
+    const uint4 kb1 = lds128(kst + (pg0 + 8) * 128 + (((4 + t) ^ sz) << 4));
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
       const uint32_t wg = pick(ka0, ka1, kk >> 1);
       const uint32_t wg8 = pick(kb0, kb1, kk >> 1);
-      uint32_t a0, a1, a2, a3;
+      uint32_t a0, a1, a2, a3, r0, r1, r2, r3;
       if (kk & 1) {
-        a0 = lut_decode<2>(lut, wg, lane4);
-        a1 = lut_decode<2>(lut, wg8, lane4);
-        a2 = lut_decode<3>(lut, wg, lane4);
-        a3 = lut_decode<3>(lut, wg8, lane4);
+        lut_decode<2>(lut, wg, lane8, a0, r0);
+        lut_decode<2>(lut, wg8, lane8, a1, r1);
+        lut_decode<3>(lut, wg, lane8, a2, r2);
+        lut_decode<3>(lut, wg8, lane8, a3, r3);
       } else {
-        a0 = lut_decode<0>(lut, wg, lane4);
-        a1 = lut_decode<0>(lut, wg8, lane4);
-        a2 = lut_decode<1>(lut, wg, lane4);
-        a3 = lut_decode<1>(lut, wg8, lane4);
+        lut_decode<0>(lut, wg, lane8, a0, r0);
+        lut_decode<0>(lut, wg8, lane8, a1, r1);
+        lut_decode<1>(lut, wg, lane8, a2, r2);
+        lut_decode<1>(lut, wg8, lane8, a3, r3);
       }
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         uint32_t bh0, bh1, bl0, bl1;
-        if constexpr (kQReg) {
-          bh0 = qh[kk][0]; bh1 = qh[kk][1]; bl0 = ql[kk][0]; bl1 = ql[kk][1];
-        } else {
-          const int m = (lane >> 3) & 1;
-          const int off = (nt * 8 + (lane & 7)) * kQvStride + kk * 16 + m * 8;
-          ldmatrix_x2(bh0, bh1, smem_u32(qv_hi + off));
-          ldmatrix_x2(bl0, bl1, smem_u32(qv_lo + off));
-        }
+        qfrag(kk, nt, bh0, bh1, bl0, bl1);
         mma_16816(shh[kk & 1][nt], a0, a1, a2, a3, bh0, bh1);
         mma_16816(sx[kk & 1][nt], a0, a1, a2, a3, bl0, bl1);
+        mma_16816(sx[kk & 1][nt], r0, r1, r2, r3, bh0, bh1);
       }
+    }
     }
 
     // ---------------------------------------------------------- online softmax over the chunk
     const float kn0 = __half2float(knr[pg0]), kn8 = __half2float(knr[pg0 + 8]);
     const float vn0 = __half2float(vnr[pg0]), vn8 = __half2float(vnr[pg0 + 8]);
     const int pos0 = c + pg0;
+    const bool vbig = (pos0 < pos_e && vn0 > kVloNorm) || (pos0 + 8 < pos_e && vn8 > kVloNorm);
     float s[NT][4], mx[NT][2];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -403,13 +488,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       const int poff = (nt * 8 + jr) * kPsStride + 16 * w + 8 * mat;
       stmatrix_x2_trans(smem_u32(ps_hi + poff), *reinterpret_cast<const uint32_t*>(&h01),
                         *reinterpret_cast<const uint32_t*>(&h23));
-      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-      const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
-      const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
-      stmatrix_x2_trans(smem_u32(ps_lo + poff), *reinterpret_cast<const uint32_t*>(&l01),
-                        *reinterpret_cast<const uint32_t*>(&l23));
+      if constexpr (kExact) {
+        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
+        const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
+        stmatrix_x2_trans(smem_u32(ps_lo + poff), *reinterpret_cast<const uint32_t*>(&l01),
+                          *reinterpret_cast<const uint32_t*>(&l23));
+      }
     }
-    __syncthreads();
+    // P' is complete; the chunk takes the C_lo P' products when one of its visible
+    // V norms is large (or the output is fp32)
+    const bool vlo = __syncthreads_or(vbig) != 0 || kExact;
 
     // ---------------------------------------------------------- V phase: O'^T += C_v^T P'^T
 #pragma unroll
@@ -421,8 +510,47 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
         o[nt][mt][2] *= alpha[nt][0];
         o[nt][mt][3] *= alpha[nt][1];
       }
+    if constexpr (kI8) {
+      // lane (g, t): 8 codes (dims 64 dg + 8 g .. + 7) of positions 2t, 2t+1, 2t+8, 2t+9
+      // of each k-step; m-tile mt's rows g, g + 8 are dims 64 dg + 8 g + 2 mt, + 1
+      const int seg = 4 * dg + (g >> 1), off8 = (g & 1) * 8;
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        const int pb = 64 * ph + 16 * ks + 2 * t;
+        const uint2 x0 = lds64(vst + pb * 256 + ((seg ^ i8_swz(pb)) << 4) + off8);
+        const uint2 x1 = lds64(vst + (pb + 1) * 256 + ((seg ^ i8_swz(pb + 1)) << 4) + off8);
+        const uint2 y0 = lds64(vst + (pb + 8) * 256 + ((seg ^ i8_swz(pb + 8)) << 4) + off8);
+        const uint2 y1 = lds64(vst + (pb + 9) * 256 + ((seg ^ i8_swz(pb + 9)) << 4) + off8);
+        uint32_t bh[NT][2], bl[NT][2] = {};
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const int m = (lane >> 3) & 1;
+          const int off = (nt * 8 + (lane & 7)) * kPsStride + 64 * ph + 16 * ks + 8 * m;
+          ldmatrix_x2(bh[nt][0], bh[nt][1], smem_u32(ps_hi + off));
+          if constexpr (kExact) ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
+        }
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt) {
+          const uint32_t xa = mt < 2 ? x0.x : x0.y, xb = mt < 2 ? x1.x : x1.y;
+          const uint32_t ya = mt < 2 ? y0.x : y0.y, yb = mt < 2 ? y1.x : y1.y;
+          constexpr uint32_t kS0 = 0x0400u, kS1 = 0x0501u, kS2 = 0x0602u, kS3 = 0x0703u;   // byte b of a, byte b of b
+          const uint32_t s0 = (mt & 1) ? kS2 : kS0, s1 = (mt & 1) ? kS3 : kS1;
+          const uint32_t a0 = i8_pair_bytes(__byte_perm(xa, xb, s0)), a1 = i8_pair_bytes(__byte_perm(xa, xb, s1));
+          const uint32_t a2 = i8_pair_bytes(__byte_perm(ya, yb, s0)), a3 = i8_pair_bytes(__byte_perm(ya, yb, s1));
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_16816(o[nt][mt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
+            if constexpr (kExact) mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          }
+        }
+      }
+      continue;
+    }
+    (void)vlo;
     const int wd = 8 * dg + g;                       // the word (8 dims) this lane decodes
     const int wseg = wd >> 2, wofs = (wd & 3) * 4;   // its 16-byte segment and offset
+    auto v_phase = [&](auto lo_tag) {
+    constexpr bool kLo = decltype(lo_tag)::value;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
       const int pb = 64 * ph + 16 * ks + 2 * t;
@@ -433,42 +561,48 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       uint32_t lo01, hi01, lo89, hi89;
       interleave_nibbles(x0, x1, lo01, hi01);
       interleave_nibbles(y0, y1, lo89, hi89);
-      uint32_t bh[NT][2], bl[NT][2];
+      uint32_t bh[NT][2], bl[NT][2] = {};
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int m = (lane >> 3) & 1;
         const int off = (nt * 8 + (lane & 7)) * kPsStride + 64 * ph + 16 * ks + 8 * m;
         ldmatrix_x2(bh[nt][0], bh[nt][1], smem_u32(ps_hi + off));
-        ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
+        if constexpr (kExact) ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
       }
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
-        uint32_t a0, a1, a2, a3;
+        uint32_t a0, a1, a2, a3, r0, r1, r2, r3;
         switch (mt) {
           case 0:
-            a0 = lut_decode<0>(lut, lo01, lane4); a1 = lut_decode<0>(lut, hi01, lane4);
-            a2 = lut_decode<0>(lut, lo89, lane4); a3 = lut_decode<0>(lut, hi89, lane4);
+            lut_decode<0>(lut, lo01, lane8, a0, r0); lut_decode<0>(lut, hi01, lane8, a1, r1);
+            lut_decode<0>(lut, lo89, lane8, a2, r2); lut_decode<0>(lut, hi89, lane8, a3, r3);
             break;
           case 1:
-            a0 = lut_decode<1>(lut, lo01, lane4); a1 = lut_decode<1>(lut, hi01, lane4);
-            a2 = lut_decode<1>(lut, lo89, lane4); a3 = lut_decode<1>(lut, hi89, lane4);
+            lut_decode<1>(lut, lo01, lane8, a0, r0); lut_decode<1>(lut, hi01, lane8, a1, r1);
+            lut_decode<1>(lut, lo89, lane8, a2, r2); lut_decode<1>(lut, hi89, lane8, a3, r3);
             break;
           case 2:
-            a0 = lut_decode<2>(lut, lo01, lane4); a1 = lut_decode<2>(lut, hi01, lane4);
-            a2 = lut_decode<2>(lut, lo89, lane4); a3 = lut_decode<2>(lut, hi89, lane4);
+            lut_decode<2>(lut, lo01, lane8, a0, r0); lut_decode<2>(lut, hi01, lane8, a1, r1);
+            lut_decode<2>(lut, lo89, lane8, a2, r2); lut_decode<2>(lut, hi89, lane8, a3, r3);
             break;
           default:
-            a0 = lut_decode<3>(lut, lo01, lane4); a1 = lut_decode<3>(lut, hi01, lane4);
-            a2 = lut_decode<3>(lut, lo89, lane4); a3 = lut_decode<3>(lut, hi89, lane4);
+            lut_decode<3>(lut, lo01, lane8, a0, r0); lut_decode<3>(lut, hi01, lane8, a1, r1);
+            lut_decode<3>(lut, lo89, lane8, a2, r2); lut_decode<3>(lut, hi89, lane8, a3, r3);
             break;
         }
+        // O'^T += (C_hi + C_lo)^T (P'_hi + P'_lo), less the C_lo P'_lo term (and, with bf16
+        // outputs, less P'_lo, and less C_lo where the chunk's V norms are all small)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816(o[nt][mt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-          mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          if constexpr (kExact) mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          if constexpr (kLo) mma_16816(o[nt][mt], r0, r1, r2, r3, bh[nt][0], bh[nt][1]);
         }
       }
     }
+    };
+    if (vlo) v_phase(std::true_type{});
+    else v_phase(std::false_type{});
   }
   cp_async_wait<0>();
 
@@ -642,12 +776,17 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const D
       o[6] = fmaf(a, v1.z, o[6]); o[7] = fmaf(a, v1.w, o[7]);
     }
   }
-  // o = R^T (o' / l) = diag(s) H (o' / l) / 16
-  warp_fwht256(o);
-  const float inv = (L > 0.f) ? 0.0625f / L : 0.f;
   float res[8];
+  if (p.rotate) {   // o = R^T (o' / l) = diag(s) H (o' / l) / 16
+    warp_fwht256(o);
+    const float inv = (L > 0.f) ? 0.0625f / L : 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) res[i] = o[i] * inv * sign_of(p.signs, lane * 8 + i);
+    for (int i = 0; i < 8; ++i) res[i] = o[i] * inv * sign_of(p.signs, lane * 8 + i);
+  } else {          // the INT8 arm attends in the original domain: o = o' / l
+    const float inv = (L > 0.f) ? 1.f / L : 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) res[i] = o[i] * inv;
+  }
   const int64_t off = ((int64_t(r) * p.n_q + tok) * kHq + qh) * kD + lane * 8;
   if (p.out_dtype == TQ4_DTYPE_F32) {
     float* dst = static_cast<float*>(p.out) + off;

@@ -26,6 +26,7 @@
 //     after both have arrived on an mbarrier (normally long before it gets there).
 #pragma once
 #include <cuda.h>
+#include <type_traits>
 #include "tq4_decode.cuh"
 #include "tq4_encode.cuh"
 
@@ -60,7 +61,7 @@ static_assert(kQ1MergeBytes <= (kQ1Bufs - kQ1LowBufs) * kQ1Buf, "merge area fits
 static_assert(kQ1DynBytes <= 227 * 1024, "fits the per-CTA shared memory");
 constexpr float kQ1PScale = 1.0f / 256.0f;   // P' = p * n_v / 256 (undone when the partial is written)
 constexpr float kQ1Lazy = 8.0f;              // rescale only when a row max grows by > 2^8 (log2 units)
-constexpr uint32_t kQ1SpinLimit = 1u << 24;  // bounded wait on a tile's arrival
+constexpr uint32_t kQ1DrainPolls = TQ4_DEFAULT_WAIT_POLLS;  // drain of a copy still in flight at exit
 
 constexpr size_t decode_q1_smem_bytes() { return kQ1DynBytes; }
 
@@ -89,11 +90,12 @@ __device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
 __device__ __forceinline__ void st_shared_u32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a), "r"(v) : "memory");
 }
-// byte K of w -> f16x2 centroid pair from the table at kQ1Lut
+// byte K of w -> the hi and lo f16x2 centroid pairs from the table at kQ1Lut
+// (lanebase = kQ1Lut | 8 * lane: one byte permute forms the slot address)
 template <int K>
-__device__ __forceinline__ uint32_t lut64k(uint32_t w, uint32_t lanebase) {
+__device__ __forceinline__ void lut64k(uint32_t w, uint32_t lanebase, uint32_t& hi, uint32_t& lo) {
   constexpr uint32_t sel = (7u << 12) | (6u << 8) | (uint32_t(K) << 4) | 4u;
-  return ld_shared_u32(__byte_perm(w, lanebase, sel));
+  ld_shared_v2(__byte_perm(w, lanebase, sel), hi, lo);
 }
 
 // ---- mbarrier and bulk-copy primitives (one CTA = its own cluster; no multicast)
@@ -128,6 +130,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // K words (4 heads x 256 slots), V words, then 32 rows of norms.
 constexpr int kRowsPerPage = int(kPageBytes / 128);   // 2,080
 
+template <bool kExact>   // fp32 outputs: every product (see kVloNorm)
 __global__ void __launch_bounds__(kQ1Threads, 1)
     decode_q1_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -144,19 +147,17 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   __half* qv_hi = reinterpret_cast<__half*>(smem + kQ1QvOff);
   __half* qv_lo = qv_hi + 8 * kQvStride;
   auto buf_addr = [&](int b) { return b < kQ1LowBufs ? low0 + b * kQ1Buf : kQ1Hi + (b - kQ1LowBufs) * kQ1Buf; };
-  const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 4u);
+  const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 8u);
 
   // prologue that reads none of the call's inputs (overlaps the previous kernel)
   const uint32_t bar_new = base + 8;   // the fused append's new position is in the pool (count 2)
   if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
   if (tid == kQ1Bufs) mbar_init(bar_new, 2);
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  {   // table rows through shuffles: lane l holds c[l & 15]
-    const uint32_t cl = g_codebook.c16[lane & 15];
-    for (int b = w; b < 256; b += kQ1Warps) {
-      const uint32_t lo = __shfl_sync(0xffffffffu, cl, b & 15), hi = __shfl_sync(0xffffffffu, cl, b >> 4);
-      st_shared_u32(kQ1Lut + b * 256 + lane * 4, lo | (hi << 16));
-    }
+  // table rows: every lane's 8-byte slot of row b holds {c16 pair, r16 pair}
+  for (int b = w; b < 256; b += kQ1Warps) {
+    const uint2 v = lut_row(b);
+    asm volatile("st.shared.v2.b32 [%0], {%1,%2};\n" ::"r"(kQ1Lut + b * 256 + lane * 8), "r"(v.x), "r"(v.y) : "memory");
   }
   __syncthreads();   // barriers initialised before any warp arms one
   pdl_wait();
@@ -234,16 +235,17 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     const int c = tile_pos(k);
     return (k < my_tiles && (c >> 8) < p.max_pages) ? __ldg(table + (c >> 8)) : -1;
   };
+  // (test hook: the first tile's copy is withheld, so the wait on it runs out)
   auto issue_tile = [&](int k, int32_t page) {
-    if (lane == 0 && k < my_tiles) {
+    if (lane == 0 && k < my_tiles && !(p.test_withhold && k == 0)) {
       const int c = tile_pos(k);
       const int b = w * kQ1Stages + (k % kQ1Stages);
       const uint32_t bar = base + kQ1BarOff + b * 8;
       if (append_here && w == last_w && k == last_k) {   // the tile with the appended position
         uint32_t spins = 0;
-        while (!mbar_try_wait(bar_new, 0) && ++spins < kQ1SpinLimit) {
+        while (!mbar_try_wait(bar_new, 0) && ++spins < p.spin_limit) {
         }
-        if (spins >= kQ1SpinLimit) record_error(p.status, TQ4_ERR_TIMEOUT);
+        if (spins >= p.spin_limit) record_error(p.status, TQ4_ERR_TIMEOUT);
       }
       if (page < 0 || page >= p.num_pages) {
         record_error(p.status, TQ4_ERR_PAGE_RANGE);
@@ -297,14 +299,14 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   __syncthreads();
   if (encoder && !encode_first) fused_encode();   // after the block-wide barrier: no warp waits for it
 
-  uint32_t qh[16][2], ql[16][2];
+  // q'_hi B fragments stay in registers; the q'_lo fragments are read from shared
+  // memory two k-steps at a time inside the K phase (registers are the limit)
+  uint32_t qh[16][2];
+  const int qfrag_off = (lane & 7) * kQvStride + ((lane >> 4) & 1) * 16 + ((lane >> 3) & 1) * 8;
+  const uint32_t ql_addr = smem_u32(qv_lo + qfrag_off);
 #pragma unroll
-  for (int kk = 0; kk < 16; kk += 2) {
-    const int m = lane >> 3;
-    const int off = (lane & 7) * kQvStride + (kk + (m >> 1)) * 16 + (m & 1) * 8;
-    ldmatrix_x4(qh[kk][0], qh[kk][1], qh[kk + 1][0], qh[kk + 1][1], smem_u32(qv_hi + off));
-    ldmatrix_x4(ql[kk][0], ql[kk][1], ql[kk + 1][0], ql[kk + 1][1], smem_u32(qv_lo + off));
-  }
+  for (int kk = 0; kk < 16; kk += 2)
+    ldmatrix_x4(qh[kk][0], qh[kk][1], qh[kk + 1][0], qh[kk + 1][1], smem_u32(qv_hi + qfrag_off + kk * 16));
 
   const bool row_ok0 = 2 * t < 6, row_ok1 = 2 * t + 1 < 6;   // query heads 2t, 2t+1
   float m_ref[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
@@ -322,6 +324,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   const uint32_t v_off0 = pv0 * 128 + ((g ^ (pv0 & 7)) << 4);        // words 4g..4g+3 of position pv0
   const uint32_t v_off1 = pv1 * 128 + ((g ^ (pv1 & 7)) << 4);
   bool timed_out = false;
+  int k_stop = my_tiles;   // first tile not consumed (a timeout stops the walk early)
 
   for (int k = 0; k < my_tiles; ++k) {
     issue_tile(k + 1, page_next);
@@ -331,10 +334,11 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     {
       uint32_t spins = 0;
       while (!mbar_try_wait(bar, (k / kQ1Stages) & 1)) {
-        if (++spins > kQ1SpinLimit) { timed_out = true; break; }
+        if (++spins > p.spin_limit) { timed_out = true; break; }
       }
       if (__any_sync(0xffffffffu, timed_out)) {
         if (lane == 0) record_error(p.status, TQ4_ERR_TIMEOUT);
+        k_stop = k;
         break;
       }
     }
@@ -352,29 +356,35 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       kc[j] = ld_shared_v4(mrow + 8 * 128 + k_off0);
       kd[j] = ld_shared_v4(mrow + 8 * 128 + k_off1);
     }
+    // S = (C_hi + C_lo)(q'_hi + q'_lo): sc = C_hi q'_hi, sd = C_hi q'_lo + C_lo q'_hi
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    uint32_t ql4[4];
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
+      if ((kk & 1) == 0) ldmatrix_x4(ql4[0], ql4[1], ql4[2], ql4[3], ql_addr + kk * 32);
+      const uint32_t ql0 = ql4[2 * (kk & 1)], ql1 = ql4[2 * (kk & 1) + 1];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const uint32_t wg = pick(ka[j], kb4[j], kk >> 1);
         const uint32_t wg8 = pick(kc[j], kd[j], kk >> 1);
-        uint32_t a0, a1, a2, a3;
+        uint32_t a0, a1, a2, a3, r0, r1, r2, r3;
         if (kk & 1) {
-          a0 = lut64k<2>(wg, lanebase); a1 = lut64k<2>(wg8, lanebase);
-          a2 = lut64k<3>(wg, lanebase); a3 = lut64k<3>(wg8, lanebase);
+          lut64k<2>(wg, lanebase, a0, r0); lut64k<2>(wg8, lanebase, a1, r1);
+          lut64k<3>(wg, lanebase, a2, r2); lut64k<3>(wg8, lanebase, a3, r3);
         } else {
-          a0 = lut64k<0>(wg, lanebase); a1 = lut64k<0>(wg8, lanebase);
-          a2 = lut64k<1>(wg, lanebase); a3 = lut64k<1>(wg8, lanebase);
+          lut64k<0>(wg, lanebase, a0, r0); lut64k<0>(wg8, lanebase, a1, r1);
+          lut64k<1>(wg, lanebase, a2, r2); lut64k<1>(wg8, lanebase, a3, r3);
         }
         mma_16816(sc[j], a0, a1, a2, a3, qh[kk][0], qh[kk][1]);
-        mma_16816(sd[j], a0, a1, a2, a3, ql[kk][0], ql[kk][1]);
+        mma_16816(sd[j], a0, a1, a2, a3, ql0, ql1);
+        mma_16816(sd[j], r0, r1, r2, r3, qh[kk][0], qh[kk][1]);
       }
     }
 
     // ------------------------------------------------------------ online softmax over 32 positions
     float s[2][4], kn[2][2], vn[2][2];
+    bool vbig = false;   // a visible position of this lane has a V norm above kVloNorm
 #pragma unroll
     for (int j = 0; j < 2; ++j)
 #pragma unroll
@@ -383,6 +393,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         kn[j][e] = __half2float(__ushort_as_half(ld_shared_u16(nb + 2 * pos)));
         vn[j][e] = __half2float(__ushort_as_half(ld_shared_u16(nb + 64 + 2 * pos))) * kQ1PScale;
         const bool ok = c + pos < pos_e;
+        vbig |= ok && vn[j][e] > kVloNorm * kQ1PScale;
         s[j][2 * e] = (ok && row_ok0) ? (sc[j][2 * e] + sd[j][2 * e]) * kn[j][e] * kLog2e : -INFINITY;
         s[j][2 * e + 1] = (ok && row_ok1) ? (sc[j][2 * e + 1] + sd[j][2 * e + 1]) * kn[j][e] * kLog2e : -INFINITY;
       }
@@ -421,7 +432,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     }
     const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
     const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
-    uint32_t bh[2][2], bl[2][2];
+    uint32_t bh[2][2], bl[2][2] = {{0u, 0u}, {0u, 0u}};
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       float pw[4];
@@ -438,16 +449,22 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       const float w2 = s[j][2] == -INFINITY ? 0.f : pw[2] * vn[j][1];
       const float w3 = s[j][3] == -INFINITY ? 0.f : pw[3] * vn[j][1];
       const __half2 h01 = __floats2half2_rn(w0, w1), h23 = __floats2half2_rn(w2, w3);
-      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-      const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
-      const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
       bh[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
       bh[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-      bl[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l01));
-      bl[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l23));
+      if constexpr (kExact) {
+        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+        const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
+        const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
+        bl[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l01));
+        bl[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l23));
+      }
     }
 
     // ------------------------------------------------------------ V phase (all 256 dims), two k-steps
+    // O'^T += (C_hi + C_lo)^T (P'_hi + P'_lo) less C_lo P'_lo; with bf16 outputs
+    // without P'_lo, and without C_lo on tiles whose V norms are all small (kVloNorm)
+    auto v_phase = [&](auto lo_tag) {
+    constexpr bool kLo = decltype(lo_tag)::value;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       const uint32_t vrow = vst + j * 16 * 128;
@@ -462,39 +479,45 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         interleave_nibbles(pick(y0, y0, q), pick(y1, y1, q), lo89, hi89);
 #pragma unroll
         for (int kb_ = 0; kb_ < 4; ++kb_) {
-          uint32_t a0, a1, a2, a3;
+          uint32_t a0, a1, a2, a3, r0, r1, r2, r3;
           switch (kb_) {
             case 0:
-              a0 = lut64k<0>(lo01, lanebase); a1 = lut64k<0>(hi01, lanebase);
-              a2 = lut64k<0>(lo89, lanebase); a3 = lut64k<0>(hi89, lanebase);
+              lut64k<0>(lo01, lanebase, a0, r0); lut64k<0>(hi01, lanebase, a1, r1);
+              lut64k<0>(lo89, lanebase, a2, r2); lut64k<0>(hi89, lanebase, a3, r3);
               break;
             case 1:
-              a0 = lut64k<1>(lo01, lanebase); a1 = lut64k<1>(hi01, lanebase);
-              a2 = lut64k<1>(lo89, lanebase); a3 = lut64k<1>(hi89, lanebase);
+              lut64k<1>(lo01, lanebase, a0, r0); lut64k<1>(hi01, lanebase, a1, r1);
+              lut64k<1>(lo89, lanebase, a2, r2); lut64k<1>(hi89, lanebase, a3, r3);
               break;
             case 2:
-              a0 = lut64k<2>(lo01, lanebase); a1 = lut64k<2>(hi01, lanebase);
-              a2 = lut64k<2>(lo89, lanebase); a3 = lut64k<2>(hi89, lanebase);
+              lut64k<2>(lo01, lanebase, a0, r0); lut64k<2>(hi01, lanebase, a1, r1);
+              lut64k<2>(lo89, lanebase, a2, r2); lut64k<2>(hi89, lanebase, a3, r3);
               break;
             default:
-              a0 = lut64k<3>(lo01, lanebase); a1 = lut64k<3>(hi01, lanebase);
-              a2 = lut64k<3>(lo89, lanebase); a3 = lut64k<3>(hi89, lanebase);
+              lut64k<3>(lo01, lanebase, a0, r0); lut64k<3>(hi01, lanebase, a1, r1);
+              lut64k<3>(lo89, lanebase, a2, r2); lut64k<3>(hi89, lanebase, a3, r3);
               break;
           }
           mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bh[j][0], bh[j][1]);
-          mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bl[j][0], bl[j][1]);
+          if constexpr (kExact) mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bl[j][0], bl[j][1]);
+          if constexpr (kLo) mma_16816(o[4 * q + kb_], r0, r1, r2, r3, bh[j][0], bh[j][1]);
         }
       }
     }
+    };
+    if (kExact || __any_sync(0xffffffffu, vbig)) v_phase(std::true_type{});
+    else v_phase(std::false_type{});
     __syncwarp();   // all lanes are done with this buffer before lane 0 refills it
   }
 
-  // drain: a warp that broke out early still has at most one tile in flight; wait for it (bounded)
-  if (my_tiles > 0) {
-    const int last = my_tiles - 1;
-    const int b = w * kQ1Stages + (last % kQ1Stages);
+  // drain: a warp that stopped early at tile k_stop may still have the copies of
+  // tiles k_stop and k_stop + 1 in flight (tile k + 1 is issued before tile k is
+  // waited for); wait for them before the buffers are reused or the CTA exits
+  for (int k = k_stop; k < min(k_stop + kQ1Stages, my_tiles); ++k) {
+    if (p.test_withhold && k == 0) continue;   // never issued
+    const int b = w * kQ1Stages + (k % kQ1Stages);
     uint32_t spins = 0;
-    while (!mbar_try_wait(base + kQ1BarOff + b * 8, (last / kQ1Stages) & 1) && ++spins < kQ1SpinLimit) {
+    while (!mbar_try_wait(base + kQ1BarOff + b * 8, (k / kQ1Stages) & 1) && ++spins < kQ1DrainPolls) {
     }
   }
 

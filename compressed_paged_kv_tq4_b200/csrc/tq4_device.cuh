@@ -28,13 +28,16 @@ constexpr int64_t kVWords = int64_t(kHkv) * kPage * kWords * 4;   // 131072
 constexpr int64_t kKNorms = 2 * kVWords;                           // 262144
 constexpr int64_t kVNorms = kKNorms + int64_t(kHkv) * kPage * 2;   // 264192
 
-// codebook in constant memory, written by the host from its fp64 Lloyd-Max
-// solution rounded to the stored fp16 table (same for every context; the signs
-// are per context)
+// Codebook in constant memory, written by the host from its fp64 Lloyd-Max
+// solution (the same for every context; the signs are per context).
+// The attention kernels feed the centroids to f16 tensor-core products as a
+// hi + lo pair: c16 = f16(c), r16 = f16(c - c16), so c16 + r16 carries c to
+// about 2^-21 relative while each half is an exact f16 operand.
 struct Codebook {
-  float c[16];        // stored centroids (exact fp16 values held in fp32)
-  float b[15];        // decision boundaries: midpoints of adjacent stored centroids (exact in fp32)
-  uint16_t c16[16];   // stored centroids as fp16 bits (round to nearest even of the fp64 solution)
+  float c[16];        // centroids rounded to fp32 (reconstruction)
+  float b[15];        // decision boundaries: fp64 midpoints of adjacent centroids, rounded to fp32 (encode)
+  uint16_t c16[16];   // f16 bits of the centroids (round to nearest even)
+  uint16_t r16[16];   // f16 bits of the rounding residuals c - c16
 };
 __constant__ Codebook g_codebook;  // one translation unit (tq4_api.cu) includes every kernel header
 
@@ -103,9 +106,9 @@ __device__ __forceinline__ float sign_of(const Signs& s, int coord) {
 // --------------------------------------------------------------------------
 // Nibble-pair decode through a per-lane table in shared memory.
 // Row b (one byte = two 4-bit indices) is 256 bytes; lane l reads its own
-// 4-byte slot at b*256 + 4*l (and b*256 + 128 + 4*l for the low-order part),
-// so the 32 lanes of a warp always hit 32 different banks. A slot holds
-// f16x2 {c[b & 15], c[b >> 4]}.
+// 8-byte slot at b*256 + 8*l, so a warp's 64-bit loads are two conflict-free
+// wavefronts. A slot holds f16x2 {c16[b & 15], c16[b >> 4]} followed by
+// f16x2 {r16[b & 15], r16[b >> 4]} (the hi and lo halves of the centroids).
 // --------------------------------------------------------------------------
 constexpr int kLutBytes = 256 * 256;
 
@@ -115,25 +118,35 @@ __device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
   asm volatile("ld.shared.b32 %0, [%1];\n" : "=r"(v) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ void ld_shared_v2(uint32_t addr, uint32_t& x, uint32_t& y) {
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];\n" : "=r"(x), "=r"(y) : "r"(addr));
+}
 
-// byte k (0..3) of w -> f16x2 of its two nibbles (low nibble in the low half).
+// byte k (0..3) of w -> hi and lo f16x2 of its two nibbles (low nibble in the low half).
 // lut_s is the table's 32-bit shared address; the byte lands in bits 8..15 of
-// the offset and the lane's slot in bits 0..7.
+// the offset and the lane's slot (8 * lane) in bits 0..7.
 template <int K>
-__device__ __forceinline__ uint32_t lut_decode(uint32_t lut_s, uint32_t w, uint32_t lane4) {
+__device__ __forceinline__ void lut_decode(uint32_t lut_s, uint32_t w, uint32_t lane8, uint32_t& hi,
+                                           uint32_t& lo) {
   constexpr uint32_t sel = (5u << 12) | (5u << 8) | (uint32_t(K) << 4) | 4u;
-  return ld_shared_u32(lut_s + __byte_perm(w, lane4, sel));
+  ld_shared_v2(lut_s + __byte_perm(w, lane8, sel), hi, lo);
+}
+
+// One table row b as the 8-byte slot every lane stores: {c pair, r pair}.
+__device__ __forceinline__ uint2 lut_row(int b) {
+  return make_uint2(uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16),
+                    uint32_t(g_codebook.r16[b & 15]) | (uint32_t(g_codebook.r16[b >> 4]) << 16));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Scores are q' . c with q' = R q * scale carried as an f16 hi + lo pair. The
-// prefill (bf16 outputs) computes the lo product (q'lo C^T) for a tile only when
-// one of its keys has a norm above kQloNorm: below it, the error the f16 q' leaves
-// in a score is about 2.5e-5 * ||k|| in log2 units (std over the rounding), far
-// below what moves a bf16 output by the tolerance. Keys 16 s with s in [0.5, 2]
-// stay under ~34; the 8x outliers of the long-context workload start at 64.
-constexpr float kQloNorm = 48.0f;
+// With bf16 outputs the attention kernels skip the products that a bf16 result
+// cannot resolve: P' lo (the f16 rounding of the softmax weights) always, and the
+// centroid residual of the V side (C_lo P') on tiles whose V norms all stay at or
+// below kVloNorm. The keys always take all three score terms. Norms 16 s with s in
+// [0.5, 2] stay under ~34; the 8x outliers of the long-context workload start at
+// 64. fp32 outputs run every product.
+constexpr float kVloNorm = 48.0f;
 
 // 16-byte global -> shared copies that bypass registers (generic proxy; wait before use)
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {

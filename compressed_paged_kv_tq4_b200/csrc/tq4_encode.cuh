@@ -177,7 +177,68 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(
   reinterpret_cast<float4*>(dst)[1] = make_float4(o[4], o[5], o[6], o[7]);
 }
 
+// Uniform INT8 comparison arm: per head vector, scale s = max |x_i| / 127 and codes
+// round-half-even(x_i / s), in double precision (the divisions and the rounding are
+// those of an fp64 reference, so the codes come out bit-identical); the scale is
+// stored as fp16. Page layout: K codes [4][256][256] int8, V codes, K scales
+// [4][256] fp16, V scales. One warp per vector; lane l owns dims 8l .. 8l + 7.
+template <typename T>
+__global__ void __launch_bounds__(256) int8_encode_kernel(
+    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table, int32_t start_pos,
+    int32_t n_tok, const T* __restrict__ k_new, const T* __restrict__ v_new, int* status) {
+  constexpr int64_t kPB = TQ4_INT8_PAGE_BYTES;
+  constexpr int64_t kVC = int64_t(kHkv) * kPage * kD, kKS = 2 * kVC, kVS = kKS + int64_t(kHkv) * kPage * 2;
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (vec >= int64_t(n_tok) * 2 * kHkv) return;
+  const int tok = int(vec / (2 * kHkv));
+  const int kv = int(vec / kHkv) & 1;
+  const int head = int(vec % kHkv);
+  float x[8];
+  load8<T>((kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8, x);
+  float am = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(x[i]));
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
+  const double sc = double(am) / 127.0;
+  uint32_t w[2] = {0u, 0u};
+  if (am > 0.f) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int q = __double2int_rn(double(x[i]) / sc);
+      w[i >> 2] |= (uint32_t(q) & 0xFFu) << (8 * (i & 3));
+    }
+  }
+  const int32_t pos = start_pos + tok;
+  const int32_t page = __ldg(page_table + (pos >> 8));
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+    return;
+  }
+  const int slot = head * kPage + (pos & (kPage - 1));
+  uint8_t* base = pool + int64_t(page) * kPB;
+  *reinterpret_cast<uint2*>(base + (kv ? kVC : 0) + int64_t(slot) * kD + lane * 8) = make_uint2(w[0], w[1]);
+  if (lane == 0) reinterpret_cast<__half*>(base + (kv ? kVS : kKS))[slot] = __double2half(sc);
+}
+
 // ---------------------------------------------------------------- launchers
+cudaError_t launch_int8_encode_append(uint8_t* pool, int32_t num_pages, const int32_t* page_table,
+                                      int32_t start_pos, int32_t n_tok, const void* k_new, const void* v_new,
+                                      int dtype, int* status, cudaStream_t stream) {
+  const int threads = 256, wpb = threads / 32;
+  const unsigned blocks = unsigned((int64_t(n_tok) * 2 * kHkv + wpb - 1) / wpb);
+  if (dtype == TQ4_DTYPE_F32)
+    return launch_pdl(int8_encode_kernel<float>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                      page_table, start_pos, n_tok, static_cast<const float*>(k_new),
+                      static_cast<const float*>(v_new), status);
+  return launch_pdl(int8_encode_kernel<uint16_t>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                    page_table, start_pos, n_tok, static_cast<const uint16_t*>(k_new),
+                    static_cast<const uint16_t*>(v_new), status);
+}
+
 cudaError_t launch_encode_append(uint8_t* pool, int32_t num_pages, const int32_t* page_table,
                                  int32_t start_pos, int32_t n_tok, const void* k_new,
                                  const void* v_new, int dtype, const Signs& signs, int* status,

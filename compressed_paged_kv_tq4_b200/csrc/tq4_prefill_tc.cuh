@@ -1,4 +1,5 @@
-// TQ4 prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+// TQ4 prefill attention on the 5th-generation tensor cores (tcgen05 + TMEM),
+// one CTA pair per 256 query rows (cta_group::2), sm_100a.
 //
 // What it computes ([KVEXEC] simpleprog.com "Fitting a 27B-Parameter LLM into
 // 24 GiB of Laptop Memory", section "KVExec": multi-query prefill reconstructs
@@ -10,72 +11,84 @@
 // K norm scales score columns, the V norm is folded into P); chunk keys/values
 // are R k, R v; each output row gets R^T once at the end.
 //
-// One CTA = 128 query rows (row = token * 6 + head within the KV head's group)
-// of one KV head, walking KV tiles of 64 positions.
+// Precision. Every tensor-core operand is an f16 hi + lo pair: q' = q'hi + q'lo,
+// a centroid c = c16 + r16 (c16 = f16(c), r16 = f16(c - c16)), chunk rows
+// likewise, P = Phi + Plo. The scores take the three terms that matter
+// (q'hi Khi + q'lo Khi + q'hi Klo); O takes Phi Vhi, plus Phi Vlo on tiles whose
+// largest V norm exceeds kVloNorm, plus Plo Vhi and Phi Vlo on every tile when
+// the output is fp32 (the fp32 check holds the result to ~1e-5 relative).
+//
+// Work split. A cluster of two CTAs (ranks 0 and 1) owns 256 query rows
+// (row = token * 6 + head within the KV head's group; rank r holds rows
+// 128 r .. 128 r + 127, one per TMEM lane) of one KV head and walks KV tiles of
+// 64 positions. The pair's MMAs have M = 256: A (q' or P) is split by rows, B by
+// its N columns and each CTA keeps its 128 rows of D. So each CTA expands only
+// half of every tile: K for positions 32 r .. 32 r + 31 (all 256 dims) and V for
+// dims 128 r .. 128 r + 127 (all 64 positions).
 //   warps 0-3   softmax: thread i of warp w owns row 32w + i = TMEM lane. Puts
-//               its q' hi row into TMEM and its q' lo row into shared memory. Reads
-//               its score row from TMEM, applies K norms, the causal mask and an
-//               online softmax with a lazily raised reference; writes
-//               P = p * n_v / 256 back into TMEM as an f16 hi + lo pair (the two
-//               halves keep P V at fp32-level precision); final epilogue.
-//   warps 4-11  dequant, two groups of four warps; group g fills the shared
-//               stage g for tiles j = g, g+2, ... : packed words are prefetched
-//               into registers one tile ahead, expanded through a per-lane
-//               centroid table (32 KiB: row = one byte of indices, one 4-byte slot
-//               per lane) into f16 panels [4 dim blocks][64 positions][128 B]
-//               with the 128-byte swizzle; the chunk's own K/V are copied.
-//   warp 12     one thread issues tcgen05.mma: S = Q'hi K^T (+ Q'lo K^T where the
-//               tile needs it; A = Q'hi in TMEM, A = Q'lo in shared memory; B = K
-//               panels, K-major) and
-//               O += P V (A = P in TMEM, B = V panels, MN-major), in the order
-//               QK(j), PV(j-1), so the tensor pipe holds the next score tile while
-//               the softmax runs.
-// TMEM (512 columns): Q'hi [0,128), S/P buffers [128,192) and [192,256), O [256,512).
-// The q' hi + lo pair keeps the scores at fp32-level precision: with a single f16
-// q', the score error grows with the key norm, and keys with 8x norms move
-// softmax weights by about 1%.
-// Every wait is bounded; on a timeout the CTA records TQ4_ERR_TIMEOUT, skips the
-// remaining work, drains its issued MMAs, frees its TMEM and returns.
+//               its q' hi row into TMEM and its q' lo row into shared memory.
+//               Reads its score row from TMEM, applies K norms, the causal mask
+//               and an online softmax with a lazily raised reference; writes
+//               P = p * n_v / 256 over S (f16 hi, and lo for fp32 outputs).
+//   warps 4-11  dequant, two groups of four; group g fills stage g for tiles
+//               g, g+2, ...: packed words are prefetched into registers two
+//               tiles ahead and expanded through a per-lane table of 8-byte
+//               {hi pair, lo pair} slots into swizzled f16 panels (K hi, K lo,
+//               V hi, V lo); chunk rows are copied from the prologue's output.
+//   warp 12     rank 0 only: one thread issues every tcgen05.mma of the pair, in
+//               the order QK(j), PV(j-1), and commits to both CTAs' barriers.
+// TMEM (512 columns per CTA): q'hi [0,128), S/P buffers [128,192) and
+// [192,256), O [256,512).
+// Producers signal the issuer through barriers in rank 0's shared memory (lane 0
+// of each producer warp arrives after the warp's writes, from either CTA); the
+// issuer's commits arrive on both CTAs' barriers. Every wait is bounded by
+// spin_limit polls; on a timeout the CTA records TQ4_ERR_TIMEOUT, raises the
+// abort flag of both CTAs, skips the remaining work, drains its issued MMAs and
+// frees its TMEM after a cluster barrier.
 #pragma once
 #include "tq4_device.cuh"
 #include "tq4_prefill.cuh"
 
 namespace tq4 {
 
-constexpr int kTcRows = 128;
-constexpr int kTcTile = 64;                              // KV positions per tile
-constexpr int kTcSoftWarps = 4, kTcDeqWarps = 8;
-constexpr int kTcMmaWarp = kTcSoftWarps + kTcDeqWarps;   // 12
-constexpr int kTcThreads = 32 * (kTcMmaWarp + 1);        // 416
-constexpr int kTcGroupThreads = 128;                     // one dequant group
-constexpr int kTcUnits = 8;                              // 16-B word groups per dequant thread per tile
-constexpr int kTcPanel = kTcTile * 128;                  // 8 KiB: 64 positions x 64 dims f16
-constexpr int kTcKV = 4 * kTcPanel;                      // 32 KiB: one K or V tile
-constexpr int kTcStage = 2 * kTcKV;                      // K then V
-constexpr int kTcQloPanel = kTcRows * 128;              // 16 KiB: 128 rows x 64 dims f16
-constexpr int kTcLutBytes = 256 * 128;                   // 256 byte values x 32 lanes x 4 B
-// dynamic shared memory (offsets from the 1 KiB-aligned base)
-constexpr uint32_t kTcStageOff = 0;                      // 2 stages x 64 KiB
-constexpr uint32_t kTcQloOff = 2 * kTcStage;             // q' lo panels [4][128 rows][128 B], 64 KiB
-constexpr uint32_t kTcLutOff = kTcQloOff + 4 * kTcQloPanel;   // 32 KiB per-lane centroid table
-constexpr uint32_t kTcNormOff = kTcLutOff + kTcLutBytes; // [2 stages][K 64, V 64] fp32
-constexpr uint32_t kTcBarOff = kTcNormOff + 2 * 2 * kTcTile * 4;
-constexpr uint32_t kTcMiscOff = kTcBarOff + 128;   // u32 [0] TMEM base, [1] abort; f32 [8 + 4 stage + warp] K norm max
-constexpr uint32_t kTcSmem = kTcMiscOff + 128 + 1024;    // + alignment slack
-constexpr int kTcOsStride = kD + 4;                      // epilogue rows (fp32), reuse the stages + q' lo
-static_assert(uint32_t(kTcRows * kTcOsStride * 4) <= kTcLutOff, "epilogue rows overlap the table");
-static_assert(kTcSmem <= 227u * 1024u, "shared memory");
-static_assert(kTcQloOff % 1024 == 0 && kTcStage % 1024 == 0, "swizzled panels start on 1 KiB");
-static_assert(kTcDeqWarps * 32 == 2 * kTcGroupThreads, "two dequant groups");
-static_assert(kTcGroupThreads * kTcUnits == 2 * kTcTile * 8, "units cover K and V of one tile");
-constexpr uint32_t kTcSpin = 1u << 24;
-constexpr float kTcPScale = 1.0f / 256.0f;   // P carries 1/256, undone in the epilogue
-constexpr float kTcLazy = 8.0f;              // raise the row reference only when the max grows by > 2^8
-// The q' lo correction (Q'lo K^T) runs for a tile when it holds chunk positions or
-// a prefix key whose norm exceeds kQloNorm (see its definition).
+constexpr int kPfRows = 128;                       // query rows per CTA; a pair covers 256
+constexpr int kPfTile = 64;                        // KV positions per tile
+constexpr int kPfKPos = kPfTile / 2;               // K positions each CTA expands per tile
+constexpr int kPfSoftWarps = 4, kPfDeqWarps = 8;
+constexpr int kPfMmaWarp = kPfSoftWarps + kPfDeqWarps;   // 12
+constexpr int kPfThreads = 32 * (kPfMmaWarp + 1);        // 416
+constexpr int kPfGroupThreads = 128;                     // one dequant group
+constexpr uint32_t kPfKPanel = kPfKPos * 128;            // 4 KiB: 32 positions x 64 dims f16
+constexpr uint32_t kPfKPart = 4 * kPfKPanel;             // 16 KiB: K hi (or lo), 4 dim blocks
+constexpr uint32_t kPfVPanel = kPfTile * 128;            // 8 KiB: 64 positions x 64 dims f16
+constexpr uint32_t kPfVPart = 2 * kPfVPanel;             // 16 KiB: V hi (or lo), this CTA's 2 dim blocks
+constexpr uint32_t kPfKHi = 0, kPfKLo = kPfKPart, kPfVHi = 2 * kPfKPart, kPfVLo = 2 * kPfKPart + kPfVPart;
+constexpr uint32_t kPfStage = 2 * kPfKPart + 2 * kPfVPart;   // 64 KiB
+constexpr uint32_t kPfQloPanel = kPfRows * 128;             // 16 KiB: 128 rows x 64 dims f16
+constexpr uint32_t kPfQloOff = 2 * kPfStage;                 // two stages first
+constexpr uint32_t kPfLutOff = kPfQloOff + 4 * kPfQloPanel;
+constexpr uint32_t kPfLutBytes = 256 * 16 * 8;              // 256 byte values x 16 copies x 8 B
+constexpr uint32_t kPfNormOff = kPfLutOff + kPfLutBytes;     // [2 stages][K 64, V 64] f32
+constexpr uint32_t kPfBarOff = kPfNormOff + 2 * 2 * kPfTile * 4;
+constexpr uint32_t kPfMiscOff = kPfBarOff + 256;   // u32 [0] TMEM base, [1] abort; f32 [8 + 2 stage + k] V norm max
+constexpr uint32_t kPfSmem = kPfMiscOff + 128 + 1024;    // + alignment slack
+constexpr int kPfOsStride = kD + 4;                      // epilogue rows (fp32) reuse the stages + q' lo
+static_assert(uint32_t(kPfRows * kPfOsStride * 4) <= kPfLutOff, "epilogue rows overlap the table");
+static_assert(kPfSmem <= 227u * 1024u, "shared memory");
+static_assert(kPfQloOff % 1024 == 0 && kPfStage % 1024 == 0 && kPfKPart % 1024 == 0 && kPfKPanel % 1024 == 0,
+              "swizzled panels start on 1 KiB");
+constexpr float kPfPScale = 1.0f / 256.0f;   // P carries 1/256, undone in the epilogue
+constexpr float kPfLazy = 8.0f;              // raise the row reference only when the max grows by > 2^8
 
 // TMEM columns
 constexpr uint32_t kTmQ = 0, kTmS0 = 128, kTmO = 256;
+
+// barriers (8 B each at kPfBarOff): in rank 0, counted from both CTAs
+constexpr int kBQReady = 0, kBKFull = 1, kBVFull = 3, kBPFull = 5;
+// in each CTA: committed by the issuer to both CTAs, or local
+constexpr int kBSFull = 7, kBKEmpty = 9, kBVEmpty = 11, kBOReady = 13, kBDrain = 14, kBNFull = 15;
+constexpr int kBarriers = 17;
+static_assert(kBarriers * 8 <= 256, "barrier area");
 
 // ---- descriptors (layouts of the PTX ISA's tcgen05 matrix descriptors)
 // instruction descriptor, kind::f16: D f32 (bit 4), A = B = f16 (formats 0),
@@ -90,39 +103,75 @@ __device__ __forceinline__ uint64_t tc_sdesc(uint32_t start, uint32_t lbo, uint3
          (uint64_t((sbo >> 4) & 0x3FFF) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
 }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                       uint32_t accumulate) {
+// pair MMA, A from TMEM (each CTA's rows at the same address)
+__device__ __forceinline__ void tc2_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
+// pair MMA, A from shared memory (each CTA's rows at the same offset)
+__device__ __forceinline__ void tc2_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+// completion of this thread's earlier MMAs -> one arrival on the barrier at this
+// offset in both CTAs of the pair
+__device__ __forceinline__ void tc2_commit_both(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n" ::"r"(
+          bar),
+      "h"(uint16_t(3))
+      : "memory");
+}
+// ... on this CTA's barrier only
+__device__ __forceinline__ void tc2_commit_own(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
                : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+// the shared::cluster address of offset `addr` (a shared::cta address) in CTA `rank`
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// arrive (release, cluster scope) on a barrier given by its shared::cluster address
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_local(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ bool tc_try_wait(uint32_t bar, uint32_t parity) {
+// acquire at cluster scope: arrivals may come from the peer CTA
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t done;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(done)
       : "r"(bar), "r"(parity)
       : "memory");
   return done != 0;
+}
+__device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\nbarrier.cluster.wait.acquire;\n" ::: "memory");
 }
 
 // 32 consecutive TMEM columns of this thread's lane -> 32 registers (load and wait
@@ -158,76 +207,76 @@ __device__ __forceinline__ void tm_st16(uint32_t taddr, const uint32_t (&r)[16])
 }
 __device__ __forceinline__ void tm_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 
-__global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const PrefillParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefill_tc_kernel(const PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t sbase = (raw_s + 1023) & ~1023u;   // the swizzled panels need 1 KiB alignment
   uint8_t* smem = smem_raw + (sbase - raw_s);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const uint32_t rank = cluster_rank();
+  const uint32_t peer = rank ^ 1u;
   const int h = blockIdx.y;
-  const int row0 = blockIdx.x * kTcRows;
+  const int pair_row0 = (blockIdx.x >> 1) * (2 * kPfRows);
+  const int row0 = pair_row0 + int(rank) * kPfRows;
   const int m_total = 6 * p.n_tok;
-  const int last_row = min(row0 + kTcRows, m_total) - 1;
+  const int last_row = min(pair_row0 + 2 * kPfRows, m_total) - 1;   // the pair's last row
   const int kv_end = p.prefix_len + last_row / 6 + 1;
-  const int n_tiles = (kv_end + kTcTile - 1) / kTcTile;
+  const int n_tiles = (kv_end + kPfTile - 1) / kPfTile;
+  const bool exact = p.out_dtype == TQ4_DTYPE_F32;
 
-  // K and V halves of a stage have their own barriers: a K slot is free again as
-  // soon as its QK has run, a V slot once its PV has run. Both norms of a tile are
-  // written with its V half (the softmax of the tile two back may still read them
-  // while the K half is refilled).
-  const uint32_t bar_k_full = sbase + kTcBarOff;    // [2] count 128 (one dequant group)
-  const uint32_t bar_v_full = bar_k_full + 16;      // [2] count 128; also covers both norms
-  const uint32_t bar_k_empty = bar_k_full + 32;     // [2] count 1 (commit after QK)
-  const uint32_t bar_v_empty = bar_k_full + 48;     // [2] count 1 (commit after PV)
-  const uint32_t bar_s_full = bar_k_full + 64;      // [2] count 1 (commit after QK)
-  const uint32_t bar_p_full = bar_k_full + 80;      // [2] count 128 (softmax threads)
-  const uint32_t bar_o_ready = bar_k_full + 96;     // count 1 (commit after PV)
-  const uint32_t bar_drain = bar_k_full + 104;      // count 1 (final commit)
-  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kTcMiscOff);   // [0] TMEM base, [1] abort
-  float* norms = reinterpret_cast<float*>(smem + kTcNormOff);
+  auto bar = [sbase](int i) -> uint32_t { return sbase + kPfBarOff + 8u * uint32_t(i); };
+  volatile uint32_t* misc = reinterpret_cast<volatile uint32_t*>(smem + kPfMiscOff);   // [0] TMEM base, [1] abort
+  float* norms = reinterpret_cast<float*>(smem + kPfNormOff);
+  const uint32_t lead_bar0 = map_to_rank(bar(0), 0);   // rank 0's barrier area, seen from this CTA
 
   if (tid == 0) {
+    mbar_init(bar(kBQReady), 2 * kPfSoftWarps);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_k_full + 8 * b, kTcGroupThreads);
-      mbar_init(bar_v_full + 8 * b, kTcGroupThreads);
-      mbar_init(bar_k_empty + 8 * b, 1);
-      mbar_init(bar_v_empty + 8 * b, 1);
-      mbar_init(bar_s_full + 8 * b, 1);
-      mbar_init(bar_p_full + 8 * b, 32 * kTcSoftWarps);
+      mbar_init(bar(kBKFull + b), 2 * (kPfGroupThreads / 32));
+      mbar_init(bar(kBVFull + b), 2 * (kPfGroupThreads / 32));
+      mbar_init(bar(kBPFull + b), 2 * kPfSoftWarps);
+      mbar_init(bar(kBSFull + b), 1);
+      mbar_init(bar(kBKEmpty + b), 1);
+      mbar_init(bar(kBVEmpty + b), 1);
+      mbar_init(bar(kBNFull + b), kPfGroupThreads / 32);
     }
-    mbar_init(bar_o_ready, 1);
-    mbar_init(bar_drain, 1);
+    mbar_init(bar(kBOReady), 1);
+    mbar_init(bar(kBDrain), 1);
     misc[1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
-  if (w == 0) {   // 512 TMEM columns; shared memory admits one CTA per SM, so no CTA of this kernel competes
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(sbase + kTcMiscOff)
+  if (w == 0) {   // 512 TMEM columns in both CTAs; shared memory admits one CTA per SM
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], 512;\n" ::"r"(sbase + kPfMiscOff)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
   }
-  // per-lane centroid table: row b (a byte = two indices, 128 B) holds f16x2
-  // {c[b & 15], c[b >> 4]} in each lane's 4-byte slot, so a warp's lookups never
-  // share a bank
-  for (int e = tid; e < 256 * 32; e += kTcThreads) {
-    const int b = e >> 5, l = e & 31;
-    reinterpret_cast<uint32_t*>(smem + kTcLutOff)[b * 32 + l] =
-        uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16);
-  }
+  // per-lane centroid table: row b (a byte = two indices, 128 B) holds, in each of
+  // 16 copies, the 8-byte slot {c16 pair, r16 pair}; lanes l and l + 16 share copy
+  // l & 15, so each half warp's 64-bit loads hit 32 different banks
+  for (int e = tid; e < 256 * 16; e += kPfThreads)
+    reinterpret_cast<uint2*>(smem + kPfLutOff)[e] = lut_row(e >> 4);
   pdl_wait();   // q', the chunk rows and the pool may come from the previous kernels
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();   // both CTAs' barriers are initialised before any remote arrival
   tc_fence_after();
   const uint32_t tmem = misc[0];
 
   int* const status = p.status;
-  auto bounded_wait = [misc, status](uint32_t bar, uint32_t parity) -> bool {
+  const uint32_t spin_limit = p.spin_limit;
+  const uint32_t peer_abort = map_to_rank(sbase + kPfMiscOff + 4, peer);
+  auto abort_both = [misc, status, peer_abort]() {
+    misc[1] = 1;
+    st_cluster_u32(peer_abort, 1u);
+    record_error(status, TQ4_ERR_TIMEOUT);
+  };
+  auto bounded_wait = [misc, spin_limit, &abort_both](uint32_t b, uint32_t parity) -> bool {
     uint32_t spins = 0;
-    while (!tc_try_wait(bar, parity)) {
+    while (!mbar_try_wait_cluster(b, parity)) {
       if (misc[1]) return false;
-      if (++spins > kTcSpin) {
-        misc[1] = 1;
-        record_error(status, TQ4_ERR_TIMEOUT);
+      if (++spins > spin_limit) {
+        abort_both();
         return false;
       }
     }
@@ -235,11 +284,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
   };
   // the softmax warps use TMEM loads/stores that all 32 lanes must execute
   // together, so every wait and every decision before one is taken warp-wide
-  auto warp_wait = [&bounded_wait](uint32_t bar, uint32_t parity) -> bool {
-    return __all_sync(0xffffffffu, bounded_wait(bar, parity));
+  auto warp_wait = [&bounded_wait](uint32_t b, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, bounded_wait(b, parity));
+  };
+  // lane 0 signals a producer barrier in rank 0 after the whole warp's writes
+  auto warp_arrive_lead = [lead_bar0, lane](int i) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(lead_bar0 + 8u * uint32_t(i));
   };
 
-  if (w < kTcSoftWarps) {
+  if (w < kPfSoftWarps) {
     // =========================================================== softmax / epilogue
     const int r_local = 32 * w + lane;
     const int row = row0 + r_local;
@@ -248,8 +302,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     const int lim = row_ok ? p.prefix_len + tok + 1 : 0;   // positions [0, lim) are visible
     const uint32_t lane_addr = tmem + (uint32_t(32 * w) << 16);
     {   // q' row -> TMEM columns [0,128) as f16 pairs (A operand of S = Q' K^T)
-      const uint4* src =
-          reinterpret_cast<const uint4*>(p.qr + (int64_t(tok) * kHq + h * kGroup + (row_ok ? row % 6 : 0)) * kD);
+      const int64_t qrow = (int64_t(tok) * kHq + h * kGroup + (row_ok ? row % 6 : 0)) * kD;
+      const uint4* src = reinterpret_cast<const uint4*>(p.qr + qrow);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t v[32];
@@ -265,33 +319,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
       }
       tm_wait_st();
       // q' lo row -> shared panels (K-major, 128-byte swizzle): dims 64 k .. 64 k + 63 in panel k
-      const uint4* src_lo =
-          reinterpret_cast<const uint4*>(p.qlo + (int64_t(tok) * kHq + h * kGroup + (row_ok ? row % 6 : 0)) * kD);
-      uint8_t* qlo_row = smem + kTcQloOff + r_local * 128;
+      const uint4* src_lo = reinterpret_cast<const uint4*>(p.qlo + qrow);
+      uint8_t* qlo_row = smem + kPfQloOff + r_local * 128;
 #pragma unroll 8
       for (int g = 0; g < 32; ++g) {   // g = 16-byte chunk (8 dims)
         const uint4 u = row_ok ? __ldg(src_lo + g) : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(qlo_row + (g >> 3) * kTcQloPanel + (((g & 7) ^ (r_local & 7)) << 4)) = u;
+        *reinterpret_cast<uint4*>(qlo_row + (g >> 3) * kPfQloPanel + (((g & 7) ^ (r_local & 7)) << 4)) = u;
       }
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic-proxy stores -> tensor-core reads
     }
     tc_fence_before();
-    mbar_arrive(bar_p_full + 8);   // extra phase of p_full[1]: q' hi is in TMEM, q' lo in shared memory
+    warp_arrive_lead(kBQReady);
 
     float m_ref = -INFINITY, l_sum = 0.f;
     for (int j = 0; j < n_tiles; ++j) {
       const int b = j & 1;
-      if (!warp_wait(bar_s_full + 8 * b, (j >> 1) & 1)) break;
-      if (!warp_wait(bar_v_full + 8 * b, (j >> 1) & 1)) break;   // V half and both norms of this tile
+      if (!warp_wait(bar(kBSFull + b), (j >> 1) & 1)) break;
+      if (!warp_wait(bar(kBNFull + b), (j >> 1) & 1)) break;   // both norm rows of this tile
       tc_fence_after();
-      const float4* kn4 = reinterpret_cast<const float4*>(norms + b * 2 * kTcTile);   // K norm * log2(e)
-      const float4* vn4 = kn4 + kTcTile / 4;                                          // V norm / 256
-      const int pos0 = j * kTcTile;
+      const float4* kn4 = reinterpret_cast<const float4*>(norms + b * 2 * kPfTile);   // K norm * log2(e)
+      const float4* vn4 = kn4 + kPfTile / 4;                                          // V norm / 256
+      const int pos0 = j * kPfTile;
       uint32_t sr[2][32];
       tm_ld32(lane_addr + kTmS0 + 64 * b, sr[0]);
       tm_ld32(lane_addr + kTmS0 + 64 * b + 32, sr[1]);
       float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // scores in log2 units
-      if (__all_sync(0xffffffffu, pos0 + kTcTile <= lim)) {           // the whole tile is visible
+      if (__all_sync(0xffffffffu, pos0 + kPfTile <= lim)) {           // the whole tile is visible
 #pragma unroll
         for (int g = 0; g < 16; ++g) {
           const float4 k = kn4[g];
@@ -318,7 +371,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         }
       }
       const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-      const bool raise = mx > m_ref + kTcLazy;   // raise the reference: rescale l and the O row accumulated so far
+      const bool raise = mx > m_ref + kPfLazy;   // raise the reference: rescale l and the O row accumulated so far
       float alpha = 1.f;
       if (raise) {
         alpha = fast_exp2(m_ref - mx);
@@ -326,7 +379,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         l_sum *= alpha;
       }
       if (j > 0 && __any_sync(0xffffffffu, raise)) {   // warp-wide; lanes that keep their reference use alpha = 1
-        if (!warp_wait(bar_o_ready, (j - 1) & 1)) break;   // PV(j-1) has completed
+        if (!warp_wait(bar(kBOReady), (j - 1) & 1)) break;   // PV(j-1) has completed
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 8; ++c) {
@@ -352,30 +405,34 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
         }
       }
       l_sum += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      // P hi (columns 0-31: positions 2k, 2k+1 in column k) and P lo = P - f16(P)
-      // (columns 32-63), written over the scores in halves of 32 positions
+      // P hi (columns 0-31: positions 2k, 2k+1 in column k) and, for fp32 outputs,
+      // P lo = P - f16(P) (columns 32-63), written over the scores in halves of 32 positions
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]), __uint_as_float(sr[c][2 * k + 1]));
         tm_st16(lane_addr + kTmS0 + 64 * b + 16 * c, pk);
+        if (exact) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
-          pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]) - hi.x, __uint_as_float(sr[c][2 * k + 1]) - hi.y);
+          for (int k = 0; k < 16; ++k) {
+            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
+            pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]) - hi.x, __uint_as_float(sr[c][2 * k + 1]) - hi.y);
+          }
+          tm_st16(lane_addr + kTmS0 + 64 * b + 32 + 16 * c, pk);
         }
-        tm_st16(lane_addr + kTmS0 + 64 * b + 32 + 16 * c, pk);
       }
       tm_wait_st();
       tc_fence_before();
-      mbar_arrive(bar_p_full + 8 * b);
+      // (test hook: tile min(1, n_tiles - 1)'s P signal is withheld, so the issuer's
+      // wait for it runs out after some MMAs of the pair have been issued)
+      if (!(p.test_withhold && j == min(1, n_tiles - 1))) warp_arrive_lead(kBPFull + b);
     }
     // ---- O / l -> shared memory rows (reusing the stages): wait for the last PV
-    const bool ok = __all_sync(0xffffffffu, misc[1] == 0) && warp_wait(bar_o_ready, (n_tiles - 1) & 1);
+    const bool ok = __all_sync(0xffffffffu, misc[1] == 0) && warp_wait(bar(kBOReady), (n_tiles - 1) & 1);
     tc_fence_after();
-    float* os = reinterpret_cast<float*>(smem + kTcStageOff) + r_local * kTcOsStride;
-    const float inv = (ok && l_sum > 0.f) ? (0.0625f / kTcPScale) / l_sum : 0.f;   // 1/256 of P and 1/16 of R^T
+    float* os = reinterpret_cast<float*>(smem) + r_local * kPfOsStride;
+    const float inv = (ok && l_sum > 0.f) ? (0.0625f / kPfPScale) / l_sum : 0.f;   // 1/256 of P and 1/16 of R^T
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       uint32_t ov[32];
@@ -390,198 +447,240 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
             make_float4(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv,
                         __uint_as_float(ov[i + 2]) * inv, __uint_as_float(ov[i + 3]) * inv);
     }
-  } else if (w < kTcMmaWarp) {
+  } else if (w < kPfMmaWarp) {
     // =========================================================== dequant groups
-    const int grp_id = (w - kTcSoftWarps) >> 2;                 // stage b == grp_id, tiles j = grp_id, +2, ...
-    const int gt = tid - 32 * kTcSoftWarps - kTcGroupThreads * grp_id;   // 0..127
-    // unit u of this thread: 16 bytes (4 words = 32 dims) of one position's K or V.
-    // A quarter warp covers 4 positions x 2 adjacent word groups, so its 16-B
-    // shared stores land in 8 distinct bank groups under the swizzle.
-    const int grp = (lane & 1) | (((lane >> 3) & 3) << 1);     // word group 0..7 -> dims 32 grp ..
-    const int pl_lo = (lane >> 1) & 3;
-    const char* lut = reinterpret_cast<const char*>(smem + kTcLutOff);
-    const uint32_t lane8 = uint32_t(lane) * 8u;   // (byte << 8 | 8 lane) >> 1 = byte * 128 + 4 lane
+    const int grp_id = (w - kPfSoftWarps) >> 2;                           // stage b == grp_id
+    const int gt = tid - 32 * kPfSoftWarps - kPfGroupThreads * grp_id;   // 0..127
+    const int wq = gt >> 5;                                               // warp within the group
+    // K units: 16 bytes (4 words = 32 dims) of one of this CTA's 32 positions. A
+    // quarter warp covers 4 positions x 2 adjacent word groups, so its 16-B stores
+    // land in 8 distinct bank groups under the swizzle.
+    const int kgrp = (lane & 1) | (((lane >> 3) & 3) << 1);   // word group 0..7 -> dims 32 kgrp ..
+    const int kpl_lo = (lane >> 1) & 3;
+    // V units: 16 bytes of this CTA's 128 dims (word groups 4 rank .. 4 rank + 3) of one
+    // of the tile's 64 positions; again 4 positions x 2 word groups per quarter warp
+    const int vgrp = (lane & 1) | (((lane >> 4) & 1) << 1);   // local word group 0..3
+    const int vpl_lo = ((lane >> 1) & 3) | (((lane >> 3) & 1) << 2);
+    const uint32_t lut_s = sbase + kPfLutOff;
+    const uint32_t lane16 = uint32_t(lane & 15) * 16u;   // (byte << 8 | 16 copy) >> 1 = byte * 128 + 8 copy
     const int prefix_end = min(p.prefix_len, kv_end);
-    uint8_t* st = smem + kTcStageOff + grp_id * kTcStage;
-    float* nb = norms + grp_id * 2 * kTcTile;
-
-    // raw[u] holds unit u's packed words for the tile about to be expanded (units
-    // 0-3: K, 4-7: V); each register is refilled with the group's next tile (j + 2)
-    // right after use, so the loads fly while the stage is waited for. A tile lies
-    // in one page; its page id is loaded two tiles ahead of use.
-    uint4 raw[kTcUnits];
-    float rawn[kTcUnits];
+    const uint32_t st_s = sbase + grp_id * kPfStage;
+    float* nb = norms + grp_id * 2 * kPfTile;
     const uint8_t* const pool = p.pool;
     const int32_t* const page_table = p.page_table;
     const int32_t num_pages = p.num_pages;
-    auto page_of = [=](int j) -> int32_t {
-      return (j < n_tiles && j * kTcTile < prefix_end) ? __ldg(page_table + ((j * kTcTile) >> 8)) : 0;
+
+    // tile-local position and source word group of unit u (0, 1: K; 2, 3: V)
+    auto unit_pos = [=](int u) -> int {
+      return u < 2 ? int(rank) * kPfKPos + 4 * (wq + 4 * u) + kpl_lo : 8 * (wq + 4 * (u - 2)) + vpl_lo;
     };
-    auto fetch = [&raw, &rawn, gt, pl_lo, prefix_end, pool, num_pages, h, grp, status](int j, int u, int32_t page) {
-      const int q = (gt >> 5) + 4 * u;   // 0..31: bit 4 = V, bits 0-3 = position group
-      const int kv = q >> 4, pos = j * kTcTile + 4 * (q & 15) + pl_lo;
+    auto unit_grp = [=](int u) -> int { return u < 2 ? kgrp : 4 * int(rank) + vgrp; };
+    // raw[u]: unit u's packed words for the tile about to be expanded; rawn: the norm
+    // this thread loads for the tile (K norm of position gt for gt < 64, V norm of
+    // position gt - 64 otherwise). Refilled with the group's next tile (j + 2) right
+    // after use, so the loads fly while the stage is waited for. A tile lies in one
+    // page; its page id is loaded two tiles ahead of use.
+    uint4 raw[4];
+    float rawn = 0.f;
+    auto page_of = [=](int j) -> int32_t {
+      return (j < n_tiles && j * kPfTile < prefix_end) ? __ldg(page_table + ((j * kPfTile) >> 8)) : 0;
+    };
+    auto fetch = [&raw, prefix_end, pool, num_pages, h, status, &unit_pos, &unit_grp](int j, int u, int32_t page) {
+      const int pos = j * kPfTile + unit_pos(u);
       raw[u] = make_uint4(0, 0, 0, 0);
-      rawn[u] = 0.f;
       if (pos < prefix_end) {
         if (page >= 0 && page < num_pages) {
           const uint8_t* pg = pool + int64_t(page) * kPageBytes;
           const int slot = h * kPage + (pos & (kPage - 1));
-          raw[u] = ldg128(pg + (kv ? kVWords : kKWords) + int64_t(slot) * 128 + grp * 16);
-          if (grp == 0) rawn[u] = ldg_half(pg + (kv ? kVNorms : kKNorms) + slot * 2);
-        } else if (grp == 0) {
+          raw[u] = ldg128(pg + (u < 2 ? kKWords : kVWords) + int64_t(slot) * 128 + unit_grp(u) * 16);
+        } else {
           record_error(status, TQ4_ERR_PAGE_RANGE);   // words stay 0 and the norm 0: no contribution
         }
       }
     };
-    // expand unit u of tile j into the stage: centroid values for a prefix position,
-    // an asynchronous copy of the prologue's f16 row for a chunk position, zeros past
-    // the CTA's last visible position. Returns the unit's norm (1 for chunk rows: the
-    // rotated row carries its own length; 0 past the end).
-    auto expand = [&](int j, int u) -> float {
-      const int q = (gt >> 5) + 4 * u;
-      const int kv = q >> 4, pl = 4 * (q & 15) + pl_lo, pos = j * kTcTile + pl;
-      // dims 32 grp .. +31 = panel grp / 2, 16-B chunks 4 (grp & 1) .. +3 of row pl, 128-byte swizzle
-      uint8_t* prow = st + kv * kTcKV + (grp >> 1) * kTcPanel + pl * 128;
-      const int sw = pl & 7, c0 = (grp & 1) * 4;
+    auto fetch_norm = [&rawn, gt, prefix_end, pool, num_pages, h](int j, int32_t page) {
+      const int pos = j * kPfTile + (gt & 63);
+      rawn = 0.f;
+      if (pos < prefix_end && page >= 0 && page < num_pages)
+        rawn = ldg_half(pool + int64_t(page) * kPageBytes + (gt < 64 ? kKNorms : kVNorms) +
+                        (h * kPage + (pos & (kPage - 1))) * 2);
+    };
+    // expand unit u of tile j into the stage: hi and lo centroid values for a prefix
+    // position, asynchronous copies of the prologue's hi and lo rows for a chunk
+    // position, zeros past the pair's last visible position
+    auto expand = [&](int j, int u) {
+      const int pl = unit_pos(u), pos = j * kPfTile + pl;
+      const int g = u < 2 ? kgrp : vgrp;   // word group within the panels of this CTA
+      const int sw = pl & 7, c0 = (g & 1) * 4;
+      const int prow = (u < 2 ? pl - int(rank) * kPfKPos : pl) * 128;
+      const uint32_t hi_s = st_s + (u < 2 ? kPfKHi + (g >> 1) * kPfKPanel : kPfVHi + (g >> 1) * kPfVPanel) + prow;
+      const uint32_t lo_s = hi_s + (u < 2 ? kPfKLo - kPfKHi : kPfVLo - kPfVHi);
       if (pos < prefix_end) {
         const uint32_t ww[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {   // word c = dims 8c .. 8c + 7 of the span
-          const uint32_t a = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5504u) >> 1));
-          const uint32_t b = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5514u) >> 1));
-          const uint32_t d = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5524u) >> 1));
-          const uint32_t e = *reinterpret_cast<const uint32_t*>(lut + (__byte_perm(ww[c], lane8, 0x5534u) >> 1));
-          *reinterpret_cast<uint4*>(prow + (((c0 + c) ^ sw) << 4)) = make_uint4(a, b, d, e);
+          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+          ld_shared_v2(lut_s + (__byte_perm(ww[c], lane16, 0x5504u) >> 1), h0, l0);
+          ld_shared_v2(lut_s + (__byte_perm(ww[c], lane16, 0x5514u) >> 1), h1, l1);
+          ld_shared_v2(lut_s + (__byte_perm(ww[c], lane16, 0x5524u) >> 1), h2, l2);
+          ld_shared_v2(lut_s + (__byte_perm(ww[c], lane16, 0x5534u) >> 1), h3, l3);
+          const uint32_t off = uint32_t(((c0 + c) ^ sw) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(hi_s + off), "r"(h0), "r"(h1), "r"(h2),
+                       "r"(h3)
+                       : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(lo_s + off), "r"(l0), "r"(l1), "r"(l2),
+                       "r"(l3)
+                       : "memory");
         }
-        return rawn[u];
+        return;
       }
       if (pos < kv_end) {
-        const __half* src = (kv ? p.vr : p.kr) + (int64_t(pos - p.prefix_len) * kHkv + h) * kD + 32 * grp;
+        const int64_t row = (int64_t(pos - p.prefix_len) * kHkv + h) * kD + 32 * unit_grp(u);
+        const __half* src_hi = (u < 2 ? p.kr : p.vr) + row;
+        const __half* src_lo = (u < 2 ? p.krlo : p.vrlo) + row;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) cp_async16(smem_u32(prow + (((c0 + c) ^ sw) << 4)), src + 8 * c);
-        return 1.f;
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t off = uint32_t(((c0 + c) ^ sw) << 4);
+          cp_async16(hi_s + off, src_hi + 8 * c);
+          cp_async16(lo_s + off, src_lo + 8 * c);
+        }
+        return;
       }
 #pragma unroll
-      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(prow + (((c0 + c) ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
-      return 0.f;
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t off = uint32_t(((c0 + c) ^ sw) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};\n" ::"r"(hi_s + off), "r"(0u) : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};\n" ::"r"(lo_s + off), "r"(0u) : "memory");
+      }
     };
     int32_t pg_next = 0;   // page of tile j + 2
     if (grp_id < n_tiles) {
       const int32_t pg0 = page_of(grp_id);
       pg_next = page_of(grp_id + 2);
 #pragma unroll
-      for (int u = 0; u < kTcUnits; ++u) fetch(grp_id, u, pg0);
+      for (int u = 0; u < 4; ++u) fetch(grp_id, u, pg0);
+      fetch_norm(grp_id, pg0);
     }
-    volatile float* kmax = reinterpret_cast<volatile float*>(misc) + 8 + 4 * grp_id;
+    volatile float* vmax_slot = reinterpret_cast<volatile float*>(misc) + 8 + 2 * grp_id;
     for (int j = grp_id; j < n_tiles; j += 2) {
       const int32_t pg_far = page_of(j + 4);
       const bool more = j + 2 < n_tiles;
-      const bool chunk_rows = (j + 1) * kTcTile > prefix_end;   // this tile reaches the chunk (or past it)
-      float kn[4];
       // ---- K half: free once QK(j - 2) has run
-      if (j >= 2 && !bounded_wait(bar_k_empty + 8 * grp_id, ((j >> 1) - 1) & 1)) break;
-      float big = chunk_rows ? INFINITY : 0.f;   // largest K norm; chunk rows always take the q' lo pass
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        kn[u] = expand(j, u);
-        big = fmaxf(big, kn[u]);
-      }
+      if (j >= 2 && !bounded_wait(bar(kBKEmpty + grp_id), ((j >> 1) - 1) & 1)) break;
+      expand(j, 0);
+      expand(j, 1);
       cp_async_commit();
       cp_async_wait<0>();
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) big = fmaxf(big, __shfl_xor_sync(0xffffffffu, big, o));
-      if (lane == 0) kmax[(w - kTcSoftWarps) & 3] = big;   // read by the MMA thread after k_full
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic-proxy writes -> tensor-core reads
-      mbar_arrive(bar_k_full + 8 * grp_id);
+      warp_arrive_lead(kBKFull + grp_id);
       // the next tile's loads go out only now: the wait and the proxy fence above
       // would otherwise wait for them as well
       if (more) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) fetch(j + 2, u, pg_next);
+        fetch(j + 2, 0, pg_next);
+        fetch(j + 2, 1, pg_next);
       }
-      // ---- V half and both norms: free once PV(j - 2) has run
-      if (j >= 2 && !bounded_wait(bar_v_empty + 8 * grp_id, ((j >> 1) - 1) & 1)) break;
+      // ---- V half and both norm rows: free once PV(j - 2) has run
+      if (j >= 2 && !bounded_wait(bar(kBVEmpty + grp_id), ((j >> 1) - 1) & 1)) break;
+      expand(j, 2);
+      expand(j, 3);
+      {
+        const int pl = gt & 63;
+        const bool chunk = j * kPfTile + pl >= prefix_end && j * kPfTile + pl < kv_end;
+        const float n = chunk ? 1.f : rawn;   // chunk rows carry their own length
+        if (gt < 64) {
+          nb[pl] = n * kLog2e;
+        } else {
+          nb[kPfTile + pl] = n * kPfPScale;
+          float m = chunk ? 16.f : n;   // a rotated N(0,1) chunk row has length ~16
 #pragma unroll
-      for (int u = 4; u < 8; ++u) {
-        const float vn = expand(j, u);
-        if (grp == 0) {
-          const int pl = 4 * (((gt >> 5) + 4 * u) & 15) + pl_lo;
-          nb[pl] = kn[u - 4] * kLog2e;
-          nb[kTcTile + pl] = vn * kTcPScale;
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          if (lane == 0) vmax_slot[wq - 2] = m;   // read by the issuer after v_full
         }
       }
       cp_async_commit();
       cp_async_wait<0>();
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
-      mbar_arrive(bar_v_full + 8 * grp_id);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_local(bar(kBNFull + grp_id));
+      warp_arrive_lead(kBVFull + grp_id);
       if (more) {
-#pragma unroll
-        for (int u = 4; u < 8; ++u) fetch(j + 2, u, pg_next);
+        fetch(j + 2, 2, pg_next);
+        fetch(j + 2, 3, pg_next);
+        fetch_norm(j + 2, pg_next);
       }
       pg_next = pg_far;
     }
-  } else {
-    // =========================================================== MMA issuer (one thread)
+  } else if (rank == 0) {
+    // =========================================================== MMA issuer (one thread of rank 0)
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = tc_idesc(kTcRows, kTcTile, 0);
-      constexpr uint32_t idesc_pv = tc_idesc(kTcRows, kD, 1);
-      bool ok = bounded_wait(bar_p_full + 8, 0);   // Q' stored
+      constexpr uint32_t idesc_qk = tc_idesc(2 * kPfRows, kPfTile, 0);
+      constexpr uint32_t idesc_pv = tc_idesc(2 * kPfRows, kD, 1);
+      bool ok = bounded_wait(bar(kBQReady), 0);   // q' of both CTAs stored
       tc_fence_after();
       for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {   // S[j & 1] = Q'hi K_j^T + Q'lo K_j^T  (K = 256 dims in 16 steps each)
+        if (j < n_tiles) {   // S[j & 1] = Q'hi Khi^T + Q'lo Khi^T + Q'hi Klo^T  (K = 256 dims in 16 steps each)
           const int b = j & 1;
-          if (!bounded_wait(bar_k_full + 8 * b, (j >> 1) & 1)) break;
+          if (!bounded_wait(bar(kBKFull + b), (j >> 1) & 1)) break;
           tc_fence_after();
-          const uint32_t kbase = sbase + kTcStageOff + b * kTcStage;
+          const uint32_t kb = sbase + b * kPfStage;
+          const uint32_t s_t = tmem + kTmS0 + 64 * b;
 #pragma unroll
           for (int kk = 0; kk < 16; ++kk) {
-            const uint64_t bd = tc_sdesc(kbase + (kk >> 2) * kTcPanel + (kk & 3) * 32, 16, 1024);
-            tc_mma(tmem + kTmS0 + 64 * b, tmem + kTmQ + 8 * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            const uint64_t bd = tc_sdesc(kb + kPfKHi + (kk >> 2) * kPfKPanel + (kk & 3) * 32, 16, 1024);
+            tc2_mma_ts(s_t, tmem + kTmQ + 8 * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
           }
-          const volatile float* km = reinterpret_cast<const volatile float*>(misc) + 8 + 4 * b;
-          if (fmaxf(fmaxf(km[0], km[1]), fmaxf(km[2], km[3])) > kQloNorm) {
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-              const uint64_t ad = tc_sdesc(sbase + kTcQloOff + (kk >> 2) * kTcQloPanel + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = tc_sdesc(kbase + (kk >> 2) * kTcPanel + (kk & 3) * 32, 16, 1024);
-              tc_mma_ss(tmem + kTmS0 + 64 * b, ad, bd, idesc_qk, 1u);
+          for (int kk = 0; kk < 16; ++kk) {
+            const uint64_t ad = tc_sdesc(sbase + kPfQloOff + (kk >> 2) * kPfQloPanel + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = tc_sdesc(kb + kPfKHi + (kk >> 2) * kPfKPanel + (kk & 3) * 32, 16, 1024);
+            tc2_mma_ss(s_t, ad, bd, idesc_qk, 1u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < 16; ++kk) {
+            const uint64_t bd = tc_sdesc(kb + kPfKLo + (kk >> 2) * kPfKPanel + (kk & 3) * 32, 16, 1024);
+            tc2_mma_ts(s_t, tmem + kTmQ + 8 * kk, bd, idesc_qk, 1u);
+          }
+          tc2_commit_both(bar(kBSFull + b));
+          tc2_commit_both(bar(kBKEmpty + b));
+        }
+        if (j >= 1) {   // O += P_hi V_hi (+ P_lo V_hi, + P_hi V_lo) for tile j - 1 (K = 64 positions in 4 steps)
+          const int jb = j - 1, b = jb & 1;
+          if (!bounded_wait(bar(kBPFull + b), (jb >> 1) & 1)) break;
+          if (!bounded_wait(bar(kBVFull + b), (jb >> 1) & 1)) break;
+          tc_fence_after();
+          const volatile float* vm = reinterpret_cast<const volatile float*>(misc) + 8 + 2 * b;
+          const bool vlo = exact || fmaxf(vm[0], vm[1]) > kVloNorm;
+          const uint32_t vb = sbase + b * kPfStage;
+          const uint32_t p_t = tmem + kTmS0 + 64 * b;
+#pragma unroll
+          for (int ks = 0; ks < kPfTile / 16; ++ks) {
+            const uint64_t bh = tc_sdesc(vb + kPfVHi + ks * 16 * 128, kPfVPanel, 1024);
+            tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, bh, idesc_pv, (jb > 0 || ks > 0) ? 1u : 0u);
+            if (exact) tc2_mma_ts(tmem + kTmO, p_t + 32 + 8 * ks, bh, idesc_pv, 1u);
+            if (vlo) {
+              const uint64_t bl = tc_sdesc(vb + kPfVLo + ks * 16 * 128, kPfVPanel, 1024);
+              tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, bl, idesc_pv, 1u);
             }
           }
-          tc_commit(bar_s_full + 8 * b);
-          tc_commit(bar_k_empty + 8 * b);
-        }
-        if (j >= 1) {   // O += P_hi V + P_lo V for tile j - 1 (K = 64 positions in 4 steps)
-          const int jb = j - 1, b = jb & 1;
-          // p_full[1] completed one extra phase for Q': its tile phases are shifted by one
-          const uint32_t par = b ? (((jb >> 1) + 1) & 1) : ((jb >> 1) & 1);
-          if (!bounded_wait(bar_p_full + 8 * b, par)) break;
-          if (!bounded_wait(bar_v_full + 8 * b, (jb >> 1) & 1)) break;
-          tc_fence_after();
-          const uint32_t vbase = sbase + kTcStageOff + b * kTcStage + kTcKV;
-#pragma unroll
-          for (int ks = 0; ks < kTcTile / 16; ++ks) {
-            const uint64_t bd = tc_sdesc(vbase + ks * 16 * 128, kTcPanel, 1024);
-            tc_mma(tmem + kTmO, tmem + kTmS0 + 64 * b + 8 * ks, bd, idesc_pv, (jb > 0 || ks > 0) ? 1u : 0u);
-            tc_mma(tmem + kTmO, tmem + kTmS0 + 64 * b + 32 + 8 * ks, bd, idesc_pv, 1u);
-          }
-          tc_commit(bar_v_empty + 8 * b);
-          tc_commit(bar_o_ready);
+          tc2_commit_both(bar(kBVEmpty + b));
+          tc2_commit_both(bar(kBOReady));
         }
       }
       // every MMA this thread issued has completed before TMEM is released
-      tc_commit(bar_drain);
-      for (uint32_t spins = 0; !tc_try_wait(bar_drain, 0) && spins < kTcSpin; ++spins) {
+      tc2_commit_own(bar(kBDrain));
+      for (uint32_t spins = 0; !mbar_try_wait_cluster(bar(kBDrain), 0) && spins < TQ4_DEFAULT_WAIT_POLLS; ++spins) {
       }
     }
     __syncwarp();
   }
 
-  // =========================================================== R^T per row, bf16 out; free TMEM
+  // =========================================================== R^T per row, out; free TMEM
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();   // no MMA of the pair and no remote access is outstanding past this point
   tc_fence_after();
-  if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;\n" ::"r"(tmem) : "memory");
-  const float* os = reinterpret_cast<const float*>(smem + kTcStageOff);
+  if (w == 0) asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, 512;\n" ::"r"(tmem) : "memory");
+  const float* os = reinterpret_cast<const float*>(smem);
   uint32_t sgn = 0;   // sign bits of coordinates 8 lane .. 8 lane + 7 (constant indices keep p in registers)
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -590,44 +689,54 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(const Prefill
     sgn = ((lane >> 2) == k) ? wk : sgn;
   }
   sgn = (sgn >> (8 * (lane & 3))) & 0xFFu;
-  for (int rl = w; rl < kTcRows; rl += kTcThreads / 32) {
+  for (int rl = w; rl < kPfRows; rl += kPfThreads / 32) {
     const int row = row0 + rl;
     if (row >= m_total) break;
     float v[8];
-    const float4 a = *reinterpret_cast<const float4*>(os + rl * kTcOsStride + lane * 8);
-    const float4 c = *reinterpret_cast<const float4*>(os + rl * kTcOsStride + lane * 8 + 4);
+    const float4 a = *reinterpret_cast<const float4*>(os + rl * kPfOsStride + lane * 8);
+    const float4 c = *reinterpret_cast<const float4*>(os + rl * kPfOsStride + lane * 8 + 4);
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
     warp_fwht256(v);
-    uint32_t pk[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(__float_as_uint(v[2 * i]) ^ (((sgn >> (2 * i)) & 1u) << 31)),
-                                                __uint_as_float(__float_as_uint(v[2 * i + 1]) ^ (((sgn >> (2 * i + 1)) & 1u) << 31)));
-      pk[i] = *reinterpret_cast<uint32_t*>(&b2);
-    }
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((sgn >> i) & 1u) << 31));
     const int tok = row / 6, jh = row % 6;
-    *reinterpret_cast<uint4*>(p.out + (int64_t(tok) * kHq + h * kGroup + jh) * kD + lane * 8) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    const int64_t off = (int64_t(tok) * kHq + h * kGroup + jh) * kD + lane * 8;
+    if (exact) {
+      float* dst = static_cast<float*>(p.out) + off;
+      reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    } else {
+      uint32_t pk[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        pk[i] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
   }
 }
 
 inline cudaError_t prefill_tc_set_attrs() {
-  return cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kTcSmem));
+  return cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPfSmem));
 }
 
-// rotate prologue, then the tcgen05 attention kernel
+// rotate prologue, then the tcgen05 attention kernel (clusters of two CTAs)
 inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,
                                      int32_t prefix_len, const uint16_t* q, const uint16_t* kc,
-                                     const uint16_t* vc, int32_t n_tok, float scale, uint16_t* out,
-                                     void* workspace, const Signs& signs, int* status, cudaStream_t stream) {
+                                     const uint16_t* vc, int32_t n_tok, float scale, void* out, int out_dtype,
+                                     void* workspace, const Signs& signs, int* status, uint32_t spin_limit,
+                                     int test_withhold, cudaStream_t stream) {
   __half* qr = static_cast<__half*>(workspace);
   __half* qlo = qr + size_t(n_tok) * kHq * kD;
   __half* kr = qlo + size_t(n_tok) * kHq * kD;
-  __half* vr = kr + size_t(n_tok) * kHkv * kD;
+  __half* krlo = kr + size_t(n_tok) * kHkv * kD;
+  __half* vr = krlo + size_t(n_tok) * kHkv * kD;
+  __half* vrlo = vr + size_t(n_tok) * kHkv * kD;
   const int64_t vecs = int64_t(n_tok) * (kHq + 2 * kHkv);
   cudaError_t e = launch_pdl(prefill_rotate_kernel, dim3(unsigned((vecs + 7) / 8)), dim3(256), 0, stream, q, kc, vc,
-                             n_tok, scale, qr, qlo, kr, vr, signs);
+                             n_tok, scale, qr, qlo, kr, krlo, vr, vrlo, signs);
   if (e != cudaSuccess) return e;
   PrefillParams p{};
   p.pool = pool;
@@ -638,12 +747,17 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
   p.qr = qr;
   p.qlo = qlo;
   p.kr = kr;
+  p.krlo = krlo;
   p.vr = vr;
+  p.vrlo = vrlo;
   p.out = out;
+  p.out_dtype = out_dtype;
   p.signs = signs;
   p.status = status;
-  const dim3 grid(unsigned((6 * n_tok + kTcRows - 1) / kTcRows), kHkv);
-  return launch_pdl(prefill_tc_kernel, grid, dim3(kTcThreads), size_t(kTcSmem), stream, p);
+  p.spin_limit = spin_limit;
+  p.test_withhold = test_withhold;
+  const unsigned pairs = unsigned((6 * n_tok + 2 * kPfRows - 1) / (2 * kPfRows));
+  return launch_pdl(prefill_tc_kernel, dim3(2 * pairs, kHkv), dim3(kPfThreads), size_t(kPfSmem), stream, p);
 }
 
 }  // namespace tq4

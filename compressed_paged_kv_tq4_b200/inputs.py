@@ -93,6 +93,34 @@ def kv_vectors(config: int, layer: int, n_pos: int, *, outlier_frac: float = 0.0
     return k, v
 
 
+def kv_vectors_device(config: int, layer: int, n_pos: int, *, outlier_frac: float = 0.0,
+                      outlier_scale: float = 8.0, request: int = 0, device="cuda"):
+    """K and V head vectors with the distribution of ``kv_vectors``, drawn on the
+    GPU with torch's generator: fp32 tensors [n_pos, 4, 256] each.
+
+    Each vector is z * s with z ~ N(0, I_256) and s ~ U(0.5, 2); a seeded
+    ``outlier_frac`` of positions has s multiplied by ``outlier_scale`` for all of
+    its K and V vectors. The stream differs from ``kv_vectors`` (same law, other
+    numbers); it fills the benchmark's multi-GB caches, where only the law
+    matters. Parity tests use ``kv_vectors``.
+    """
+    import torch
+    seed = int(np.random.SeedSequence([SEED_BASE + int(config), _KV + 16 * int(request), int(layer)])
+               .generate_state(1, dtype=np.uint64)[0] & ((1 << 63) - 1))
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    k = torch.randn((n_pos, H_KV, D), generator=g, device=device, dtype=torch.float32)
+    v = torch.randn((n_pos, H_KV, D), generator=g, device=device, dtype=torch.float32)
+    sk = torch.rand((n_pos, H_KV, 1), generator=g, device=device) * 1.5 + 0.5
+    sv = torch.rand((n_pos, H_KV, 1), generator=g, device=device) * 1.5 + 0.5
+    if outlier_frac > 0.0:
+        mask = (torch.rand((n_pos, 1, 1), generator=g, device=device) < outlier_frac).float()
+        boost = 1.0 + (outlier_scale - 1.0) * mask
+        sk = sk * boost
+        sv = sv * boost
+    return k * sk, v * sv
+
+
 def queries(config: int, layer: int, shape) -> np.ndarray:
     """N(0,1) queries rounded to bf16; returns uint16 bits of the given shape."""
     r = _rng(config, _Q, layer)
@@ -143,7 +171,7 @@ class Workload:
     pool_pages: int
     seq_lens: tuple          # attended positions per request (new positions included)
     n_q: int                 # query tokens per request (decode) or chunk length (prefill)
-    kind: str                # "decode" or "prefill"
+    kind: str                # "decode", "decode_int8" (the INT8 comparison arm) or "prefill"
     outlier_frac: float = 0.0
     append_per_step: int = 0  # positions appended by tq4_encode_append per layer per step
     shared_prefix_pages: int = 0
@@ -166,6 +194,9 @@ WORKLOADS = {
     # 2 requests (163,840 and 65,536 positions; first 64 pages shared), 4 causal query tokens each
     "verify_2req_229k": Workload("verify_2req_229k", 3, 16, POOL_PAGES, (163_840, 65_536), 4,
                                  "decode", shared_prefix_pages=64, append_per_step=4),
+    # the uniform INT8 comparison arm on the decode_32k shape (same config, same law of K/V)
+    "int8_decode_32k": Workload("int8_decode_32k", 1, 16, POOL_PAGES, (32768,), 1, "decode_int8",
+                                append_per_step=1),
     # prefill: 2,048 causal query tokens against a 32,768-position TQ4 prefix + the chunk
     "prefill_2k_on_32k": Workload("prefill_2k_on_32k", 4, 16, POOL_PAGES, (32_768 + 2048,), 2048,
                                   "prefill", prefix_len=32_768, append_per_step=2048),

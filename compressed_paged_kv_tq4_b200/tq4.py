@@ -31,6 +31,8 @@ KV_HEADS = 4
 Q_HEADS = 24
 PAGE_BYTES = 266240
 POSITION_BYTES = 1040
+INT8_PAGE_BYTES = 528384
+INT8_POSITION_BYTES = 2064
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
@@ -39,13 +41,14 @@ EXPORTS = (
     "tq4_ctx_create", "tq4_ctx_destroy", "tq4_codebook", "tq4_encode_append", "tq4_reconstruct",
     "tq4_decode_workspace_bytes", "tq4_decode_attention", "tq4_prefill_workspace_bytes",
     "tq4_prefill_attention", "tq4_get_status", "tq4_status_string", "tq4_decode_attention_noalloc",
-    "tq4_decode_append_attention",
+    "tq4_decode_append_attention", "tq4_ctx_set_wait_limit", "tq4_int8_encode_append", "tq4_int8_decode_attention",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
     "tq4_pages_available", "tq4_pages_refcount", "tq4_pages_free_list",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
+DEFAULT_WAIT_POLLS = 1 << 24
 
 
 def _load():
@@ -73,8 +76,12 @@ _sig = {
     "tq4_decode_attention": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int,
                               _p, _sz, _p], ctypes.c_int),
     "tq4_prefill_workspace_bytes": ([_i32], _sz),
-    "tq4_prefill_attention": ([_p, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p, _p, _sz, _p],
-                              ctypes.c_int),
+    "tq4_prefill_attention": ([_p, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p, ctypes.c_int, _p, _sz,
+                               _p], ctypes.c_int),
+    "tq4_ctx_set_wait_limit": ([_p, ctypes.c_uint32, ctypes.c_int], ctypes.c_int),
+    "tq4_int8_encode_append": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p], ctypes.c_int),
+    "tq4_int8_decode_attention": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int,
+                                   _p, _sz, _p], ctypes.c_int),
     "tq4_get_status": ([_p, _p], ctypes.c_int),
     "tq4_decode_attention_noalloc": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int, _p],
                                      ctypes.c_int),
@@ -191,10 +198,28 @@ def tq4_prefill_workspace_bytes(n_tok) -> int:
 
 
 def tq4_prefill_attention(ctx, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk, v_chunk,
-                          n_tok, scale, out, workspace, workspace_bytes, stream=None) -> int:
+                          n_tok, scale, out, out_dtype, workspace, workspace_bytes, stream=None) -> int:
     return _lib.tq4_prefill_attention(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, prefix_len,
-                                      _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale, _ptr(out),
+                                      _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale, _ptr(out), out_dtype,
                                       _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_int8_encode_append(ctx, pool, num_pages, page_table, table_len, start_pos, n_tok, k_new, v_new,
+                           dtype, stream=None) -> int:
+    return _lib.tq4_int8_encode_append(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, start_pos,
+                                       n_tok, _ptr(k_new), _ptr(v_new), dtype, _stream(stream))
+
+
+def tq4_int8_decode_attention(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
+                              total_seq_len, scale, out, out_dtype, workspace, workspace_bytes,
+                              stream=None) -> int:
+    return _lib.tq4_int8_decode_attention(ctx, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
+                                          _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out),
+                                          out_dtype, _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_ctx_set_wait_limit(ctx, polls, withhold_signal=0) -> int:
+    return _lib.tq4_ctx_set_wait_limit(ctx, polls, withhold_signal)
 
 
 def tq4_decode_attention_noalloc(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
@@ -342,6 +367,11 @@ class Context:
     def status(self, stream=None) -> int:
         return tq4_get_status(self.handle, stream)
 
+    def set_wait_limit(self, polls: int, withhold_signal: bool = False) -> None:
+        """Polls a bounded device wait makes before it gives up (0 = the default);
+        withhold_signal makes later calls withhold one producer signal (testing)."""
+        _check(tq4_ctx_set_wait_limit(self.handle, polls, int(withhold_signal)), "tq4_ctx_set_wait_limit")
+
     # -- pool helpers
     @staticmethod
     def new_pool(num_pages: int, device="cuda") -> torch.Tensor:
@@ -410,19 +440,50 @@ class Context:
                "tq4_decode_append_attention")
         return out
 
+    # -- the uniform INT8 comparison arm
+    @staticmethod
+    def new_int8_pool(num_pages: int, device="cuda") -> torch.Tensor:
+        return torch.zeros(num_pages * INT8_PAGE_BYTES, dtype=torch.uint8, device=device)
+
+    def int8_encode_append(self, pool, page_table, start_pos, k_new, v_new, stream=None):
+        _need_cuda(pool, page_table, k_new, v_new)
+        dtype = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(k_new.dtype)
+        if dtype is None or v_new.dtype != k_new.dtype:
+            raise ValueError("k_new/v_new must both be float32 or bfloat16")
+        _check(tq4_int8_encode_append(self.handle, pool, pool.numel() // INT8_PAGE_BYTES, page_table,
+                                      page_table.numel(), start_pos, k_new.shape[0], k_new, v_new, dtype, stream),
+               "tq4_int8_encode_append")
+
+    def int8_decode_attention(self, pool, q, page_tables, seq_lens, total_seq_len, scale, out=None,
+                              out_dtype=torch.bfloat16, workspace=None, stream=None):
+        _need_cuda(pool, q, page_tables, seq_lens)
+        if q.dtype != torch.bfloat16:
+            raise ValueError("q must be bfloat16")
+        n_req, n_q = q.shape[0], q.shape[1]
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        if workspace is None:
+            workspace = self.decode_workspace(n_req, n_q, total_seq_len, q.device)
+        _check(tq4_int8_decode_attention(self.handle, pool, pool.numel() // INT8_PAGE_BYTES, q, page_tables,
+                                         page_tables.shape[1], seq_lens, n_req, n_q, total_seq_len, scale, out,
+                                         od, workspace, workspace.numel(), stream), "tq4_int8_decode_attention")
+        return out
+
     def prefill_attention(self, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,
-                          workspace=None, stream=None):
-        """q: bf16 [n_tok, 24, 256]; k_chunk/v_chunk bf16 [n_tok, 4, 256]."""
+                          out_dtype=torch.bfloat16, workspace=None, stream=None):
+        """q: bf16 [n_tok, 24, 256]; k_chunk/v_chunk bf16 [n_tok, 4, 256]; out bf16 or float32."""
         _need_cuda(q, k_chunk, v_chunk)
         n_tok = q.shape[0]
         if out is None:
-            out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
         if workspace is None:
             workspace = torch.empty(max(tq4_prefill_workspace_bytes(n_tok), 256), dtype=torch.uint8,
                                     device=q.device)
         num_pages = pool.numel() // PAGE_BYTES if pool is not None else 0
         tlen = page_table.numel() if page_table is not None else 0
         _check(tq4_prefill_attention(self.handle, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk,
-                                     v_chunk, n_tok, scale, out, workspace, workspace.numel(), stream),
+                                     v_chunk, n_tok, scale, out, od, workspace, workspace.numel(), stream),
                "tq4_prefill_attention")
         return out

@@ -17,9 +17,14 @@
  *            on a 24 GB Mac", mechanism table, row KVExec: rotated-domain attention.
  *
  * Conventions fixed by this library where the pages are silent:
- *   codebook   16-level Lloyd-Max quantiser for N(0, 1/256) (computed by the
- *              library in fp64 at context creation); index j -> centroid c_j,
- *              ascending; nearest centroid, ties to the lower index.
+ *   codebook   16-level Lloyd-Max quantiser for N(0, 1/256), solved by the
+ *              library in fp64 at context creation; index j -> centroid c_j,
+ *              ascending; nearest centroid, ties to the lower index. Encode
+ *              compares against the fp64 midpoints rounded to fp32;
+ *              reconstruction reads the centroids rounded to fp32; the attention
+ *              kernels feed each centroid to f16 tensor-core products as the
+ *              pair c16 = f16(c_j), r16 = f16(c_j - c16), which carries c_j to
+ *              about 2^-21 relative.
  *   rotation   R = H diag(s) / 16, H the Sylvester Hadamard matrix, s the
  *              caller's +-1 sign diagonal. Encode quantises y = R x / ||x||;
  *              reconstruction is x_hat = fp16(||x||) * R^T c[idx].
@@ -81,6 +86,8 @@ extern "C" {
 #define TQ4_POSITION_BYTES  1040          /* one layer-position: 4 heads x (K+V) x 130 B */
 #define TQ4_PAGE_BYTES      266240        /* 256 layer-positions                         */
 #define TQ4_MAX_QUERY_TOKENS 4
+#define TQ4_INT8_POSITION_BYTES 2064      /* INT8 arm: 4 heads x (K+V) x (256 + 2) B    */
+#define TQ4_INT8_PAGE_BYTES     528384    /* INT8 arm: 256 layer-positions             */
 
 #define TQ4_DTYPE_F32   0
 #define TQ4_DTYPE_BF16  1
@@ -182,14 +189,37 @@ int tq4_decode_append_attention(tq4_ctx* ctx, void* pool, int32_t num_pages,
  *   q                 device bf16 [n_tok][24][256].
  *   k_chunk, v_chunk  device bf16 [n_tok][4][256].
  *   page_table        device int32[table_len] covering the prefix.
- *   out               device bf16 [n_tok][24][256].
- *   workspace         device scratch of tq4_prefill_workspace_bytes(n_tok) bytes. */
+ *   out               device [n_tok][24][256], out_dtype TQ4_DTYPE_BF16 or _F32.
+ *                     The fp32 output also runs the products that only an fp32
+ *                     result can resolve (about 1.5x the tensor work).
+ *   workspace         device scratch of tq4_prefill_workspace_bytes(n_tok) bytes,
+ *                     256-B aligned.
+ * Softmax and all accumulation are fp32. */
 size_t tq4_prefill_workspace_bytes(int32_t n_tok);
 int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                           const int32_t* page_table, int32_t table_len, int32_t prefix_len,
                           const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk,
-                          int32_t n_tok, float scale, uint16_t* out,
+                          int32_t n_tok, float scale, void* out, int out_dtype,
                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bounded device-side waits (a tile's copy, a tensor-core step, the fused
+ * append) give up after a number of polls, record TQ4_ERR_TIMEOUT in the status
+ * word and let the kernel finish without the rest of its work: it drains the
+ * copies and tensor-core operations it has issued, frees its tensor memory and
+ * returns, and the context stays usable. This call exists to test that path.
+ *   polls            polls before a wait gives up, for later calls on the
+ *                    context; 0 restores the default TQ4_DEFAULT_WAIT_POLLS.
+ *                    The drains before exit always use the default.
+ *   withhold_signal  nonzero: later calls withhold one producer signal so that
+ *                    a wait is sure to run out (the one-token decode kernel
+ *                    does not issue the copy of each warp's first tile; the
+ *                    prefill kernel does not signal the tensor-core issuer that
+ *                    P of tile min(1, tiles - 1) is ready); their results are
+ *                    then undefined and the status is TQ4_ERR_TIMEOUT. 0 (the
+ *                    default) restores normal operation.
+ * Returns TQ4_ERR_ARG for a NULL context. */
+#define TQ4_DEFAULT_WAIT_POLLS (1u << 24)
+int tq4_ctx_set_wait_limit(tq4_ctx* ctx, uint32_t polls, int withhold_signal);
 
 /* Decode attention for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for the library's users.
@@ -201,9 +231,12 @@ int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
  * results in a fixed array of TQ4_NOALLOC_SCRATCH_BYTES (8 MiB) that is part of
  * the library: every GPU that loads the library holds it until the process
  * exits. It allocates nothing and calls no allocating routine.
- *   - The first call on a device looks up the array's device address (the
- *     runtime call cudaGetSymbolAddress, under a lock) and caches it; make that
- *     first call on each device before any stream capture.
+ *   - tq4_ctx_create looks up the array's device address on the context's
+ *     device (the runtime call cudaGetSymbolAddress, with that device current)
+ *     and keeps it in the context, so this call does no set-up of its own. A
+ *     device reset (cudaDeviceReset, or any teardown of the device's primary
+ *     context) invalidates every context made before it, this address included:
+ *     create a new context afterwards.
  *   - Every call on a device shares the one array, so calls whose kernels may
  *     overlap on the GPU (different streams, no ordering between them) race
  *     and give wrong results; order them, e.g. issue them on one stream.
@@ -211,13 +244,42 @@ int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
  *     partial result it later reads.
  *   - A problem whose tq4_decode_workspace_bytes() exceeds
  *     TQ4_NOALLOC_SCRATCH_BYTES is rejected with TQ4_ERR_WORKSPACE before
- *     anything is launched (about 200 single-token requests at most). */
+ *     anything is launched. The workspace grows with the number of split-K
+ *     items (about one per SM / 4 KV heads for the whole batch, plus one per
+ *     request) times 8 (one query token) or 24 (two to four) query rows: on a
+ *     148-SM B200 the array holds 254 items with one query token (about 217
+ *     requests with long histories) and 84 items with four (about 47). */
 #define TQ4_NOALLOC_SCRATCH_BYTES (8u << 20)
 int tq4_decode_attention_noalloc(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                                  const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
                                  const int32_t* seq_lens, int32_t n_req, int32_t n_q,
                                  int64_t total_seq_len, float scale,
                                  void* out, int out_dtype, void* stream);
+
+/* The uniform INT8 comparison arm ([REASONING] simpleprog.com, "Fitting a
+ * 27B-Parameter LLM into 24 GiB of Laptop Memory", section "Reasoning at 200K":
+ * "a uniform INT8 comparison" arm runs next to TQ4; the page defines it no
+ * further). This library's reading: each 256-dim K or V head vector is stored as
+ * 256 int8 codes q_i = round-half-to-even(x_i / s), s = max_i |x_i| / 127, plus s
+ * as fp16 (the codes use the unrounded s; a zero vector stores s = 0); no rotation
+ * and no codebook; reconstruction is x_hat = fp16(s) * q. A pool of the INT8 arm is
+ * num_pages pages of TQ4_INT8_PAGE_BYTES bytes:
+ *   [0, 262144)       K codes  [4 heads][256 slots][256 int8]
+ *   [262144, 524288)  V codes  [4 heads][256 slots][256 int8]
+ *   [524288, 526336)  K scales [4 heads][256 slots] fp16
+ *   [526336, 528384)  V scales [4 heads][256 slots] fp16
+ * Page tables, lengths, queries, outputs, workspaces (tq4_decode_workspace_bytes)
+ * and errors are as for the TQ4 calls of the same shape. */
+int tq4_int8_encode_append(tq4_ctx* ctx, void* pool, int32_t num_pages,
+                           const int32_t* page_table, int32_t table_len,
+                           int32_t start_pos, int32_t n_tok,
+                           const void* k_new, const void* v_new, int dtype, void* stream);
+int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
+                              const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                              const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                              int64_t total_seq_len, float scale,
+                              void* out, int out_dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise the stream, return the first device-side error recorded since
  * the last call (TQ4_OK if none) and clear it. */

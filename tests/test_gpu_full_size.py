@@ -82,11 +82,20 @@ def test_prefill_full_size(codebook):
                                 _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE)
     torch.cuda.synchronize()
     assert ctx.status() == tq4.TQ4_OK
-    rows = np.unique(np.concatenate([[0, 1, 21, 22, 1023, w.n_q - 2, w.n_q - 1],
-                                     np.random.default_rng(7).choice(w.n_q, 9, replace=False)]))
+    out32 = ctx.prefill_attention(torch.from_numpy(pool).cuda(), torch.from_numpy(tab).cuda(), w.prefix_len,
+                                  _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE,
+                                  out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    # 64 chunk tokens: first and last, both sides of every 256-row CTA pair boundary, and a seeded draw
+    fixed = np.array([0, 1, 21, 22, 42, 43, 1023, w.n_q - 2, w.n_q - 1])
+    others = np.setdiff1d(np.arange(w.n_q), fixed)
+    rows = np.sort(np.concatenate([fixed, np.random.default_rng(7).choice(others, 64 - len(fixed), replace=False)]))
     exp = O.prefill_attention(pool, tab, w.prefix_len, I.bf16_bits_to_f32(qb), I.bf16_bits_to_f32(kb),
                               I.bf16_bits_to_f32(vb), SCALE, signs, c, rows=rows)
     H.assert_bf16_close(out.float().cpu().numpy()[rows], exp, "prefill 2048 on 32768")
+    err = np.abs(out32.cpu().numpy()[rows].astype(np.float64) - exp).max()
+    assert err <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), err
 
 
 def test_chunk_append_full_size(codebook):

@@ -184,6 +184,10 @@ def test_decode_variants_parity(seq_lens, n_q, shared):
     got = case.decode(q)
     exp = case.oracle_decode(q)
     H.assert_bf16_close(got, exp, f"decode {seq_lens} n_q={n_q}")
+    # the attention arithmetic in fp32 on the oracle's own pool bytes (5% x8 outliers)
+    got32 = case.decode_oracle_pool(q)
+    err = np.abs(got32 - exp).max()
+    assert err <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), err
 
 
 @pytest.mark.parametrize("n_q", [1, 4])
@@ -254,7 +258,7 @@ def test_decode_page_table_permutation_invariance():
 # 5% x8 outlier norms, whose large scores raise the softmax reference mid-walk
 @pytest.mark.parametrize("prefix_len,n_tok,outliers", [(300, 70, 0.0), (0, 5, 0.0), (512, 64, 0.0), (1, 1, 0.0),
                                                        (777, 130, 0.0), (1000, 200, 0.0), (600, 43, 0.05),
-                                                       (2048, 22, 0.05)])
+                                                       (2048, 22, 0.05), (1500, 90, 0.05), (64, 300, 0.0)])
 def test_prefill_parity(codebook, prefix_len, n_tok, outliers):
     c, _ = codebook
     signs = I.signs(4)
@@ -277,6 +281,13 @@ def test_prefill_parity(codebook, prefix_len, n_tok, outliers):
     exp = O.prefill_attention(opool, table, prefix_len, I.bf16_bits_to_f32(qb), I.bf16_bits_to_f32(kb),
                               I.bf16_bits_to_f32(vb), SCALE, signs, c)
     H.assert_bf16_close(out.float().cpu().numpy(), exp, f"prefill {prefix_len}+{n_tok} outliers {outliers}")
+    # fp32 output on the oracle's own pool bytes: the attention arithmetic alone, every row
+    out32 = ctx.prefill_attention(torch.from_numpy(opool).cuda(), tt, prefix_len, _bf16_tensor(qb), _bf16_tensor(kb),
+                                  _bf16_tensor(vb), SCALE, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    err = np.abs(out32.cpu().numpy().astype(np.float64) - exp).max()
+    assert err <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), (prefix_len, n_tok, outliers, err)
 
 
 # ------------------------------------------------------------------ failure paths (no GPU fault)

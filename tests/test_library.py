@@ -73,8 +73,8 @@ def test_status_strings():
 
 def test_workspace_sizes_are_host_arithmetic():
     assert tq4.tq4_prefill_workspace_bytes(0) == 0
-    # q' hi + lo ([n][24][256] f16 each) and the rotated chunk K, V ([n][4][256] f16 each)
-    assert tq4.tq4_prefill_workspace_bytes(2048) == 2048 * (2 * 24 + 2 * 4) * 256 * 2
+    # q' hi + lo ([n][24][256] f16 each) and the rotated chunk K, V as hi + lo ([n][4][256] f16 each)
+    assert tq4.tq4_prefill_workspace_bytes(2048) == 2048 * (2 * 24 + 4 * 4) * 256 * 2
     assert tq4.tq4_decode_workspace_bytes(None, 1, 1, 32768) == 0   # no context: no plan
 
 
@@ -87,7 +87,8 @@ def test_argument_errors_return_before_any_launch():
                                     None) == E
     assert lib.tq4_decode_append_attention(None, None, 0, None, None, 0, None, None, 0, None, 1, 1, 1, 0.0625,
                                            None, 1, None, 0, None) == E
-    assert lib.tq4_prefill_attention(None, None, 0, None, 0, 0, None, None, None, 1, 0.0625, None, None, 0,
+    assert lib.tq4_prefill_attention(None, None, 0, None, 0, 0, None, None, None, 1, 0.0625, None, 1, None, 0,
                                      None) == E
+    assert lib.tq4_ctx_set_wait_limit(None, 4, 0) == E
     assert lib.tq4_reconstruct(None, None, 0, None, 0, 0, 1, None, None, None) == E
     assert lib.tq4_get_status(None, None) == E

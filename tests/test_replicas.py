@@ -81,3 +81,44 @@ def test_reference_arm_prints_the_contract_line(capsys):
     assert cb["kind"] == "oracle" and cb["value"] == line["value"] and cb["cores"] >= 1 and cb["sample"]
     assert line["e2e"] == {"value": line["value"], "unit": bench.UNIT, "h2d_bytes_per_step": 0,
                            "d2h_bytes_per_step": 0}
+
+
+def _fake_measure(name, args, dist_, world, steps, headline):
+    """Stands in for the GPU measurement: rank r's step takes 2 + r ms."""
+    ms = bench.max_over_ranks(2.0 + dist_.get_rank(), dist_, torch.device("cpu"))
+    return {"value": bench.job_value(100, world, ms), "unit": bench.UNIT, "ms_per_step": ms, "steps": steps,
+            "gpu_launches": 2 * steps, "clocks": {"sm_mhz": None}, "roofline": None, "e2e": None,
+            "tokens_per_s": world / (ms * 1e-3), "graph": True}
+
+
+def _main_rank(rank, world, port, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world), RANK=str(rank),
+                      LOCAL_RANK=str(rank))
+    import contextlib
+    with open(os.path.join(out_dir, f"main{rank}.txt"), "w") as f, contextlib.redirect_stdout(f):
+        bench.main(["--gpus", str(world), "--steps", "3", "--warmup", "3", "--extra", "verify_2req_229k"],
+                   measure=_fake_measure)
+
+
+def test_bench_main_runs_two_ranks_end_to_end(tmp_path):
+    """bench.main()'s rank logic on two gloo ranks: process-group set-up, the same
+    measurements in the same order on every rank, max over ranks, one JSON line
+    from rank 0 (headline + extra workload), one clean teardown, exit 0."""
+    world = 2
+    mp.spawn(_main_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    out0 = (tmp_path / "main0.txt").read_text().splitlines()
+    out1 = (tmp_path / "main1.txt").read_text().splitlines()
+    assert out1 == []
+    assert len(out0) == 1
+    line = json.loads(out0[0])
+    assert line["n_gpus"] == 2 and line["ms_per_step"] == 3.0
+    assert line["value"] == pytest.approx(100 * 2 / 3e-3)
+    assert line["scaling"] == "weak" and line["config"]["parallelism"] == "replicas x2"
+    assert list(line["workloads"]) == ["verify_2req_229k"]
+    assert line["workloads"]["verify_2req_229k"]["ms_per_step"] == 3.0
+
+
+def test_bench_refuses_gpus_that_do_not_match_the_ranks(monkeypatch):
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    with pytest.raises(SystemExit):
+        bench.main(["--gpus", "8"], measure=_fake_measure)
