@@ -170,7 +170,7 @@ __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_
 __device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
-template <int NT, bool kI8, bool kExact>   // kExact: fp32 outputs, every product (see kVloNorm)
+template <int NT, bool kI8, bool kExact>   // kExact: fp32 outputs, C_lo P' on every chunk (see kVloNorm)
 __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kRB = kI8 ? 256 : 128;                 // bytes of one staged K or V row
@@ -488,13 +488,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       const int poff = (nt * 8 + jr) * kPsStride + 16 * w + 8 * mat;
       stmatrix_x2_trans(smem_u32(ps_hi + poff), *reinterpret_cast<const uint32_t*>(&h01),
                         *reinterpret_cast<const uint32_t*>(&h23));
-      if constexpr (kExact) {
-        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-        const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
-        const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
-        stmatrix_x2_trans(smem_u32(ps_lo + poff), *reinterpret_cast<const uint32_t*>(&l01),
-                          *reinterpret_cast<const uint32_t*>(&l23));
-      }
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
+      const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
+      stmatrix_x2_trans(smem_u32(ps_lo + poff), *reinterpret_cast<const uint32_t*>(&l01),
+                        *reinterpret_cast<const uint32_t*>(&l23));
     }
     // P' is complete; the chunk takes the C_lo P' products when one of its visible
     // V norms is large (or the output is fp32)
@@ -521,13 +519,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
         const uint2 x1 = lds64(vst + (pb + 1) * 256 + ((seg ^ i8_swz(pb + 1)) << 4) + off8);
         const uint2 y0 = lds64(vst + (pb + 8) * 256 + ((seg ^ i8_swz(pb + 8)) << 4) + off8);
         const uint2 y1 = lds64(vst + (pb + 9) * 256 + ((seg ^ i8_swz(pb + 9)) << 4) + off8);
-        uint32_t bh[NT][2], bl[NT][2] = {};
+        uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           const int m = (lane >> 3) & 1;
           const int off = (nt * 8 + (lane & 7)) * kPsStride + 64 * ph + 16 * ks + 8 * m;
           ldmatrix_x2(bh[nt][0], bh[nt][1], smem_u32(ps_hi + off));
-          if constexpr (kExact) ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
+          ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
         }
 #pragma unroll
         for (int mt = 0; mt < 4; ++mt) {
@@ -540,7 +538,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
             mma_16816(o[nt][mt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-            if constexpr (kExact) mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+            mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
           }
         }
       }
@@ -561,13 +559,13 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       uint32_t lo01, hi01, lo89, hi89;
       interleave_nibbles(x0, x1, lo01, hi01);
       interleave_nibbles(y0, y1, lo89, hi89);
-      uint32_t bh[NT][2], bl[NT][2] = {};
+      uint32_t bh[NT][2], bl[NT][2];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const int m = (lane >> 3) & 1;
         const int off = (nt * 8 + (lane & 7)) * kPsStride + 64 * ph + 16 * ks + 8 * m;
         ldmatrix_x2(bh[nt][0], bh[nt][1], smem_u32(ps_hi + off));
-        if constexpr (kExact) ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
+        ldmatrix_x2(bl[nt][0], bl[nt][1], smem_u32(ps_lo + off));
       }
 #pragma unroll
       for (int mt = 0; mt < 4; ++mt) {
@@ -591,11 +589,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
             break;
         }
         // O'^T += (C_hi + C_lo)^T (P'_hi + P'_lo), less the C_lo P'_lo term (and, with bf16
-        // outputs, less P'_lo, and less C_lo where the chunk's V norms are all small)
+        // outputs, less C_lo where the chunk's V norms are all small)
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
           mma_16816(o[nt][mt], a0, a1, a2, a3, bh[nt][0], bh[nt][1]);
-          if constexpr (kExact) mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
+          mma_16816(o[nt][mt], a0, a1, a2, a3, bl[nt][0], bl[nt][1]);
           if constexpr (kLo) mma_16816(o[nt][mt], r0, r1, r2, r3, bh[nt][0], bh[nt][1]);
         }
       }

@@ -130,7 +130,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // K words (4 heads x 256 slots), V words, then 32 rows of norms.
 constexpr int kRowsPerPage = int(kPageBytes / 128);   // 2,080
 
-template <bool kExact>   // fp32 outputs: every product (see kVloNorm)
+template <bool kExact>   // fp32 outputs: C_lo P' on every tile (see kVloNorm)
 __global__ void __launch_bounds__(kQ1Threads, 1)
     decode_q1_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     }
     const float mu0 = m_ref[0] == -INFINITY ? 0.f : m_ref[0];
     const float mu1 = m_ref[1] == -INFINITY ? 0.f : m_ref[1];
-    uint32_t bh[2][2], bl[2][2] = {{0u, 0u}, {0u, 0u}};
+    uint32_t bh[2][2], bl[2][2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       float pw[4];
@@ -449,20 +449,18 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       const float w2 = s[j][2] == -INFINITY ? 0.f : pw[2] * vn[j][1];
       const float w3 = s[j][3] == -INFINITY ? 0.f : pw[3] * vn[j][1];
       const __half2 h01 = __floats2half2_rn(w0, w1), h23 = __floats2half2_rn(w2, w3);
+      const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+      const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
+      const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
       bh[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h01));
       bh[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&h23));
-      if constexpr (kExact) {
-        const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
-        const __half2 l01 = __floats2half2_rn(w0 - f01.x, w1 - f01.y);
-        const __half2 l23 = __floats2half2_rn(w2 - f23.x, w3 - f23.y);
-        bl[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l01));
-        bl[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l23));
-      }
+      bl[j][0] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l01));
+      bl[j][1] = movmatrix_trans(*reinterpret_cast<const uint32_t*>(&l23));
     }
 
     // ------------------------------------------------------------ V phase (all 256 dims), two k-steps
     // O'^T += (C_hi + C_lo)^T (P'_hi + P'_lo) less C_lo P'_lo; with bf16 outputs
-    // without P'_lo, and without C_lo on tiles whose V norms are all small (kVloNorm)
+    // without C_lo on tiles whose V norms are all small (kVloNorm)
     auto v_phase = [&](auto lo_tag) {
     constexpr bool kLo = decltype(lo_tag)::value;
 #pragma unroll
@@ -499,7 +497,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
               break;
           }
           mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bh[j][0], bh[j][1]);
-          if constexpr (kExact) mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bl[j][0], bl[j][1]);
+          mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bl[j][0], bl[j][1]);
           if constexpr (kLo) mma_16816(o[4 * q + kb_], r0, r1, r2, r3, bh[j][0], bh[j][1]);
         }
       }

@@ -14,9 +14,9 @@
 // Precision. Every tensor-core operand is an f16 hi + lo pair: q' = q'hi + q'lo,
 // a centroid c = c16 + r16 (c16 = f16(c), r16 = f16(c - c16)), chunk rows
 // likewise, P = Phi + Plo. The scores take the three terms that matter
-// (q'hi Khi + q'lo Khi + q'hi Klo); O takes Phi Vhi, plus Phi Vlo on tiles whose
-// largest V norm exceeds kVloNorm, plus Plo Vhi and Phi Vlo on every tile when
-// the output is fp32 (the fp32 check holds the result to ~1e-5 relative).
+// (q'hi Khi + q'lo Khi + q'hi Klo); O takes Phi Vhi + Plo Vhi, plus Phi Vlo on
+// tiles whose largest V norm exceeds kVloNorm and on every tile when the output is
+// fp32 (the fp32 check holds the result to ~1e-5 relative).
 //
 // Work split. A cluster of two CTAs (ranks 0 and 1) owns 256 query rows
 // (row = token * 6 + head within the KV head's group; rank r holds rows
@@ -29,7 +29,7 @@
 //               its q' hi row into TMEM and its q' lo row into shared memory.
 //               Reads its score row from TMEM, applies K norms, the causal mask
 //               and an online softmax with a lazily raised reference; writes
-//               P = p * n_v / 256 over S (f16 hi, and lo for fp32 outputs).
+//               P = p * n_v / 256 over S (f16 hi and lo).
 //   warps 4-11  dequant, two groups of four; group g fills stage g for tiles
 //               g, g+2, ...: packed words are prefetched into registers two
 //               tiles ahead and expanded through a per-lane table of 8-byte
@@ -378,19 +378,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
         m_ref = mx;
         l_sum *= alpha;
       }
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {   // warp-wide; lanes that keep their reference use alpha = 1
-        if (!warp_wait(bar(kBOReady), (j - 1) & 1)) break;   // PV(j-1) has completed
-        tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t ov[32];
-          tm_ld32(lane_addr + kTmO + 32 * c, ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tm_st32(lane_addr + kTmO + 32 * c, ov);
-        }
-        tm_wait_st();
-      }
       const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
       float l4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -405,24 +392,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
         }
       }
       l_sum += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-      // P hi (columns 0-31: positions 2k, 2k+1 in column k) and, for fp32 outputs,
-      // P lo = P - f16(P) (columns 32-63), written over the scores in halves of 32 positions
+      // P hi (columns 0-31: positions 2k, 2k+1 in column k) and P lo = P - f16(P)
+      // (columns 32-63), written over the scores in halves of 32 positions
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]), __uint_as_float(sr[c][2 * k + 1]));
         tm_st16(lane_addr + kTmS0 + 64 * b + 16 * c, pk);
-        if (exact) {
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
-            pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]) - hi.x, __uint_as_float(sr[c][2 * k + 1]) - hi.y);
-          }
-          tm_st16(lane_addr + kTmS0 + 64 * b + 32 + 16 * c, pk);
+        for (int k = 0; k < 16; ++k) {
+          const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&pk[k]));
+          pk[k] = pack_half2(__uint_as_float(sr[c][2 * k]) - hi.x, __uint_as_float(sr[c][2 * k + 1]) - hi.y);
         }
+        tm_st16(lane_addr + kTmS0 + 64 * b + 32 + 16 * c, pk);
       }
       tm_wait_st();
+      // PV(j - 1) has completed. Waited for at every tile, not only when O is rescaled:
+      // the barrier then never trails this warp by more than one phase, so its parity
+      // names one phase only (the final wait below relies on the same).
+      if (j > 0) {
+        if (!warp_wait(bar(kBOReady), (j - 1) & 1)) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, raise)) {   // lanes that keep their reference use alpha = 1
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t ov[32];
+            tm_ld32(lane_addr + kTmO + 32 * c, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tm_st32(lane_addr + kTmO + 32 * c, ov);
+          }
+          tm_wait_st();
+        }
+      }
       tc_fence_before();
       // (test hook: tile min(1, n_tiles - 1)'s P signal is withheld, so the issuer's
       // wait for it runs out after some MMAs of the pair have been issued)
@@ -656,7 +659,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
           for (int ks = 0; ks < kPfTile / 16; ++ks) {
             const uint64_t bh = tc_sdesc(vb + kPfVHi + ks * 16 * 128, kPfVPanel, 1024);
             tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, bh, idesc_pv, (jb > 0 || ks > 0) ? 1u : 0u);
-            if (exact) tc2_mma_ts(tmem + kTmO, p_t + 32 + 8 * ks, bh, idesc_pv, 1u);
+            tc2_mma_ts(tmem + kTmO, p_t + 32 + 8 * ks, bh, idesc_pv, 1u);
             if (vlo) {
               const uint64_t bl = tc_sdesc(vb + kPfVLo + ks * 16 * 128, kPfVPanel, 1024);
               tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, bl, idesc_pv, 1u);

@@ -30,9 +30,9 @@ def assert_bf16_close(got, expect, what=""):
     expect = np.asarray(expect, np.float64)
     err = np.abs(got - expect)
     tol = bf16_tolerance(expect)
-    bad = err > tol
+    bad = ~(err <= tol)   # a NaN or Inf anywhere fails too
     if bad.any():
-        i = np.unravel_index(np.argmax(err - tol), err.shape)
+        i = np.unravel_index(np.argmax(np.where(np.isfinite(err), err - tol, np.inf)), err.shape)
         raise AssertionError(f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst at {i}: "
                              f"got {got[i]} expect {expect[i]} (tol {tol[i]})")
     return float(err.max())
