@@ -7,7 +7,10 @@
 // each other inside the main loop:
 //
 //   * a CTA (8 warps) owns one (request, KV head, split); warp w takes the
-//     32-position tiles w, w+8, w+16, ... of the split;
+//     32-position tiles w, w+8, w+16, ... of the split's full rounds of 256
+//     positions; a last round of at most 128 positions is dealt out as 16-position
+//     half tiles (one per warp), so every warp of a split of 256 r + 128 positions
+//     does the same work;
 //   * lane 0 of each warp streams its tiles with TMA (2D tensor loads of the
 //     K and V word rows with the 128-byte swizzle, bulk copies of the two norm
 //     rows) into a private two-stage ring, completion on an mbarrier;
@@ -39,11 +42,14 @@ constexpr int kQ1Stages = 2;                   // TMA ring depth per warp
 constexpr int kQ1KV = kQ1Tile * 128;           // 4,096 B: one K (or V) tile, 128-B swizzled rows
 constexpr int kQ1Buf = 2 * kQ1KV;              // K then V
 constexpr int kQ1Bufs = kQ1Warps * kQ1Stages;  // 16 tile buffers
-constexpr uint32_t kQ1TxBytes = 2 * kQ1KV + 2 * kQ1Tile * 2;   // words + both norm rows
 // Shared-window layout (absolute 32-bit shared addresses). The centroid table
 // sits at 0x10000 so that one byte permute builds a lookup address
-// (0x10000 | byte << 8 | lane * 4). Below it: control words, q', mbarriers,
-// norm rows and the first tile buffers; above it: the other tile buffers.
+// (0x10000 | byte << 8 | lane * 4). Row `byte` (256 B) holds 32 copies of the
+// byte's c16 pair, then 32 copies of its r16 pair: each lane reads its own copy,
+// so a warp's 4-byte loads of either half hit 32 different banks, and a lookup
+// that needs only the c16 pair costs one wavefront. Below the table: control
+// words, q', mbarriers, norm rows and the first tile buffers; above it: the other
+// tile buffers.
 constexpr uint32_t kQ1Lut = 0x10000;
 constexpr uint32_t kQ1Hi = 0x20000;
 constexpr uint32_t kQ1QvOff = 128;
@@ -90,12 +96,39 @@ __device__ __forceinline__ uint16_t ld_shared_u16(uint32_t a) {
 __device__ __forceinline__ void st_shared_u32(uint32_t a, uint32_t v) {
   asm volatile("st.shared.b32 [%0], %1;\n" ::"r"(a), "r"(v) : "memory");
 }
-// byte K of w -> the hi and lo f16x2 centroid pairs from the table at kQ1Lut
-// (lanebase = kQ1Lut | 8 * lane: one byte permute forms the slot address)
+// byte K of w -> the hi (c16) and lo (r16) f16x2 centroid pairs from the table at
+// kQ1Lut (lanebase = kQ1Lut | 4 * lane: one byte permute forms the address)
+template <int K>
+__device__ __forceinline__ uint32_t lut_addr(uint32_t w, uint32_t lanebase) {
+  constexpr uint32_t sel = (7u << 12) | (6u << 8) | (uint32_t(K) << 4) | 4u;
+  return __byte_perm(w, lanebase, sel);
+}
 template <int K>
 __device__ __forceinline__ void lut64k(uint32_t w, uint32_t lanebase, uint32_t& hi, uint32_t& lo) {
-  constexpr uint32_t sel = (7u << 12) | (6u << 8) | (uint32_t(K) << 4) | 4u;
-  ld_shared_v2(__byte_perm(w, lanebase, sel), hi, lo);
+  const uint32_t a = lut_addr<K>(w, lanebase);
+  hi = ld_shared_u32(a);
+  lo = ld_shared_u32(a + 128);
+}
+template <int K>
+__device__ __forceinline__ uint32_t lut64k_hi(uint32_t w, uint32_t lanebase) {
+  return ld_shared_u32(lut_addr<K>(w, lanebase));
+}
+// byte K of four words -> four A-fragment registers (hi), and their lo pairs when kLo
+template <int K, bool kLo>
+__device__ __forceinline__ void lut4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t lanebase,
+                                     uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3, uint32_t& r0,
+                                     uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  if constexpr (kLo) {
+    lut64k<K>(w0, lanebase, a0, r0);
+    lut64k<K>(w1, lanebase, a1, r1);
+    lut64k<K>(w2, lanebase, a2, r2);
+    lut64k<K>(w3, lanebase, a3, r3);
+  } else {
+    a0 = lut64k_hi<K>(w0, lanebase);
+    a1 = lut64k_hi<K>(w1, lanebase);
+    a2 = lut64k_hi<K>(w2, lanebase);
+    a3 = lut64k_hi<K>(w3, lanebase);
+  }
 }
 
 // ---- mbarrier and bulk-copy primitives (one CTA = its own cluster; no multicast)
@@ -147,17 +180,19 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   __half* qv_hi = reinterpret_cast<__half*>(smem + kQ1QvOff);
   __half* qv_lo = qv_hi + 8 * kQvStride;
   auto buf_addr = [&](int b) { return b < kQ1LowBufs ? low0 + b * kQ1Buf : kQ1Hi + (b - kQ1LowBufs) * kQ1Buf; };
-  const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 8u);
+  const uint32_t lanebase = kQ1Lut | (uint32_t(lane) * 4u);
 
   // prologue that reads none of the call's inputs (overlaps the previous kernel)
   const uint32_t bar_new = base + 8;   // the fused append's new position is in the pool (count 2)
   if (tid < kQ1Bufs) mbar_init(base + kQ1BarOff + tid * 8, 1);
   if (tid == kQ1Bufs) mbar_init(bar_new, 2);
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-  // table rows: every lane's 8-byte slot of row b holds {c16 pair, r16 pair}
-  for (int b = w; b < 256; b += kQ1Warps) {
-    const uint2 v = lut_row(b);
-    asm volatile("st.shared.v2.b32 [%0], {%1,%2};\n" ::"r"(kQ1Lut + b * 256 + lane * 8), "r"(v.x), "r"(v.y) : "memory");
+  // table rows: 32 copies of the c16 pair, then 32 copies of the r16 pair (16-B stores of 4 copies)
+  for (int e = tid; e < 256 * 16; e += kQ1Threads) {
+    const uint2 v = lut_row(e >> 4);
+    const uint32_t x = (e & 8) ? v.y : v.x;
+    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};\n" ::"r"(kQ1Lut + (e >> 4) * 256 + (e & 15) * 16), "r"(x)
+                 : "memory");
   }
   __syncthreads();   // barriers initialised before any warp arms one
   pdl_wait();
@@ -174,6 +209,11 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         s_item[1] = sp;
         if (blockIdx.x == 0 && h == 0 && total > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
       }
+      if (blockIdx.x == 0 && h == 0) {   // a length the page table cannot hold: no output for that request
+        bool bad = false;
+        for (int rr = lane; rr < p.n_req; rr += 32) bad |= !seq_ok(__ldg(p.seq_lens + rr), p.n_q, p.max_pages);
+        if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(p.status, TQ4_ERR_SEQ);
+      }
     }
     __syncthreads();
     r = s_item[0];
@@ -183,21 +223,31 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
   const int pos_b = split * p.split_len;
   // independent loads go out together: the length, this warp's first page id
-  // (speculative, inside the table) and this warp's query row
+  // (speculative, inside the table: its first tile starts at 32 w, or at 16 w when
+  // the split is a single half round) and this warp's query row
   const int seq_len = __ldg(p.seq_lens + r);
-  const int c_first = pos_b + w * kQ1Tile;
-  const int32_t page_first = (c_first >> 8) < p.max_pages ? __ldg(table + (c_first >> 8)) : -1;
+  const int c_full = pos_b + w * kQ1Tile, c_half = pos_b + w * (kQ1Tile / 2);
+  const int32_t page_full = (c_full >> 8) < p.max_pages ? __ldg(table + (c_full >> 8)) : -1;
+  const int32_t page_half = (c_half >> 8) < p.max_pages ? __ldg(table + (c_half >> 8)) : -1;
   uint4 qraw = make_uint4(0, 0, 0, 0);
   if (w < kGroup)
     qraw = __ldg(reinterpret_cast<const uint4*>(p.q + (int64_t(r) * kHq + h * kGroup + w) * kD + lane * 8));
   if (p.n_req == 1) {
-    const int S = seq_ok(seq_len, p.n_q, p.max_pages) ? (seq_len + p.split_len - 1) / p.split_len : 0;
-    if (tid == 0 && blockIdx.x == 0 && h == 0 && S > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
+    const bool len_ok = seq_ok(seq_len, p.n_q, p.max_pages);
+    const int S = len_ok ? (seq_len + p.split_len - 1) / p.split_len : 0;
+    if (tid == 0 && blockIdx.x == 0 && h == 0 && (!len_ok || S > p.items_ub)) record_error(p.status, TQ4_ERR_SEQ);
     if (split >= S || split >= p.items_ub) return;   // the same decision in every thread of the CTA
   }
   const int pos_e = min(pos_b + p.split_len, seq_len);
-  const int n_tiles = (pos_e - pos_b + kQ1Tile - 1) / kQ1Tile;
-  const int my_tiles = n_tiles > w ? (n_tiles - w + kQ1Warps - 1) / kQ1Warps : 0;
+  // Tiles: full rounds of 8 x 32 positions (warp w takes the w-th tile of each), then
+  // the remainder: at most 128 positions as eight 16-position half tiles, else as
+  // eight 32-position tiles (masked past pos_e).
+  const int n_pos = pos_e - pos_b;
+  const int rounds = n_pos >> 8, rem = n_pos & 255;
+  const bool half_round = rem > 0 && rem <= 128;
+  const int chunk = half_round ? kQ1Tile / 2 : kQ1Tile;
+  const int my_tiles = rounds + ((rem > 0 && chunk * w < rem) ? 1 : 0);
+  const int32_t page_first = (rounds == 0 && half_round) ? page_half : page_full;
   // fused append: this CTA holds the request's last position (seq_len - 1)
   const bool append_here = p.pool_w != nullptr && pos_e == seq_len && pos_b < pos_e;
   // warp 6: K, warp 7: V of KV head h. The input row is loaded early (fused_load);
@@ -220,17 +270,22 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive_q1(bar_new);
   };
-  const int last_w = (n_tiles - 1) % kQ1Warps, last_k = (n_tiles - 1) / kQ1Warps;
+  const int p_last = n_pos - 1;   // split-relative position of the last one
+  const int last_w = p_last < rounds * 256 ? (p_last >> 5) & (kQ1Warps - 1) : (p_last - rounds * 256) / chunk;
+  const int last_k = p_last < rounds * 256 ? (p_last >> 8) : rounds;
   const bool encoder = append_here && w >= kQ1Warps - 2;
   // When the tile with the new position is its owner's first tile, its TMA is issued
   // before the block-wide barrier below, so the encode must precede that barrier;
   // otherwise it follows it and delays no warp.
   const bool encode_first = encoder && last_k == 0;
 
-  // ---- lane 0 of each warp streams the warp's tiles: tile w + 8k -> buffer w*2 + k%2
-  auto tile_pos = [&](int k) { return pos_b + (w + k * kQ1Warps) * kQ1Tile; };
+  // ---- lane 0 of each warp streams the warp's tiles: tile k -> buffer w*2 + k%2
+  auto tile_pos = [&](int k) {
+    return pos_b + (k < rounds ? (w + k * kQ1Warps) * kQ1Tile : rounds * 256 + chunk * w);
+  };
+  auto tile_half = [&](int k) { return half_round && k == rounds; };
   // page id of tile k of this warp, loaded one iteration before its copy is issued
-  // (a warp's consecutive tiles are one page apart); -1 past the table
+  // (a tile never straddles a page); -1 past the table
   auto tile_page = [&](int k) -> int32_t {
     const int c = tile_pos(k);
     return (k < my_tiles && (c >> 8) < p.max_pages) ? __ldg(table + (c >> 8)) : -1;
@@ -255,11 +310,15 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       const int row = page * kRowsPerPage + slot0;
       const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
       const uint32_t kdst = buf_addr(b), ndst = base + kQ1NrmOff + b * 128;
-      mbar_expect_tx(bar, kQ1TxBytes);
+      // A half tile still takes 32-row word boxes (the extra rows stay inside the
+      // page: at most row 2,063 of its 2,080) but only its own 16 norms, since the
+      // V norms end the page.
+      const uint32_t nbytes = tile_half(k) ? kQ1Tile : 2 * kQ1Tile;
+      mbar_expect_tx(bar, 2 * kQ1KV + 2 * nbytes);
       tma_load_2d(kdst, &tmap, 0, row, bar);                       // K words of 32 positions
       tma_load_2d(kdst + kQ1KV, &tmap, 0, row + 4 * kPage, bar);   // V words
-      bulk_load(ndst, pg + kKNorms + slot0 * 2, kQ1Tile * 2, bar);
-      bulk_load(ndst + 64, pg + kVNorms + slot0 * 2, kQ1Tile * 2, bar);
+      bulk_load(ndst, pg + kKNorms + slot0 * 2, nbytes, bar);
+      bulk_load(ndst + 64, pg + kVNorms + slot0 * 2, nbytes, bar);
     }
   };
   if (encoder) fused_load();
@@ -345,20 +404,27 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     const uint32_t kst = buf_addr(b), vst = kst + kQ1KV;
     const uint32_t nb = base + kQ1NrmOff + b * 128;
     const int c = tile_pos(k);
+    const bool two = !tile_half(k);   // warp-uniform: m-tile 1 exists (a half tile has m-tile 0 only)
 
     // ------------------------------------------------------------ K phase, two m-tiles
     uint4 ka[2], kb4[2], kc[2], kd[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
+      if (j == 1 && !two) {
+        ka[1] = kb4[1] = kc[1] = kd[1] = make_uint4(0, 0, 0, 0);
+        break;
+      }
       const uint32_t mrow = kst + j * 16 * 128;
       ka[j] = ld_shared_v4(mrow + k_off0);
       kb4[j] = ld_shared_v4(mrow + k_off1);
       kc[j] = ld_shared_v4(mrow + 8 * 128 + k_off0);
       kd[j] = ld_shared_v4(mrow + 8 * 128 + k_off1);
     }
-    // S = (C_hi + C_lo)(q'_hi + q'_lo): sc = C_hi q'_hi, sd = C_hi q'_lo + C_lo q'_hi
+    // S = (C_hi + C_lo)(q'_hi + q'_lo) less C_lo q'_lo: sc = C_hi q'_hi, sd = C_hi q'_lo,
+    // se = C_lo q'_hi (three accumulators: three independent chains of 16 MMAs)
     float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     float sd[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float se[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     uint32_t ql4[4];
 #pragma unroll
     for (int kk = 0; kk < 16; ++kk) {
@@ -366,6 +432,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       const uint32_t ql0 = ql4[2 * (kk & 1)], ql1 = ql4[2 * (kk & 1) + 1];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
+        if (j == 1 && !two) break;
         const uint32_t wg = pick(ka[j], kb4[j], kk >> 1);
         const uint32_t wg8 = pick(kc[j], kd[j], kk >> 1);
         uint32_t a0, a1, a2, a3, r0, r1, r2, r3;
@@ -378,7 +445,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         }
         mma_16816(sc[j], a0, a1, a2, a3, qh[kk][0], qh[kk][1]);
         mma_16816(sd[j], a0, a1, a2, a3, ql0, ql1);
-        mma_16816(sd[j], r0, r1, r2, r3, qh[kk][0], qh[kk][1]);
+        mma_16816(se[j], r0, r1, r2, r3, qh[kk][0], qh[kk][1]);
       }
     }
 
@@ -392,10 +459,10 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         const int pos = 16 * j + pk + 8 * e;
         kn[j][e] = __half2float(__ushort_as_half(ld_shared_u16(nb + 2 * pos)));
         vn[j][e] = __half2float(__ushort_as_half(ld_shared_u16(nb + 64 + 2 * pos))) * kQ1PScale;
-        const bool ok = c + pos < pos_e;
+        const bool ok = (j == 0 || two) && c + pos < pos_e;
         vbig |= ok && vn[j][e] > kVloNorm * kQ1PScale;
-        s[j][2 * e] = (ok && row_ok0) ? (sc[j][2 * e] + sd[j][2 * e]) * kn[j][e] * kLog2e : -INFINITY;
-        s[j][2 * e + 1] = (ok && row_ok1) ? (sc[j][2 * e + 1] + sd[j][2 * e + 1]) * kn[j][e] * kLog2e : -INFINITY;
+        s[j][2 * e] = (ok && row_ok0) ? (sc[j][2 * e] + (sd[j][2 * e] + se[j][2 * e])) * kn[j][e] * kLog2e : -INFINITY;
+        s[j][2 * e + 1] = (ok && row_ok1) ? (sc[j][2 * e + 1] + (sd[j][2 * e + 1] + se[j][2 * e + 1])) * kn[j][e] * kLog2e : -INFINITY;
       }
     // Lazy reference: a row's reference is raised only when the row max exceeds it by
     // more than 2^8. Each lane first tests its own scores; the row maxima (shuffles)
@@ -460,11 +527,13 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
 
     // ------------------------------------------------------------ V phase (all 256 dims), two k-steps
     // O'^T += (C_hi + C_lo)^T (P'_hi + P'_lo) less C_lo P'_lo; with bf16 outputs
-    // without C_lo on tiles whose V norms are all small (kVloNorm)
+    // without C_lo on tiles whose V norms are all small (kVloNorm), where only the
+    // c16 halves of the table are read
     auto v_phase = [&](auto lo_tag) {
     constexpr bool kLo = decltype(lo_tag)::value;
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
+      if (j == 1 && !two) break;   // a half tile's positions 16-31 carry P' = 0
       const uint32_t vrow = vst + j * 16 * 128;
       const uint4 x0 = ld_shared_v4(vrow + v_off0);              // position sigma(2t)
       const uint4 x1 = ld_shared_v4(vrow + v_off1);              // position sigma(2t+1)
@@ -477,24 +546,12 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         interleave_nibbles(pick(y0, y0, q), pick(y1, y1, q), lo89, hi89);
 #pragma unroll
         for (int kb_ = 0; kb_ < 4; ++kb_) {
-          uint32_t a0, a1, a2, a3, r0, r1, r2, r3;
+          uint32_t a0, a1, a2, a3, r0 = 0, r1 = 0, r2 = 0, r3 = 0;
           switch (kb_) {
-            case 0:
-              lut64k<0>(lo01, lanebase, a0, r0); lut64k<0>(hi01, lanebase, a1, r1);
-              lut64k<0>(lo89, lanebase, a2, r2); lut64k<0>(hi89, lanebase, a3, r3);
-              break;
-            case 1:
-              lut64k<1>(lo01, lanebase, a0, r0); lut64k<1>(hi01, lanebase, a1, r1);
-              lut64k<1>(lo89, lanebase, a2, r2); lut64k<1>(hi89, lanebase, a3, r3);
-              break;
-            case 2:
-              lut64k<2>(lo01, lanebase, a0, r0); lut64k<2>(hi01, lanebase, a1, r1);
-              lut64k<2>(lo89, lanebase, a2, r2); lut64k<2>(hi89, lanebase, a3, r3);
-              break;
-            default:
-              lut64k<3>(lo01, lanebase, a0, r0); lut64k<3>(hi01, lanebase, a1, r1);
-              lut64k<3>(lo89, lanebase, a2, r2); lut64k<3>(hi89, lanebase, a3, r3);
-              break;
+            case 0: lut4<0, kLo>(lo01, hi01, lo89, hi89, lanebase, a0, a1, a2, a3, r0, r1, r2, r3); break;
+            case 1: lut4<1, kLo>(lo01, hi01, lo89, hi89, lanebase, a0, a1, a2, a3, r0, r1, r2, r3); break;
+            case 2: lut4<2, kLo>(lo01, hi01, lo89, hi89, lanebase, a0, a1, a2, a3, r0, r1, r2, r3); break;
+            default: lut4<3, kLo>(lo01, hi01, lo89, hi89, lanebase, a0, a1, a2, a3, r0, r1, r2, r3); break;
           }
           mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bh[j][0], bh[j][1]);
           mma_16816(o[4 * q + kb_], a0, a1, a2, a3, bl[j][0], bl[j][1]);

@@ -140,12 +140,11 @@ __device__ __forceinline__ uint2 lut_row(int b) {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// With bf16 outputs the attention kernels skip the products that a bf16 result
-// cannot resolve: P' lo (the f16 rounding of the softmax weights) always, and the
-// centroid residual of the V side (C_lo P') on tiles whose V norms all stay at or
-// below kVloNorm. The keys always take all three score terms. Norms 16 s with s in
-// [0.5, 2] stay under ~34; the 8x outliers of the long-context workload start at
-// 64. fp32 outputs run every product.
+// With bf16 outputs the attention kernels skip the one product that a bf16 result
+// cannot resolve: the centroid residual of the V side (C_lo P') on tiles whose V
+// norms all stay at or below kVloNorm. The keys always take all three score terms
+// and P' lo always enters. Norms 16 s with s in [0.5, 2] stay under ~34; the 8x
+// outliers of the long-context workload start at 64. fp32 outputs run every product.
 constexpr float kVloNorm = 48.0f;
 
 // 16-byte global -> shared copies that bypass registers (generic proxy; wait before use)

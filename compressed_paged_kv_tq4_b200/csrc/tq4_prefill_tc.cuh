@@ -85,9 +85,11 @@ constexpr uint32_t kTmQ = 0, kTmS0 = 128, kTmO = 256;
 
 // barriers (8 B each at kPfBarOff): in rank 0, counted from both CTAs
 constexpr int kBQReady = 0, kBKFull = 1, kBVFull = 3, kBPFull = 5;
-// in each CTA: committed by the issuer to both CTAs, or local
-constexpr int kBSFull = 7, kBKEmpty = 9, kBVEmpty = 11, kBOReady = 13, kBDrain = 14, kBNFull = 15;
-constexpr int kBarriers = 17;
+// in each CTA: committed by the issuer to both CTAs, or local. S_FULL(b) completes when
+// QK of a stage-b tile is done (its scores are in TMEM, its K half is free); V_EMPTY(b)
+// when PV of a stage-b tile is done (its V half is free, O holds it).
+constexpr int kBSFull = 7, kBVEmpty = 9, kBDrain = 11, kBNFull = 12;
+constexpr int kBarriers = 14;
 static_assert(kBarriers * 8 <= 256, "barrier area");
 
 // ---- descriptors (layouts of the PTX ISA's tcgen05 matrix descriptors)
@@ -167,6 +169,17 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
       : "memory");
   return done != 0;
 }
+// one non-blocking look at the phase (acquire, cluster scope)
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
 __device__ __forceinline__ void st_cluster_u32(uint32_t cluster_addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(cluster_addr), "r"(v) : "memory");
 }
@@ -236,11 +249,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       mbar_init(bar(kBVFull + b), 2 * (kPfGroupThreads / 32));
       mbar_init(bar(kBPFull + b), 2 * kPfSoftWarps);
       mbar_init(bar(kBSFull + b), 1);
-      mbar_init(bar(kBKEmpty + b), 1);
       mbar_init(bar(kBVEmpty + b), 1);
       mbar_init(bar(kBNFull + b), kPfGroupThreads / 32);
     }
-    mbar_init(bar(kBOReady), 1);
     mbar_init(bar(kBDrain), 1);
     misc[1] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -408,11 +419,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
         tm_st16(lane_addr + kTmS0 + 64 * b + 32 + 16 * c, pk);
       }
       tm_wait_st();
-      // PV(j - 1) has completed. Waited for at every tile, not only when O is rescaled:
-      // the barrier then never trails this warp by more than one phase, so its parity
-      // names one phase only (the final wait below relies on the same).
+      // PV(j - 1) has completed (V_EMPTY of its stage). Waited for at every tile, not
+      // only when O is rescaled: each stage's barrier is then waited for every other
+      // tile and never trails this warp by more than one phase, so its parity names
+      // one phase only (the final wait below relies on the same).
       if (j > 0) {
-        if (!warp_wait(bar(kBOReady), (j - 1) & 1)) break;
+        if (!warp_wait(bar(kBVEmpty + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, raise)) {   // lanes that keep their reference use alpha = 1
 #pragma unroll 1
@@ -432,7 +444,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       if (!(p.test_withhold && j == min(1, n_tiles - 1))) warp_arrive_lead(kBPFull + b);
     }
     // ---- O / l -> shared memory rows (reusing the stages): wait for the last PV
-    const bool ok = __all_sync(0xffffffffu, misc[1] == 0) && warp_wait(bar(kBOReady), (n_tiles - 1) & 1);
+    const bool ok = __all_sync(0xffffffffu, misc[1] == 0) && warp_wait(bar(kBVEmpty + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1);
     tc_fence_after();
     float* os = reinterpret_cast<float*>(smem) + r_local * kPfOsStride;
     const float inv = (ok && l_sum > 0.f) ? (0.0625f / kPfPScale) / l_sum : 0.f;   // 1/256 of P and 1/16 of R^T
@@ -569,7 +581,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       const int32_t pg_far = page_of(j + 4);
       const bool more = j + 2 < n_tiles;
       // ---- K half: free once QK(j - 2) has run
-      if (j >= 2 && !bounded_wait(bar(kBKEmpty + grp_id), ((j >> 1) - 1) & 1)) break;
+      if (j >= 2 && !bounded_wait(bar(kBSFull + grp_id), ((j >> 1) - 1) & 1)) break;   // QK(j - 2) done
       expand(j, 0);
       expand(j, 1);
       cp_async_commit();
@@ -620,53 +632,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       constexpr uint32_t idesc_pv = tc_idesc(2 * kPfRows, kD, 1);
       bool ok = bounded_wait(bar(kBQReady), 0);   // q' of both CTAs stored
       tc_fence_after();
+      // Waits on barriers that have long completed still cost hundreds of cycles, and
+      // between two MMA bursts they would leave the tensor pipe idle. The issue of an
+      // MMA blocks while the tensor core's queue is full, so the next burst's barriers
+      // are looked at (non-blocking) between the MMAs of the current one; the blocking,
+      // bounded wait runs only for a barrier not yet seen complete.
+      bool k_seen = false;    // K_FULL of the next QK seen complete during the last PV burst
       for (int j = 0; ok && j <= n_tiles; ++j) {
+        bool pv_seen = false;   // P_FULL and V_FULL of tile j - 1 seen complete during the QK burst
+        const int jb = j - 1, bp = jb & 1;
+        const uint32_t pv_par = uint32_t(jb >> 1) & 1u;
+        auto look_pv = [&]() {
+          if (j >= 1 && !pv_seen)
+            pv_seen = mbar_test_wait_cluster(bar(kBPFull + bp), pv_par) && mbar_test_wait_cluster(bar(kBVFull + bp), pv_par);
+        };
         if (j < n_tiles) {   // S[j & 1] = Q'hi Khi^T + Q'lo Khi^T + Q'hi Klo^T  (K = 256 dims in 16 steps each)
           const int b = j & 1;
-          if (!bounded_wait(bar(kBKFull + b), (j >> 1) & 1)) break;
+          if (!k_seen && !bounded_wait(bar(kBKFull + b), (j >> 1) & 1)) break;
+          k_seen = false;
           tc_fence_after();
           const uint32_t kb = sbase + b * kPfStage;
           const uint32_t s_t = tmem + kTmS0 + 64 * b;
+          // descriptors of the panels' first rows; a k-step adds its byte offset >> 4 to the
+          // start-address field (no carry: shared addresses stay below 2^18)
+          const uint64_t khi0 = tc_sdesc(kb + kPfKHi, 16, 1024), klo0 = tc_sdesc(kb + kPfKLo, 16, 1024);
+          const uint64_t qlo0 = tc_sdesc(sbase + kPfQloOff, 16, 1024);
 #pragma unroll
           for (int kk = 0; kk < 16; ++kk) {
-            const uint64_t bd = tc_sdesc(kb + kPfKHi + (kk >> 2) * kPfKPanel + (kk & 3) * 32, 16, 1024);
-            tc2_mma_ts(s_t, tmem + kTmQ + 8 * kk, bd, idesc_qk, kk > 0 ? 1u : 0u);
+            const uint64_t o = uint64_t(((kk >> 2) * kPfKPanel + (kk & 3) * 32) >> 4);
+            tc2_mma_ts(s_t, tmem + kTmQ + 8 * kk, khi0 + o, idesc_qk, kk > 0 ? 1u : 0u);
           }
+          look_pv();
 #pragma unroll
           for (int kk = 0; kk < 16; ++kk) {
-            const uint64_t ad = tc_sdesc(sbase + kPfQloOff + (kk >> 2) * kPfQloPanel + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = tc_sdesc(kb + kPfKHi + (kk >> 2) * kPfKPanel + (kk & 3) * 32, 16, 1024);
-            tc2_mma_ss(s_t, ad, bd, idesc_qk, 1u);
+            const uint64_t o = uint64_t(((kk >> 2) * kPfKPanel + (kk & 3) * 32) >> 4);
+            const uint64_t oq = uint64_t(((kk >> 2) * kPfQloPanel + (kk & 3) * 32) >> 4);
+            tc2_mma_ss(s_t, qlo0 + oq, khi0 + o, idesc_qk, 1u);
           }
+          look_pv();
 #pragma unroll
           for (int kk = 0; kk < 16; ++kk) {
-            const uint64_t bd = tc_sdesc(kb + kPfKLo + (kk >> 2) * kPfKPanel + (kk & 3) * 32, 16, 1024);
-            tc2_mma_ts(s_t, tmem + kTmQ + 8 * kk, bd, idesc_qk, 1u);
+            const uint64_t o = uint64_t(((kk >> 2) * kPfKPanel + (kk & 3) * 32) >> 4);
+            tc2_mma_ts(s_t, tmem + kTmQ + 8 * kk, klo0 + o, idesc_qk, 1u);
           }
+          look_pv();
+          // S_FULL also tells the dequant group that the K half of stage b is free again
           tc2_commit_both(bar(kBSFull + b));
-          tc2_commit_both(bar(kBKEmpty + b));
         }
         if (j >= 1) {   // O += P_hi V_hi (+ P_lo V_hi, + P_hi V_lo) for tile j - 1 (K = 64 positions in 4 steps)
-          const int jb = j - 1, b = jb & 1;
-          if (!bounded_wait(bar(kBPFull + b), (jb >> 1) & 1)) break;
-          if (!bounded_wait(bar(kBVFull + b), (jb >> 1) & 1)) break;
+          if (!pv_seen) {
+            if (!bounded_wait(bar(kBPFull + bp), pv_par)) break;
+            if (!bounded_wait(bar(kBVFull + bp), pv_par)) break;
+          }
           tc_fence_after();
-          const volatile float* vm = reinterpret_cast<const volatile float*>(misc) + 8 + 2 * b;
+          const volatile float* vm = reinterpret_cast<const volatile float*>(misc) + 8 + 2 * bp;
           const bool vlo = exact || fmaxf(vm[0], vm[1]) > kVloNorm;
-          const uint32_t vb = sbase + b * kPfStage;
-          const uint32_t p_t = tmem + kTmS0 + 64 * b;
+          const uint32_t vb = sbase + bp * kPfStage;
+          const uint32_t p_t = tmem + kTmS0 + 64 * bp;
+          const uint64_t vhi0 = tc_sdesc(vb + kPfVHi, kPfVPanel, 1024), vlo0 = tc_sdesc(vb + kPfVLo, kPfVPanel, 1024);
+          const int jn = j + 1;   // the next QK's tile
 #pragma unroll
           for (int ks = 0; ks < kPfTile / 16; ++ks) {
-            const uint64_t bh = tc_sdesc(vb + kPfVHi + ks * 16 * 128, kPfVPanel, 1024);
-            tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, bh, idesc_pv, (jb > 0 || ks > 0) ? 1u : 0u);
-            tc2_mma_ts(tmem + kTmO, p_t + 32 + 8 * ks, bh, idesc_pv, 1u);
-            if (vlo) {
-              const uint64_t bl = tc_sdesc(vb + kPfVLo + ks * 16 * 128, kPfVPanel, 1024);
-              tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, bl, idesc_pv, 1u);
-            }
+            const uint64_t o = uint64_t((ks * 16 * 128) >> 4);
+            tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, vhi0 + o, idesc_pv, (jb > 0 || ks > 0) ? 1u : 0u);
+            tc2_mma_ts(tmem + kTmO, p_t + 32 + 8 * ks, vhi0 + o, idesc_pv, 1u);
+            if (vlo) tc2_mma_ts(tmem + kTmO, p_t + 8 * ks, vlo0 + o, idesc_pv, 1u);
+            if (ks == 1 && jn < n_tiles) k_seen = mbar_test_wait_cluster(bar(kBKFull + (jn & 1)), uint32_t(jn >> 1) & 1u);
           }
-          tc2_commit_both(bar(kBVEmpty + b));
-          tc2_commit_both(bar(kBOReady));
+          // V_EMPTY: the V half of stage bp is free, and (to the softmax) PV(j - 1) has completed
+          tc2_commit_both(bar(kBVEmpty + bp));
         }
       }
       // every MMA this thread issued has completed before TMEM is released
