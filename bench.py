@@ -41,7 +41,7 @@ from compressed_paged_kv_tq4_b200 import inputs as I  # noqa: E402
 METRIC = "TQ4 fused attention KV positions/s & HBM GB/s (% of roofline) at 32K–229K ctx"
 UNIT = "KV positions/s"
 SCALE = 1.0 / 16.0
-EXTRA_DEFAULT = "decode_213k_outliers,verify_2req_229k,prefill_2k_on_32k,int8_decode_32k"
+EXTRA_DEFAULT = "decode_213k_outliers,verify_2req_229k,shared_prefix_8req_33k,prefill_2k_on_32k,int8_decode_32k"
 
 
 def parse(argv=None):
@@ -78,7 +78,10 @@ WORKLOAD_DESC = {
     "decode_32k": "16 layers x 32,768 TQ4 positions, 1 request, 1 bf16 query token, 24 Q / 4 KV heads x 256",
     "decode_213k_outliers": "16 layers x 212,992 TQ4 positions (5% x8 outliers), 1 request, 1 query token",
     "verify_2req_229k": "2 requests (163,840 + 65,536 positions, 64 shared pages), 4 causal query tokens each, "
-                        "16 layers",
+                        "16 layers (timed ungrouped; the grouped decode is timed beside it)",
+    "shared_prefix_8req_33k": "8 requests of 33,792 positions sharing their first 32,768 (128 pages), 1 query token "
+                              "each, 16 layers, grouped decode (the shared pages read once; the ungrouped decode "
+                              "is timed beside it)",
     "prefill_2k_on_32k": "2,048 causal bf16 query tokens on a 32,768-position TQ4 prefix + the chunk, 16 layers",
     "single_layer_2k": "1 layer, 2,048 TQ4 positions, 1 query token",
     "int8_decode_32k": "uniform INT8 comparison arm: 16 layers x 32,768 INT8 positions (2,064 B per "
@@ -231,7 +234,17 @@ class DecodeSetup:
         self.total = int(self.seq_np.sum())
         self.n_q = w.n_q
         self.pools = []
+        # requests sharing their first pages: the grouped decode (shared pages read once)
+        # times the workload when w.grouped, else it is timed beside the plain decode
+        self.has_groups = w.shared_prefix_pages > 0 and w.n_req > 1
+        self.shared = self.has_groups and w.grouped
+        self.leader = np.zeros(w.n_req, np.int32)
+        self.pages = np.full(w.n_req, w.shared_prefix_pages, np.int32)
         self.ws = self.ctx.decode_workspace(w.n_req, w.n_q, self.total, device)
+        if self.has_groups:
+            nbytes = tq4.tq4_decode_shared_workspace_bytes(self.ctx.handle, w.n_req, w.n_q, self.total,
+                                                           self.tables.shape[1], self.leader, self.pages)
+            self.ws_shared = torch.empty(nbytes, dtype=torch.uint8, device=device)
         ain, aout = Arena(torch, device), Arena(torch, device)
         qi, ki, vi, oi = [], [], [], []
         for layer in range(w.layers):
@@ -270,10 +283,17 @@ class DecodeSetup:
     def attend(self, layer):
         """The step's append and decode of one layer, one call (the timed attention call)."""
         tq4, w = self.tq4, self.w
-        rc = tq4.tq4_decode_append_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.knew[layer],
-                                             self.vnew[layer], tq4.DTYPE_F32, self.qs[layer], self.tables,
-                                             self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total, SCALE,
-                                             self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
+        if self.shared:
+            rc = tq4.tq4_decode_attention_shared(self.ctx.handle, self.pools[layer], w.pool_pages, self.knew[layer],
+                                                 self.vnew[layer], tq4.DTYPE_F32, self.qs[layer], self.tables,
+                                                 self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total,
+                                                 self.leader, self.pages, SCALE, self.outs[layer], tq4.DTYPE_BF16,
+                                                 self.ws_shared, self.ws_shared.numel())
+        else:
+            rc = tq4.tq4_decode_append_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.knew[layer],
+                                                 self.vnew[layer], tq4.DTYPE_F32, self.qs[layer], self.tables,
+                                                 self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total, SCALE,
+                                                 self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
         assert rc == 0, rc
 
     def step(self):
@@ -288,15 +308,20 @@ class DecodeSetup:
         return self.w.layers * (2 if self.w.n_q == 1 else 3)
 
     def roofline(self, att_ms, peaks_):
-        """Dominant call: one layer's tq4_decode_append_attention; algorithmic bytes =
-        the packed history it must read (1,040 B per attended layer-position)."""
+        """Dominant call: one layer's tq4_decode_append_attention (tq4_decode_attention_shared
+        when requests share pages); algorithmic bytes = the packed history it must read,
+        1,040 B per distinct layer-position (shared pages count once)."""
         hbm = peaks_[0]
-        nbytes = self.total * I.H_KV * 2 * 130
+        distinct = self.total - (self.w.n_req - 1) * self.w.shared_prefix_pages * I.PAGE if self.shared else self.total
+        nbytes = distinct * I.H_KV * 2 * 130
         ach = nbytes / (att_ms * 1e-3) / 1e9
+        kernel = ("tq4_decode_attention_shared with its append (tail encode + one split-K launch of group and "
+                  "private items + combine)" if self.shared else
+                  "tq4_decode_append_attention (split-K decode with the append inside it for one query token "
+                  "+ combine)")
         return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": measured_traffic("decode_q1" if self.w.n_q == 1 else "decode_splitk", self.total),
-                "kernel": "tq4_decode_append_attention (split-K decode with the append inside it for one "
-                          "query token + combine)",
+                "traffic": measured_traffic("decode_q1" if self.w.n_q == 1 else "decode_splitk", distinct),
+                "kernel": kernel,
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms,
                 "peak_source": f"{peaks_[3]} hbm_gbs"}
 
@@ -643,6 +668,26 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
     torch.cuda.synchronize()
     att_ms = ev0.elapsed_time(ev1) / (reps * w.layers)
     res["roofline"] = S.roofline(att_ms, peaks())
+    if getattr(S, "has_groups", False):   # the other decode path on the same pools, timed the same way
+        S.shared = not S.shared
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g3, stream=stream):
+                for layer in range(w.layers):
+                    S.attend(layer)
+            for _ in range(5):
+                g3.replay()
+            ev0.record(stream)
+            for _ in range(reps):
+                g3.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+        del g3
+        S.shared = not S.shared
+        res["roofline"]["other_path"] = {
+            "path": "ungrouped (tq4_decode_append_attention)" if S.shared else "grouped (tq4_decode_attention_shared)",
+            "launch_ms": ev0.elapsed_time(ev1) / (reps * w.layers)}
 
     # end to end through the public API: pinned host inputs in, every layer's output out, each step
     h2d, d2h = S.h2d_d2h()

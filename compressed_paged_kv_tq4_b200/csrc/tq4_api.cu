@@ -1,6 +1,7 @@
 // C ABI of the TQ4 paged-KV attention library: context, argument checks,
 // planning and launches. Every kernel of the library is compiled in this one
 // translation unit (the kernel headers are included below).
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -76,30 +77,48 @@ int check_device(const tq4_ctx* ctx) {
   return dev == ctx->device ? TQ4_OK : TQ4_ERR_ARG;
 }
 
-template <int NT, bool kI8>
+template <int NT, int NTG, bool kI8>
 cudaError_t set_decode_attrs() {
-  cudaError_t e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, kI8, false>,
+  cudaError_t e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, NTG, kI8, false>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(tq4::decode_smem_bytes<NT, kI8>()));
+                                       int(tq4::decode_smem_bytes<NT, NTG, kI8>()));
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, kI8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(tq4::decode_smem_bytes<NT, kI8>()));
+    e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, NTG, kI8, true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(tq4::decode_smem_bytes<NT, NTG, kI8>()));
   return e;
 }
 
 // one split-K decode launch with the output precision chosen at run time
-template <int NT, bool kI8>
+template <int NT, int NTG, bool kI8>
 cudaError_t launch_splitk(dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
   if (p.out_dtype == TQ4_DTYPE_F32)
-    return tq4::launch_pdl(tq4::decode_splitk_kernel<NT, kI8, true>, grid, dim3(tq4::kDecThreads),
-                           tq4::decode_smem_bytes<NT, kI8>(), st, p);
-  return tq4::launch_pdl(tq4::decode_splitk_kernel<NT, kI8, false>, grid, dim3(tq4::kDecThreads),
-                         tq4::decode_smem_bytes<NT, kI8>(), st, p);
+    return tq4::launch_pdl(tq4::decode_splitk_kernel<NT, NTG, kI8, true>, grid, dim3(tq4::kDecThreads),
+                           tq4::decode_smem_bytes<NT, NTG, kI8>(), st, p);
+  return tq4::launch_pdl(tq4::decode_splitk_kernel<NT, NTG, kI8, false>, grid, dim3(tq4::kDecThreads),
+                         tq4::decode_smem_bytes<NT, NTG, kI8>(), st, p);
+}
+// with shared-prefix groups: their items use kShareNT n-tiles
+template <bool kI8>
+cudaError_t launch_splitk_nt(int nt, bool groups, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  constexpr int G = tq4::kShareNT;
+  if (groups && !kI8) {
+    switch (nt) {
+      case 1: return launch_splitk<1, G, false>(grid, st, p);
+      case 2: return launch_splitk<2, G, false>(grid, st, p);
+      default: return launch_splitk<3, G, false>(grid, st, p);
+    }
+  }
+  switch (nt) {
+    case 1: return launch_splitk<1, 1, kI8>(grid, st, p);
+    case 2: return launch_splitk<2, 2, kI8>(grid, st, p);
+    default: return launch_splitk<3, 3, kI8>(grid, st, p);
+  }
 }
 
 struct DecodePlan {
   int split_len;
   int items_ub;
+  int records_ub;
   int rows_pad;
   size_t ws_o_bytes;
   size_t ws_ml_bytes;
@@ -139,17 +158,101 @@ int pool_tensor_map(const void* pool, int32_t num_pages, CUtensorMap* map) {
   return r == CUDA_SUCCESS ? TQ4_OK : TQ4_ERR_CUDA;
 }
 
-DecodePlan plan_decode(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len) {
+// Shared-prefix groups from the caller's per-request description (host arrays):
+// requests with the same leader (leader[r] == r for a leader) share their first
+// pages[r] pages. Groups of more members than one group item's rows allow are cut
+// into several groups over the same pages; past kMaxShareGroups, requests read
+// their shared pages on their own. Returns TQ4_ERR_ARG for an inconsistent
+// description.
+int build_share(int32_t n_req, int32_t n_q, int32_t max_pages, const int32_t* leader, const int32_t* pages,
+                tq4::SharePlan& sp, int64_t& grouped_pos, int64_t& group_pos) {
+  std::memset(&sp, 0, sizeof(sp));
+  grouped_pos = group_pos = 0;
+  if (!leader || !pages) return TQ4_OK;
+  for (int r = 0; r < n_req; ++r) {
+    const int l = leader[r];
+    if (l < 0 || l >= n_req || leader[l] != l || pages[r] < 0 || pages[r] > max_pages || pages[r] != pages[l])
+      return TQ4_ERR_ARG;
+  }
+  const int cap = std::min(tq4::kMaxShareMembers, (8 * tq4::kShareNT) / (tq4::kGroup * n_q));
+  for (int l = 0; l < n_req; ++l) {
+    if (leader[l] != l || pages[l] == 0) continue;
+    int k = 0;
+    for (int r = l; r < n_req; ++r) {
+      if (leader[r] != l) continue;
+      if (k == 0) {
+        if (sp.n_groups == tq4::kMaxShareGroups) break;
+        sp.pos[sp.n_groups] = pages[l] * tq4::kPage;
+        sp.n_mem[sp.n_groups] = 0;
+      }
+      sp.mem[sp.n_groups][k++] = r;
+      sp.n_mem[sp.n_groups] = k;
+      if (k == cap) {   // close this group
+        ++sp.n_groups;
+        k = 0;
+      }
+    }
+    if (k > 0) ++sp.n_groups;
+  }
+  // a group of one member dedups nothing: drop it
+  int out = 0;
+  for (int g = 0; g < sp.n_groups; ++g) {
+    if (sp.n_mem[g] < 2) continue;
+    if (out != g) {
+      sp.pos[out] = sp.pos[g];
+      sp.n_mem[out] = sp.n_mem[g];
+      std::memcpy(sp.mem[out], sp.mem[g], sizeof(sp.mem[g]));
+    }
+    grouped_pos += int64_t(sp.pos[out]) * sp.n_mem[out];
+    group_pos += sp.pos[out];
+    ++out;
+  }
+  sp.n_groups = out;
+  return TQ4_OK;
+}
+
+// Split lengths: one wave of CTAs (one per SM, 4 KV heads each) even in the worst
+// case, where every request's (and group's) last split is a sliver: a request of
+// length s has ceil(s / L) <= s / L + 1 items. With one request the count is exact.
+// A group item scores up to kShareNT n-tiles of rows against each position, so it
+// gets proportionally fewer positions (cost per position taken as 2 + n-tiles: the
+// centroid expansion plus the MMAs of each n-tile).
+DecodePlan plan_decode(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len,
+                       tq4::SharePlan* share = nullptr, int64_t grouped_pos = 0, int64_t group_pos = 0) {
   DecodePlan pl{};
-  const int64_t ctas = int64_t(ctx->num_sms);                // one resident CTA per SM
-  int64_t L = (total_seq_len * tq4::kHkv + ctas - 1) / ctas;  // positions per split
-  L = ((L + tq4::kChunk - 1) / tq4::kChunk) * tq4::kChunk;
-  if (L < tq4::kChunk) L = tq4::kChunk;
-  if (L > (1 << 30)) L = 1 << 30;
+  const int64_t slots = std::max<int64_t>(ctx->num_sms / tq4::kHkv, 1);   // items per KV head in one wave
+  const int64_t own = std::max<int64_t>(total_seq_len - grouped_pos, 0);   // positions outside the groups
+  const int n_groups = share ? share->n_groups : 0;
+  const int nt = tq4::decode_nt(n_q);
+  const double wg = n_groups ? double(2 + tq4::kShareNT) / double(2 + nt) : 1.0;   // group / own cost per position
+  const double work = double(own) + double(group_pos) * wg;
+  const int64_t spare = slots - (n_req == 1 && !n_groups ? 0 : n_req + n_groups);
+  const int64_t div = spare > 0 ? spare : slots;              // too many requests for one wave: as many as fit
+  auto round_chunk = [](int64_t L) {
+    L = ((L + tq4::kChunk - 1) / tq4::kChunk) * tq4::kChunk;
+    return std::min<int64_t>(std::max<int64_t>(L, tq4::kChunk), int64_t(1) << 30);
+  };
+  const int64_t L = round_chunk(int64_t(std::ceil(work / double(div))));
   pl.split_len = int(L);
-  pl.items_ub = int(total_seq_len / L) + n_req;
+  int64_t g_items = 0, g_records = 0;
+  if (share) {
+    // group split: L / wg positions, down to a whole number of chunks
+    const int64_t Lg = std::max<int64_t>(int64_t(double(L) / wg) / tq4::kChunk * tq4::kChunk, tq4::kChunk);
+    share->split_len = int32_t(Lg);
+    share->item0[0] = 0;
+    for (int g = 0; g < share->n_groups; ++g) {
+      const int64_t n = (share->pos[g] + Lg - 1) / Lg;
+      share->item0[g + 1] = int32_t(share->item0[g] + n);
+      g_records += n * share->n_mem[g];
+    }
+    share->n_gitems = share->item0[share->n_groups];
+    g_items = share->n_gitems;
+  }
+  const int64_t own_items = (n_req == 1 && !n_groups) ? (own + L - 1) / L : own / L + n_req;
+  pl.items_ub = int(g_items + own_items);
+  pl.records_ub = int(g_records + own_items);
   pl.rows_pad = 8 * tq4::decode_nt(n_q);
-  const size_t recs = size_t(pl.items_ub) * tq4::kHkv * pl.rows_pad;
+  const size_t recs = size_t(pl.records_ub) * tq4::kHkv * pl.rows_pad;
   pl.ws_o_bytes = align256(recs * tq4::kD * sizeof(float));
   pl.ws_ml_bytes = align256(recs * sizeof(float2));
   pl.total = pl.ws_o_bytes + pl.ws_ml_bytes;
@@ -210,12 +313,15 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(tq4::decode_q1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(tq4::decode_q1_smem_bytes()));
-  if (e == cudaSuccess) e = set_decode_attrs<1, false>();
-  if (e == cudaSuccess) e = set_decode_attrs<2, false>();
-  if (e == cudaSuccess) e = set_decode_attrs<3, false>();
-  if (e == cudaSuccess) e = set_decode_attrs<1, true>();
-  if (e == cudaSuccess) e = set_decode_attrs<2, true>();
-  if (e == cudaSuccess) e = set_decode_attrs<3, true>();
+  if (e == cudaSuccess) e = set_decode_attrs<1, 1, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<2, 2, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<3, 3, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<1, tq4::kShareNT, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<2, tq4::kShareNT, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<3, tq4::kShareNT, false>();
+  if (e == cudaSuccess) e = set_decode_attrs<1, 1, true>();
+  if (e == cudaSuccess) e = set_decode_attrs<2, 2, true>();
+  if (e == cudaSuccess) e = set_decode_attrs<3, 3, true>();
   if (e == cudaSuccess) e = tq4::prefill_tc_set_attrs();
   if (e == cudaSuccess) e = cudaGetSymbolAddress(&ctx->noalloc_scratch, g_noalloc_scratch);
   if (e == cudaSuccess && !ctx->noalloc_scratch) e = cudaErrorInvalidSymbol;
@@ -286,6 +392,16 @@ size_t tq4_decode_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q
   return plan_decode(ctx, n_req, n_q, total_seq_len).total;
 }
 
+size_t tq4_decode_shared_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len,
+                                         int32_t max_pages, const int32_t* prefix_leader,
+                                         const int32_t* prefix_pages) {
+  if (!ctx || n_req <= 0 || n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS || total_seq_len <= 0 || max_pages <= 0) return 0;
+  tq4::SharePlan sp;
+  int64_t grouped_pos = 0, group_pos = 0;
+  if (build_share(n_req, n_q, max_pages, prefix_leader, prefix_pages, sp, grouped_pos, group_pos) != TQ4_OK) return 0;
+  return plan_decode(ctx, n_req, n_q, total_seq_len, &sp, grouped_pos, group_pos).total;
+}
+
 }  // extern "C"
 
 namespace {
@@ -300,7 +416,8 @@ struct AppendArgs {   // the fused append of tq4_decode_append_attention
 int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_t* q, const int32_t* page_tables,
                 int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q, int64_t total_seq_len,
                 float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream,
-                const AppendArgs* app, bool int8 = false) {
+                const AppendArgs* app, bool int8 = false, const int32_t* prefix_leader = nullptr,
+                const int32_t* prefix_pages = nullptr) {
   if (!ctx || n_req < 0) return TQ4_ERR_ARG;
   if (n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS) return TQ4_ERR_UNSUPPORTED;
   if (n_req == 0) return TQ4_OK;
@@ -315,11 +432,15 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
     if (!app->k_new || !app->v_new || !aligned(app->k_new, 16) || !aligned(app->v_new, 16)) return TQ4_ERR_ARG;
     if (app->dtype != TQ4_DTYPE_F32 && app->dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
   }
-  const DecodePlan pl = plan_decode(ctx, n_req, n_q, total_seq_len);
+  tq4::DecodeParams p{};
+  int64_t grouped_pos = 0, group_pos = 0;
+  if (int rc = build_share(n_req, n_q, max_pages, prefix_leader, prefix_pages, p.share, grouped_pos, group_pos))
+    return rc;
+  const bool groups = p.share.n_groups > 0;
+  const DecodePlan pl = plan_decode(ctx, n_req, n_q, total_seq_len, &p.share, grouped_pos, group_pos);
   if (!workspace || workspace_bytes < pl.total || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
   if (int rc = check_device(ctx)) return rc;
 
-  tq4::DecodeParams p{};
   p.pool = static_cast<const uint8_t*>(pool);
   p.num_pages = num_pages;
   p.q = q;
@@ -331,6 +452,7 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
   p.scale = scale;
   p.split_len = pl.split_len;
   p.items_ub = pl.items_ub;
+  p.records_ub = pl.records_ub;
   p.rows_pad = pl.rows_pad;
   p.ws_o = static_cast<float*>(workspace);
   p.ws_ml = reinterpret_cast<float2*>(static_cast<char*>(workspace) + pl.ws_o_bytes);
@@ -343,7 +465,7 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
   p.rotate = int8 ? 0 : 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (app && n_q == 1) {   // appended inside the decode kernel
+  if (app && n_q == 1 && !groups) {   // appended inside the decode kernel
     p.pool_w = static_cast<uint8_t*>(app->pool);
     p.k_new = app->k_new;
     p.v_new = app->v_new;
@@ -355,11 +477,9 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
   }
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   if (int8) {
-    switch (tq4::decode_nt(n_q)) {
-      case 1: e = launch_splitk<1, true>(grid, st, p); break;
-      case 2: e = launch_splitk<2, true>(grid, st, p); break;
-      default: e = launch_splitk<3, true>(grid, st, p); break;
-    }
+    e = launch_splitk_nt<true>(tq4::decode_nt(n_q), false, grid, st, p);
+  } else if (groups) {     // group items and the requests' own items in one launch
+    e = launch_splitk_nt<false>(tq4::decode_nt(n_q), true, grid, st, p);
   } else {
     switch (tq4::decode_nt(n_q)) {
       case 1: {
@@ -373,8 +493,7 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
                               tq4::decode_q1_smem_bytes(), st, p, map);
         break;
       }
-      case 2: e = launch_splitk<2, false>(grid, st, p); break;
-      default: e = launch_splitk<3, false>(grid, st, p); break;
+      default: e = launch_splitk_nt<false>(tq4::decode_nt(n_q), false, grid, st, p); break;
     }
   }
   if (e != cudaSuccess) return TQ4_ERR_CUDA;
@@ -402,6 +521,18 @@ int tq4_decode_append_attention(tq4_ctx* ctx, void* pool, int32_t num_pages, con
   const AppendArgs app{pool, k_new, v_new, new_dtype};
   return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
                      out, out_dtype, workspace, workspace_bytes, stream, &app);
+}
+
+int tq4_decode_attention_shared(tq4_ctx* ctx, void* pool, int32_t num_pages, const void* k_new, const void* v_new,
+                                int new_dtype, const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                const int32_t* seq_lens, int32_t n_req, int32_t n_q, int64_t total_seq_len,
+                                const int32_t* prefix_leader, const int32_t* prefix_pages, float scale, void* out,
+                                int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!prefix_leader || !prefix_pages || (k_new == nullptr) != (v_new == nullptr)) return TQ4_ERR_ARG;
+  const AppendArgs app{pool, k_new, v_new, new_dtype};
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, k_new ? &app : nullptr, false, prefix_leader,
+                     prefix_pages);
 }
 
 int tq4_int8_encode_append(tq4_ctx* ctx, void* pool, int32_t num_pages, const int32_t* page_table,

@@ -13,8 +13,15 @@
 // domain and the combine pass applies R^T once per output row.
 //
 // Work split: grid (items, 4 KV heads); an item is (request, split) where a
-// split is split_len consecutive positions (split_len % 64 == 0). A CTA of 4
-// warps walks its split in chunks of 64 positions:
+// split is split_len consecutive positions (split_len % 128 == 0). Requests that
+// share their leading pages ([STATE] simpleprog.com "Fitting a 27B-Parameter LLM
+// into 24 GiB of Laptop Memory", section "StateTrans": reference-counted shared
+// prefixes) may be grouped: a group item covers a split of the group's shared
+// positions and scores every member's query rows against it, so those pages are
+// loaded and expanded once for the group (up to kShareNT n-tiles of rows); each
+// member's own positions after the shared ones are ordinary items. Every item
+// writes one partial record per request it serves. A CTA of 8 warps walks its
+// split in chunks of 128 positions:
 //   K phase  warp w takes positions 16w..16w+15 of the chunk: S = C_k . Q'^T
 //            on mma.m16n8k16 (M = positions, N = 6 query heads x n_q tokens,
 //            K = dims), nibble pairs decoded through a per-lane smem table.
@@ -49,6 +56,25 @@ constexpr int64_t kI8VScales = kI8KScales + int64_t(kHkv) * kPage * 2;   // 526,
 constexpr int kI8Stages = 2;
 constexpr int kI8StageBytes = 2 * kChunk * 256 + 2 * kChunk * 2;   // K codes, V codes, K scales, V scales
 
+// Shared-prefix groups (the one-launch dedup of shared pages). Items
+// [0, n_gitems) are group items, item0[g] .. item0[g + 1] - 1 those of group g,
+// each over share.split_len shared positions (shorter than a private item's:
+// it scores more query rows); the rest are the requests' private items. A
+// request's records are consecutive: first ceil(pos / share.split_len) for the
+// shared positions of its group (if any), then one per split of its own positions.
+constexpr int kMaxShareGroups = 32;
+constexpr int kMaxShareMembers = 8;
+constexpr int kShareNT = 6;   // a group item's n-tiles: up to 48 query rows
+struct SharePlan {
+  int32_t n_groups;
+  int32_t n_gitems;
+  int32_t split_len;                                   // positions per group item
+  int32_t item0[kMaxShareGroups + 1];
+  int32_t pos[kMaxShareGroups];                        // shared positions (whole pages)
+  int32_t n_mem[kMaxShareGroups];
+  int32_t mem[kMaxShareGroups][kMaxShareMembers];      // member request ids, ascending
+};
+
 struct DecodeParams {
   const uint8_t* pool;
   int32_t num_pages;
@@ -60,10 +86,11 @@ struct DecodeParams {
   int32_t n_q;
   float scale;
   int32_t split_len;
-  int32_t items_ub;
-  int32_t rows_pad;    // 8 * NT
-  float* ws_o;         // [items_ub][4][rows_pad][256]
-  float2* ws_ml;       // [items_ub][4][rows_pad] (m, l)
+  int32_t items_ub;    // grid size (items)
+  int32_t records_ub;  // partial records the workspace holds
+  int32_t rows_pad;    // 8 * NT (one request's query rows, padded)
+  float* ws_o;         // [records][4][rows_pad][256]
+  float2* ws_ml;       // [records][4][rows_pad] (m, l)
   void* out;
   int out_dtype;
   Signs signs;
@@ -78,15 +105,25 @@ struct DecodeParams {
   uint32_t spin_limit;   // polls before a bounded wait gives up (TQ4_ERR_TIMEOUT)
   int test_withhold;     // test hook: withhold the first tile copy of each warp (its wait runs out)
   int rotate;            // 1: o = R^T o' (TQ4, rotated domain); 0: o = o' (the INT8 arm)
+  SharePlan share;       // n_groups == 0: no shared-prefix groups
 };
 
 __host__ __device__ constexpr int decode_nt(int n_q) { return (6 * n_q + 7) / 8; }
 
+// ring stages: three, two for the wide group items (shared memory)
 template <int NT, bool kI8>
-constexpr size_t decode_smem_bytes() {
-  return (kI8 ? size_t(kI8Stages) * kI8StageBytes : size_t(kLutBytes) + size_t(kStages) * kStageBytes) +
+constexpr int decode_stages() { return kI8 ? kI8Stages : (NT >= 4 ? 2 : kStages); }
+template <int NT, bool kI8>
+constexpr size_t decode_item_smem_bytes() {
+  return (kI8 ? size_t(kI8Stages) * kI8StageBytes : size_t(kLutBytes) + size_t(decode_stages<NT, kI8>()) * kStageBytes) +
          2 * size_t(8 * NT) * kQvStride * 2 + 2 * size_t(8 * NT) * kPsStride * 2 + size_t(kDecWarps) * 8 * NT * 4;
 }
+template <int NT, int NTG, bool kI8>
+constexpr size_t decode_smem_bytes() {
+  return decode_item_smem_bytes<NT, kI8>() > decode_item_smem_bytes<NTG, kI8>() ? decode_item_smem_bytes<NT, kI8>()
+                                                                                : decode_item_smem_bytes<NTG, kI8>();
+}
+static_assert(decode_item_smem_bytes<kShareNT, false>() <= 227u * 1024u, "group items fit shared memory");
 
 __device__ __forceinline__ int warp_incl_scan(int v) {
   const int lane = threadIdx.x & 31;
@@ -102,8 +139,25 @@ __device__ __forceinline__ bool seq_ok(int s, int n_q, int max_pages) {
   return s >= n_q && s <= max_pages * kPage;
 }
 
-// Warp-collective: find (request, split) of item x. Returns false if x is not
-// an item. *total receives the number of items (sum of splits).
+// Shared positions of request r (those of its group; 0 if it is in none).
+__device__ __forceinline__ int shared_pos(const DecodeParams& p, int r) {
+  for (int g = 0; g < p.share.n_groups; ++g)
+    for (int k = 0; k < p.share.n_mem[g]; ++k)
+      if (p.share.mem[g][k] == r) return p.share.pos[g];
+  return 0;
+}
+// Records of request r: its group's shared splits, then its own splits (none if
+// its length is inconsistent, which the kernels report).
+__device__ __forceinline__ void request_records(const DecodeParams& p, int r, int s_len, int& n_shared,
+                                                int& n_own) {
+  const int P = shared_pos(p, r);
+  n_shared = P > 0 ? (P + p.share.split_len - 1) / p.share.split_len : 0;
+  n_own = seq_ok(s_len, p.n_q, p.max_pages) ? (max(s_len - P, 0) + p.split_len - 1) / p.split_len : 0;
+}
+
+// Warp-collective: find (request, split) of private item x (counted after the
+// group items). Returns false if x is not an item. *total receives the number of
+// private items.
 __device__ __forceinline__ bool find_item(const DecodeParams& p, int x, int& req, int& split,
                                           int& total) {
   const int lane = threadIdx.x & 31;
@@ -113,8 +167,8 @@ __device__ __forceinline__ bool find_item(const DecodeParams& p, int x, int& req
     const int r = r0 + lane;
     int S = 0;
     if (r < p.n_req) {
-      const int s = __ldg(p.seq_lens + r);
-      S = seq_ok(s, p.n_q, p.max_pages) ? (s + p.split_len - 1) / p.split_len : 0;
+      int nsh = 0;
+      request_records(p, r, __ldg(p.seq_lens + r), nsh, S);
     }
     const int incl = warp_incl_scan(S);
     const int excl = incl - S;
@@ -130,6 +184,25 @@ __device__ __forceinline__ bool find_item(const DecodeParams& p, int x, int& req
   }
   total = base;
   return found;
+}
+
+// Warp-collective: the first record of request r (the records of requests 0..r-1).
+__device__ __forceinline__ int request_first_record(const DecodeParams& p, int r) {
+  const int lane = threadIdx.x & 31;
+  int first = 0;
+  for (int r0 = 0; r0 < r; r0 += 32) {
+    const int rr = r0 + lane;
+    int n = 0;
+    if (rr < r) {
+      int nsh = 0, own = 0;
+      request_records(p, rr, __ldg(p.seq_lens + rr), nsh, own);
+      n = nsh + own;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    first += n;
+  }
+  return first;
 }
 
 __device__ __forceinline__ uint32_t pick(const uint4& a, const uint4& b, int i) {
@@ -170,11 +243,18 @@ __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_
 __device__ __forceinline__ uint2 lds64(const uint8_t* p) { return *reinterpret_cast<const uint2*>(p); }
 __device__ __forceinline__ uint32_t lds32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
+// An item's description in shared memory (written by warp 0 of the CTA)
+constexpr int kItPosB = 0, kItPosE = 1, kItTable = 2, kItNMem = 3, kItReq = 4,
+              kItRec = kItReq + kMaxShareMembers, kItWords = kItRec + kMaxShareMembers;
+
+// One item: positions [pos_b, pos_e) of the pages in request item[kItTable]'s
+// table, scored against the query rows of item[kItNMem] requests (request
+// item[kItReq + k], partial record item[kItRec + k]); NT n-tiles hold their
+// n_mem * 6 * n_q rows (member-major, then token, then head).
 template <int NT, bool kI8, bool kExact>   // kExact: fp32 outputs, C_lo P' on every chunk (see kVloNorm)
-__global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const DecodeParams p) {
-  extern __shared__ __align__(128) uint8_t smem[];
+__device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem, const int* item) {
   constexpr int kRB = kI8 ? 256 : 128;                 // bytes of one staged K or V row
-  constexpr int kNS = kI8 ? kI8Stages : kStages;       // ring stages; chunks prefetched kNS - 1 ahead
+  constexpr int kNS = decode_stages<NT, kI8>();        // ring stages; chunks prefetched kNS - 1 ahead
   constexpr int kSB = kI8 ? kI8StageBytes : kStageBytes;
   const uint32_t lut = smem_u32(smem);                 // the centroid table (TQ4 only)
   uint8_t* ring = smem + (kI8 ? 0 : kLutBytes);
@@ -183,34 +263,17 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   __half* ps_hi = qv_lo + 8 * NT * kQvStride;
   __half* ps_lo = ps_hi + 8 * NT * kPsStride;   // P' = hi + lo, both f16
   float* red = reinterpret_cast<float*>(ps_lo + 8 * NT * kPsStride);   // [warps][8*NT]
-  __shared__ int s_item[2];
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int h = blockIdx.y;
   const uint32_t lane8 = uint32_t(lane) * 8u;
 
-  pdl_wait();   // every read of the call's inputs comes after the previous kernel
-  pdl_launch_dependents();
-  if (w == 0) {
-    int req = 0, split = 0, total = 0;
-    const bool ok = find_item(p, blockIdx.x, req, split, total);
-    if (lane == 0) {
-      s_item[0] = ok ? req : -1;
-      s_item[1] = split;
-      if (blockIdx.x == 0 && h == 0 && total > p.items_ub) record_error(p.status, TQ4_ERR_SEQ);
-    }
-  }
-  __syncthreads();
-  const int r = s_item[0];
-  if (r < 0 || int(blockIdx.x) >= p.items_ub) return;
-  const int split = s_item[1];
-  const int seq_len = __ldg(p.seq_lens + r);
-  const int pos_b = split * p.split_len;
-  const int pos_e = min(pos_b + p.split_len, seq_len);
+  const int pos_b = item[kItPosB], pos_e = item[kItPosE];
   const int n_chunks = (pos_e - pos_b + kChunk - 1) / kChunk;
-  const int NR = 6 * p.n_q;
-  const int32_t* table = p.page_tables + int64_t(r) * p.max_pages;
+  const int NR = 6 * p.n_q;                 // query rows of one request
+  const int NRT = item[kItNMem] * NR;       // query rows of the item
+  const int32_t* table = p.page_tables + int64_t(item[kItTable]) * p.max_pages;
   const int64_t head_slot0 = int64_t(h) * kPage;
 
   // ---- staging: chunk i -> ring stage i % kStages (all threads issue 16-byte copies)
@@ -257,9 +320,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   // (INT8), split hi + lo f16, stored in the K phase's virtual dim order
   for (int row = w; row < 8 * NT; row += kDecWarps) {
     float v[8];
-    if (row < NR) {
-      const int tok = row / 6, j = row % 6;
-      const uint16_t* src = p.q + ((int64_t(r) * p.n_q + tok) * kHq + h * kGroup + j) * kD + lane * 8;
+    if (row < NRT) {
+      const int rq = item[kItReq + row / NR], tok = (row % NR) / 6, j = row % 6;
+      const uint16_t* src = p.q + ((int64_t(rq) * p.n_q + tok) * kHq + h * kGroup + j) * kD + lane * 8;
       const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
       const uint32_t ww[4] = {raw.x, raw.y, raw.z, raw.w};
       if constexpr (kI8) {
@@ -318,14 +381,15 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
     }
   }
 
-  // per-row visibility limits for the rows this thread scores (rows nt*8 + 2t + e)
+  // per-row visibility limits for the rows this thread scores (rows nt*8 + 2t + e):
+  // token tok of request rq sees positions [0, seq_len(rq) - n_q + tok]
   int lim[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int row = nt * 8 + 2 * t + e;
-      lim[nt][e] = row < NR ? seq_len - p.n_q + row / 6 + 1 : 0;
+      lim[nt][e] = row < NRT ? __ldg(p.seq_lens + item[kItReq + row / NR]) - p.n_q + (row % NR) / 6 + 1 : 0;
     }
 
   float m_run[NT][2], l_part[NT][2];
@@ -358,9 +422,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
     // (the two small terms share one accumulator; C_lo q'_lo is below fp32 resolution);
     // INT8 codes are exact f16 values, so there C_lo = 0. Even/odd k-steps use
     // separate accumulators to halve the dependent mma chains.
-    float shh[2][NT][4], sx[2][NT][4];
+    constexpr int kAcc = NT >= 4 ? 1 : 2;   // wide items have NT independent chains already
+    float shh[kAcc][NT][4], sx[kAcc][NT][4];
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int a = 0; a < kAcc; ++a)
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -392,8 +457,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
           for (int nt = 0; nt < NT; ++nt) {
             uint32_t bh0, bh1, bl0, bl1;
             qfrag(kk, nt, bh0, bh1, bl0, bl1);
-            mma_16816(shh[kk & 1][nt], a0, a1, a2, a3, bh0, bh1);
-            mma_16816(sx[kk & 1][nt], a0, a1, a2, a3, bl0, bl1);
+            mma_16816(shh[kk % kAcc][nt], a0, a1, a2, a3, bh0, bh1);
+            mma_16816(sx[kk % kAcc][nt], a0, a1, a2, a3, bl0, bl1);
           }
         }
       }
@@ -423,9 +488,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       for (int nt = 0; nt < NT; ++nt) {
         uint32_t bh0, bh1, bl0, bl1;
         qfrag(kk, nt, bh0, bh1, bl0, bl1);
-        mma_16816(shh[kk & 1][nt], a0, a1, a2, a3, bh0, bh1);
-        mma_16816(sx[kk & 1][nt], a0, a1, a2, a3, bl0, bl1);
-        mma_16816(sx[kk & 1][nt], r0, r1, r2, r3, bh0, bh1);
+        mma_16816(shh[kk % kAcc][nt], a0, a1, a2, a3, bh0, bh1);
+        mma_16816(sx[kk % kAcc][nt], a0, a1, a2, a3, bl0, bl1);
+        mma_16816(sx[kk % kAcc][nt], r0, r1, r2, r3, bh0, bh1);
       }
     }
     }
@@ -442,7 +507,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       for (int j = 0; j < 4; ++j) {
         const int pos = pos0 + 8 * (j >> 1);
         const bool ok = pos < pos_e && pos < lim[nt][j & 1];
-        const float acc = (shh[0][nt][j] + shh[1][nt][j]) + (sx[0][nt][j] + sx[1][nt][j]);
+        const float acc = kAcc == 2 ? (shh[0][nt][j] + shh[kAcc - 1][nt][j]) + (sx[0][nt][j] + sx[kAcc - 1][nt][j])
+                                    : shh[0][nt][j] + sx[0][nt][j];
         s[nt][j] = ok ? acc * ((j >> 1) ? kn8 : kn0) : -INFINITY;
       }
 #pragma unroll
@@ -625,17 +691,21 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
       }
     }
   __syncthreads();
-  const int64_t rec = (int64_t(blockIdx.x) * kHkv + h) * p.rows_pad;
+  // row -> its request's record: (record * 4 + h) * rows_pad + row within the request
+  auto rec_row = [&](int row) {
+    return (int64_t(item[kItRec + row / NR]) * kHkv + h) * p.rows_pad + row % NR;
+  };
   if (ph == 0) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int row = nt * 8 + 2 * t + e;
+        if (row >= NRT) continue;
         const float* sidx = ohalf + (dg * 8 * NT + row) * 64 + 8 * g;
         const float4 u0 = reinterpret_cast<const float4*>(sidx)[0];
         const float4 u1 = reinterpret_cast<const float4*>(sidx)[1];
-        float* dst = p.ws_o + (rec + row) * kD + 64 * dg + 8 * g;
+        float* dst = p.ws_o + rec_row(row) * kD + 64 * dg + 8 * g;
         reinterpret_cast<float4*>(dst)[0] = make_float4(o[nt][0][e] + u0.x, o[nt][0][e + 2] + u0.y,
                                                         o[nt][1][e] + u0.z, o[nt][1][e + 2] + u0.w);
         reinterpret_cast<float4*>(dst)[1] = make_float4(o[nt][2][e] + u1.x, o[nt][2][e + 2] + u1.y,
@@ -648,12 +718,86 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int row = nt * 8 + 2 * t + e;
+        if (row >= NRT) continue;
         float l = 0.f;
 #pragma unroll
         for (int ww = 0; ww < kDecWarps; ++ww) l += red[ww * 8 * NT + row];
-        p.ws_ml[rec + row] = make_float2(m_run[nt][e], l);
+        p.ws_ml[rec_row(row)] = make_float2(m_run[nt][e], l);
       }
   }
+}
+
+// Split-K decode: grid (items, 4 KV heads). Items [0, share.n_gitems) are group
+// items (NTG n-tiles), the rest the requests' own items (NT n-tiles).
+template <int NT, int NTG, bool kI8, bool kExact>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int s_item[kItWords];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int h = blockIdx.y;
+  pdl_wait();   // every read of the call's inputs comes after the previous kernel
+  pdl_launch_dependents();
+  const int x = int(blockIdx.x);
+  const bool group = x < p.share.n_gitems;
+  if (w == 0) {
+    if (group) {   // group gi, split s of its shared positions; one record per member
+      int gi = 0;
+      while (gi + 1 < p.share.n_groups && x >= p.share.item0[gi + 1]) ++gi;
+      const int sp = x - p.share.item0[gi];
+      const int nm = p.share.n_mem[gi];
+      const int gl = p.share.split_len;
+      for (int k = 0; k < nm; ++k) {
+        const int rq = p.share.mem[gi][k];
+        const int first = request_first_record(p, rq);
+        if (lane == 0) {
+          s_item[kItReq + k] = rq;
+          s_item[kItRec + k] = first + sp;
+        }
+      }
+      if (lane == 0) {
+        s_item[kItPosB] = sp * gl;
+        s_item[kItPosE] = min((sp + 1) * gl, p.share.pos[gi]);
+        s_item[kItTable] = p.share.mem[gi][0];
+        s_item[kItNMem] = nm;
+      }
+    } else {       // request req, split sp of its own positions
+      int req = 0, sp = 0, total = 0;
+      const bool ok = find_item(p, x - p.share.n_gitems, req, sp, total);
+      int first = 0, P = 0, nsh = 0, own = 0;
+      if (ok) {
+        first = request_first_record(p, req);
+        P = shared_pos(p, req);
+        request_records(p, req, __ldg(p.seq_lens + req), nsh, own);
+      }
+      if (lane == 0) {
+        s_item[kItNMem] = ok ? 1 : 0;
+        s_item[kItReq] = req;
+        s_item[kItRec] = first + nsh + sp;
+        s_item[kItTable] = req;
+        s_item[kItPosB] = P + sp * p.split_len;
+        s_item[kItPosE] = min(P + (sp + 1) * p.split_len, ok ? __ldg(p.seq_lens + req) : 0);
+        if (x == p.share.n_gitems && h == 0 && p.share.n_gitems + total > p.items_ub)
+          record_error(p.status, TQ4_ERR_SEQ);
+      }
+    }
+  }
+  if (w == 0 && lane == 0) {   // every record this item writes must lie inside the workspace
+    bool in = true;
+    for (int k = 0; k < s_item[kItNMem]; ++k) in = in && s_item[kItRec + k] < p.records_ub;
+    if (!in) {
+      record_error(p.status, TQ4_ERR_SEQ);
+      s_item[kItNMem] = 0;
+    }
+  }
+  __syncthreads();
+  if (s_item[kItNMem] == 0 || x >= p.items_ub) return;
+  if constexpr (NTG != NT) {
+    if (group) {
+      decode_item<NTG, kI8, kExact>(p, smem, s_item);
+      return;
+    }
+  }
+  decode_item<NT, kI8, kExact>(p, smem, s_item);
 }
 
 // One CTA of 8 warps per output row (request, token, query head). Warp w
@@ -663,23 +807,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
 // and written out.
 constexpr int kCombWarps = 8;
 constexpr int kCombBatch = 8;   // splits each warp loads before using any (one L2 round for up to 64 splits)
-
-__device__ __forceinline__ int request_first_item(const DecodeParams& p, int r) {
-  const int lane = threadIdx.x & 31;
-  int first = 0;
-  for (int r0 = 0; r0 < r; r0 += 32) {
-    const int rr = r0 + lane;
-    int S = 0;
-    if (rr < r) {
-      const int s = __ldg(p.seq_lens + rr);
-      S = seq_ok(s, p.n_q, p.max_pages) ? (s + p.split_len - 1) / p.split_len : 0;
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
-    first += S;
-  }
-  return first;
-}
 
 __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const DecodeParams p) {
   __shared__ float s_m[kCombWarps], s_l[kCombWarps];
@@ -696,18 +823,20 @@ __global__ void __launch_bounds__(32 * kCombWarps) decode_combine_kernel(const D
   const int row = tok * kGroup + qh % kGroup;
 
   const int s_len = __ldg(p.seq_lens + r);   // issued before the scan below needs anything
-  int first = 0;   // a single request's splits start at item 0
+  int first = 0;   // a single request's records start at 0
   if (p.n_req > 1) {
     if (w == 0) {
-      const int f = request_first_item(p, r);
+      const int f = request_first_record(p, r);
       if (lane == 0) s_first = f;
     }
     __syncthreads();
     first = s_first;
   }
   const bool ok = seq_ok(s_len, p.n_q, p.max_pages);
-  int n_split = ok ? (s_len + p.split_len - 1) / p.split_len : 0;
-  if (first + n_split > p.items_ub) n_split = 0;
+  int nsh = 0, own = 0;
+  request_records(p, r, s_len, nsh, own);
+  int n_split = ok ? nsh + own : 0;   // the request's records: shared splits, then its own
+  if (first + n_split > p.records_ub) n_split = 0;
   if (threadIdx.x == 0 && (!ok || n_split == 0)) record_error(p.status, TQ4_ERR_SEQ);
 
   float m = -INFINITY, l = 0.f, acc[8];

@@ -175,6 +175,7 @@ class Workload:
     outlier_frac: float = 0.0
     append_per_step: int = 0  # positions appended by tq4_encode_append per layer per step
     shared_prefix_pages: int = 0
+    grouped: bool = False    # attend through the shared-prefix (grouped) decode
     prefix_len: int = 0      # prefill only
 
     @property
@@ -194,6 +195,10 @@ WORKLOADS = {
     # 2 requests (163,840 and 65,536 positions; first 64 pages shared), 4 causal query tokens each
     "verify_2req_229k": Workload("verify_2req_229k", 3, 16, POOL_PAGES, (163_840, 65_536), 4,
                                  "decode", shared_prefix_pages=64, append_per_step=4),
+    # 8 requests sharing a 32,768-position prefix (128 pages), 1,024 own positions each,
+    # one query token: the grouped decode reads the shared pages once for all eight
+    "shared_prefix_8req_33k": Workload("shared_prefix_8req_33k", 5, 16, POOL_PAGES, (33_792,) * 8, 1, "decode",
+                                       shared_prefix_pages=128, grouped=True, append_per_step=1),
     # the uniform INT8 comparison arm on the decode_32k shape (same config, same law of K/V)
     "int8_decode_32k": Workload("int8_decode_32k", 1, 16, POOL_PAGES, (32768,), 1, "decode_int8",
                                 append_per_step=1),

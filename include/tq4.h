@@ -182,6 +182,40 @@ int tq4_decode_append_attention(tq4_ctx* ctx, void* pool, int32_t num_pages,
                                 void* out, int out_dtype,
                                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode over requests that share leading pages, reading the shared pages once
+ * ([STATE] simpleprog.com, "Fitting a 27B-Parameter LLM into 24 GiB of Laptop
+ * Memory", section "StateTrans", and [REUSE] section "Prefix Reuse": a restored
+ * prefix is referenced by every request that reuses it, so several requests'
+ * tables hold the same page ids). Same computation and arguments as
+ * tq4_decode_attention (tq4_decode_append_attention when k_new, v_new are given;
+ * both NULL: no append), plus:
+ *   prefix_leader host int32[n_req]: the request whose table this request's first
+ *                 pages share (the same page ids); a leader names itself.
+ *   prefix_pages  host int32[n_req]: the number of shared leading pages; equal for
+ *                 every request of a group (leader included), at most max_pages.
+ * Requests with the same leader form a group; its shared positions are loaded
+ * and expanded once per KV head and scored against all members' query rows in
+ * one pass (at most 48 rows, i.e. 8 one-token, 4 two-token or 2 three/four-token
+ * members per group; larger groups are cut into several; past 32 groups the
+ * rest read their shared pages on their own). Shared pages must hold history:
+ * every member's seq_len - n_q must be at least prefix_pages * 256 (positions a
+ * query may not see are still masked). Results equal tq4_decode_attention's up
+ * to fp32 summation order. A leader out of range, a leader that is not its own
+ * leader, or unequal page counts within a group: TQ4_ERR_ARG. The append (n_q
+ * tokens per request) runs as a tail-encode kernel ahead of the decode.
+ *   workspace    device, at least tq4_decode_shared_workspace_bytes(...) bytes. */
+size_t tq4_decode_shared_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q,
+                                         int64_t total_seq_len, int32_t max_pages,
+                                         const int32_t* prefix_leader, const int32_t* prefix_pages);
+int tq4_decode_attention_shared(tq4_ctx* ctx, void* pool, int32_t num_pages,
+                                const void* k_new, const void* v_new, int new_dtype,
+                                const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                int64_t total_seq_len, const int32_t* prefix_leader,
+                                const int32_t* prefix_pages, float scale,
+                                void* out, int out_dtype,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Prefill attention: a causal chunk of n_tok query tokens against the request's
  * TQ4 prefix [0, prefix_len) plus the chunk itself, whose K/V are given at full
  * precision ([KVEXEC] multi-query prefill). The chunk is not appended; call
