@@ -82,7 +82,8 @@ WORKLOAD_DESC = {
     "shared_prefix_8req_33k": "8 requests of 33,792 positions sharing their first 32,768 (128 pages), 1 query token "
                               "each, 16 layers, grouped decode (the shared pages read once; the ungrouped decode "
                               "is timed beside it)",
-    "prefill_2k_on_32k": "2,048 causal bf16 query tokens on a 32,768-position TQ4 prefix + the chunk, 16 layers",
+    "prefill_2k_on_32k": "2,048 causal bf16 query tokens on a 32,768-position TQ4 prefix + the chunk, 16 layers "
+                         "(packed prefix; direct inverse reconstruction timed beside it)",
     "single_layer_2k": "1 layer, 2,048 TQ4 positions, 1 query token",
     "int8_decode_32k": "uniform INT8 comparison arm: 16 layers x 32,768 INT8 positions (2,064 B per "
                        "layer-position), 1 request, 1 bf16 query token, append of 1 position per layer",
@@ -237,6 +238,7 @@ class DecodeSetup:
         # requests sharing their first pages: the grouped decode (shared pages read once)
         # times the workload when w.grouped, else it is timed beside the plain decode
         self.has_groups = w.shared_prefix_pages > 0 and w.n_req > 1
+        self.has_alt = self.has_groups
         self.shared = self.has_groups and w.grouped
         self.leader = np.zeros(w.n_req, np.int32)
         self.pages = np.full(w.n_req, w.shared_prefix_pages, np.int32)
@@ -299,6 +301,12 @@ class DecodeSetup:
     def step(self):
         for layer in range(self.w.layers):
             self.attend(layer)
+
+    def flip(self):   # grouped <-> ungrouped decode
+        self.shared = not self.shared
+
+    def alt_name(self):   # the path not timed as the workload's
+        return "ungrouped (tq4_decode_append_attention)" if self.shared else "grouped (tq4_decode_attention_shared)"
 
     def units_per_step(self):
         return self.total * self.w.layers  # attended KV positions x layers
@@ -412,7 +420,11 @@ class PrefillSetup:
         self.table = torch.from_numpy(self.tables_np[0]).to(device)
         self.P, self.n = w.prefix_len, w.n_q
         self.pools = []
-        self.ws = torch.empty(tq4.tq4_prefill_workspace_bytes(self.n), dtype=torch.uint8, device=device)
+        # room for the direct-reconstruction variant too (timed beside the packed path)
+        self.reconstruct = False
+        self.has_alt = True
+        self.ws = torch.empty(tq4.tq4_prefill_reconstructed_workspace_bytes(self.P, self.n), dtype=torch.uint8,
+                              device=device)
         ain, aout = Arena(torch, device), Arena(torch, device)
         idx = []
         for layer in range(w.layers):
@@ -439,10 +451,19 @@ class PrefillSetup:
 
     def attend(self, layer):
         tq4, w = self.tq4, self.w
-        rc = tq4.tq4_prefill_attention(self.ctx.handle, self.pools[layer], w.pool_pages, self.table,
-                                       self.table.numel(), self.P, self.q[layer], self.kc[layer], self.vc[layer],
-                                       self.n, SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
+        fn = tq4.tq4_prefill_attention_reconstructed if self.reconstruct else tq4.tq4_prefill_attention
+        rc = fn(self.ctx.handle, self.pools[layer], w.pool_pages, self.table, self.table.numel(), self.P,
+                self.q[layer], self.kc[layer], self.vc[layer], self.n, SCALE, self.outs[layer], tq4.DTYPE_BF16,
+                self.ws, self.ws.numel())
         assert rc == 0, rc
+
+    def flip(self):   # packed prefix <-> direct inverse reconstruction
+        self.reconstruct = not self.reconstruct
+
+    def alt_name(self):
+        return ("packed prefix (tq4_prefill_attention)" if self.reconstruct else
+                "direct inverse reconstruction (tq4_prefill_attention_reconstructed: dense prefix rows, then "
+                "the same attention kernel)")
 
     def append(self, layer):
         tq4, w = self.tq4, self.w
@@ -668,8 +689,8 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
     torch.cuda.synchronize()
     att_ms = ev0.elapsed_time(ev1) / (reps * w.layers)
     res["roofline"] = S.roofline(att_ms, peaks())
-    if getattr(S, "has_groups", False):   # the other decode path on the same pools, timed the same way
-        S.shared = not S.shared
+    if getattr(S, "has_alt", False):   # the workload's other path on the same inputs, timed the same way
+        S.flip()
         g3 = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             torch.cuda.synchronize()
@@ -684,10 +705,8 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
             ev1.record(stream)
         torch.cuda.synchronize()
         del g3
-        S.shared = not S.shared
-        res["roofline"]["other_path"] = {
-            "path": "ungrouped (tq4_decode_append_attention)" if S.shared else "grouped (tq4_decode_attention_shared)",
-            "launch_ms": ev0.elapsed_time(ev1) / (reps * w.layers)}
+        S.flip()
+        res["roofline"]["other_path"] = {"path": S.alt_name(), "launch_ms": ev0.elapsed_time(ev1) / (reps * w.layers)}
 
     # end to end through the public API: pinned host inputs in, every layer's output out, each step
     h2d, d2h = S.h2d_d2h()

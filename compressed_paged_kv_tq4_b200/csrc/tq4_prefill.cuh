@@ -29,11 +29,69 @@ struct PrefillParams {
   int* status;
   uint32_t spin_limit;  // polls before a bounded wait gives up (TQ4_ERR_TIMEOUT)
   int test_withhold;    // test hook: withhold the softmax's P signal of one tile (the issuer's wait runs out)
+  // direct inverse reconstruction: the prefix rebuilt as dense rows [prefix_len][4][256]
+  // (n c[idx] in the rotated domain, hi and lo) read like the chunk's rows; nullptr:
+  // the prefix is expanded from the packed pages inside the kernel
+  const __half* pkr;
+  const __half* pkrlo;
+  const __half* pvr;
+  const __half* pvrlo;
 };
 
 // q' hi, q' lo, R k hi, R k lo, R v hi, R v lo
 inline size_t prefill_workspace_bytes(int32_t n_tok) {
   return size_t(n_tok) * (2 * kHq + 4 * kHkv) * kD * sizeof(__half);
+}
+// the reconstructed prefix's K hi, K lo, V hi, V lo rows
+inline size_t prefill_prefix_rows_bytes(int32_t prefix_len) {
+  return size_t(prefix_len) * 4 * kHkv * kD * sizeof(__half);
+}
+
+// Direct inverse reconstruction of the prefix ([KVEXEC] simpleprog.com "Fitting a
+// 27B-Parameter LLM into 24 GiB of Laptop Memory", section "KVExec": multi-query
+// prefill reconstructs the history directly, with the packed path as the
+// alternative): every prefix vector becomes a dense row n * c[idx] in the rotated
+// domain, split f16 hi + lo. One warp per (position, KV head, K/V); lane l unpacks
+// word l (coordinates 8 l .. 8 l + 7). A page id out of range records
+// TQ4_ERR_PAGE_RANGE and leaves a zero row.
+__global__ void __launch_bounds__(256) prefill_reconstruct_rows_kernel(
+    const uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table, int32_t prefix_len,
+    __half* __restrict__ kr, __half* __restrict__ krlo, __half* __restrict__ vr, __half* __restrict__ vrlo,
+    int* status) {
+  __shared__ float cb[16];   // the centroids (a per-lane index into constant memory would serialise)
+  if (threadIdx.x < 16) cb[threadIdx.x] = g_codebook.c[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);   // (pos, h, kv)
+  pdl_wait();   // the pool may be written by the previous kernel
+  pdl_launch_dependents();
+  if (vec >= int64_t(prefix_len) * kHkv * 2) return;
+  const int kv = int(vec & 1), h = int((vec >> 1) % kHkv);
+  const int64_t pos = (vec >> 1) / kHkv;
+  const int32_t page = __ldg(page_table + (pos >> 8));
+  float v[8];
+  if (page >= 0 && page < num_pages) {
+    const uint8_t* pg = pool + int64_t(page) * kPageBytes;
+    const int slot = h * kPage + int(pos & (kPage - 1));
+    const uint32_t word = __ldg(reinterpret_cast<const uint32_t*>(pg + (kv ? kVWords : kKWords) + int64_t(slot) * 128) + lane);
+    const float n = ldg_half(pg + (kv ? kVNorms : kKNorms) + slot * 2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = n * cb[(word >> (4 * i)) & 15u];
+  } else {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  }
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hi[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hi[i]));
+    lo[i] = pack_half2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+  }
+  const int64_t row = (pos * kHkv + h) * kD + lane * 8;
+  *reinterpret_cast<uint4*>((kv ? vr : kr) + row) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  *reinterpret_cast<uint4*>((kv ? vrlo : krlo) + row) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
 // one warp per vector: rotate queries (with scale) and the chunk's K/V; f16 hi + lo

@@ -29,7 +29,7 @@
 //               its q' hi row into TMEM and its q' lo row into shared memory.
 //               Reads its score row from TMEM, applies K norms, the causal mask
 //               and an online softmax with a lazily raised reference; writes
-//               P = p * n_v / 256 over S (f16 hi and lo).
+//               P = p * n_v / 16 over S (f16 hi and lo).
 //   warps 4-11  dequant, two groups of four; group g fills stage g for tiles
 //               g, g+2, ...: packed words are prefetched into registers two
 //               tiles ahead and expanded through a per-lane table of 8-byte
@@ -77,7 +77,11 @@ static_assert(uint32_t(kPfRows * kPfOsStride * 4) <= kPfLutOff, "epilogue rows o
 static_assert(kPfSmem <= 227u * 1024u, "shared memory");
 static_assert(kPfQloOff % 1024 == 0 && kPfStage % 1024 == 0 && kPfKPart % 1024 == 0 && kPfKPanel % 1024 == 0,
               "swizzled panels start on 1 KiB");
-constexpr float kPfPScale = 1.0f / 256.0f;   // P carries 1/256, undone in the epilogue
+// P = p * n_v * kPfPScale, undone in the epilogue. p <= 2^8 (the lazy reference) and
+// n_v stays below ~300 even for 8x outliers, so P < 4,800 fits f16; a larger scale
+// keeps the small weights of dense rows (n_v = 1: chunk rows, reconstructed prefix
+// rows) out of f16's subnormal range.
+constexpr float kPfPScale = 1.0f / 16.0f;
 constexpr float kPfLazy = 8.0f;              // raise the row reference only when the max grows by > 2^8
 
 // TMEM columns
@@ -447,7 +451,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     const bool ok = __all_sync(0xffffffffu, misc[1] == 0) && warp_wait(bar(kBVEmpty + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1);
     tc_fence_after();
     float* os = reinterpret_cast<float*>(smem) + r_local * kPfOsStride;
-    const float inv = (ok && l_sum > 0.f) ? (0.0625f / kPfPScale) / l_sum : 0.f;   // 1/256 of P and 1/16 of R^T
+    const float inv = (ok && l_sum > 0.f) ? (0.0625f / kPfPScale) / l_sum : 0.f;   // the scale of P and 1/16 of R^T
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       uint32_t ov[32];
@@ -479,6 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     const uint32_t lut_s = sbase + kPfLutOff;
     const uint32_t lane16 = uint32_t(lane & 15) * 16u;   // (byte << 8 | 16 copy) >> 1 = byte * 128 + 8 copy
     const int prefix_end = min(p.prefix_len, kv_end);
+    const bool dense = p.pkr != nullptr;   // the prefix comes as reconstructed rows, not packed words
     const uint32_t st_s = sbase + grp_id * kPfStage;
     float* nb = norms + grp_id * 2 * kPfTile;
     const uint8_t* const pool = p.pool;
@@ -500,10 +505,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     auto page_of = [=](int j) -> int32_t {
       return (j < n_tiles && j * kPfTile < prefix_end) ? __ldg(page_table + ((j * kPfTile) >> 8)) : 0;
     };
-    auto fetch = [&raw, prefix_end, pool, num_pages, h, status, &unit_pos, &unit_grp](int j, int u, int32_t page) {
+    auto fetch = [&raw, prefix_end, dense, pool, num_pages, h, status, &unit_pos, &unit_grp](int j, int u, int32_t page) {
       const int pos = j * kPfTile + unit_pos(u);
       raw[u] = make_uint4(0, 0, 0, 0);
-      if (pos < prefix_end) {
+      if (pos < prefix_end && !dense) {
         if (page >= 0 && page < num_pages) {
           const uint8_t* pg = pool + int64_t(page) * kPageBytes;
           const int slot = h * kPage + (pos & (kPage - 1));
@@ -530,7 +535,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       const int prow = (u < 2 ? pl - int(rank) * kPfKPos : pl) * 128;
       const uint32_t hi_s = st_s + (u < 2 ? kPfKHi + (g >> 1) * kPfKPanel : kPfVHi + (g >> 1) * kPfVPanel) + prow;
       const uint32_t lo_s = hi_s + (u < 2 ? kPfKLo - kPfKHi : kPfVLo - kPfVHi);
-      if (pos < prefix_end) {
+      if (pos < prefix_end && !dense) {
         const uint32_t ww[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {   // word c = dims 8c .. 8c + 7 of the span
@@ -549,10 +554,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
         }
         return;
       }
-      if (pos < kv_end) {
-        const int64_t row = (int64_t(pos - p.prefix_len) * kHkv + h) * kD + 32 * unit_grp(u);
-        const __half* src_hi = (u < 2 ? p.kr : p.vr) + row;
-        const __half* src_lo = (u < 2 ? p.krlo : p.vrlo) + row;
+      if (pos < kv_end) {   // a chunk row, or a reconstructed prefix row
+        const bool pre = pos < p.prefix_len;
+        const int64_t row = (int64_t(pre ? pos : pos - p.prefix_len) * kHkv + h) * kD + 32 * unit_grp(u);
+        const __half* src_hi = (u < 2 ? (pre ? p.pkr : p.kr) : (pre ? p.pvr : p.vr)) + row;
+        const __half* src_lo = (u < 2 ? (pre ? p.pkrlo : p.krlo) : (pre ? p.pvrlo : p.vrlo)) + row;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint32_t off = uint32_t(((c0 + c) ^ sw) << 4);
@@ -601,12 +607,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       {
         const int pl = gt & 63;
         const bool chunk = j * kPfTile + pl >= prefix_end && j * kPfTile + pl < kv_end;
-        const float n = chunk ? 1.f : rawn;   // chunk rows carry their own length
+        const bool row = chunk || (dense && j * kPfTile + pl < prefix_end);
+        const float n = row ? 1.f : rawn;   // dense rows (chunk or reconstructed) carry their own length
         if (gt < 64) {
           nb[pl] = n * kLog2e;
         } else {
           nb[kPfTile + pl] = n * kPfPScale;
-          float m = chunk ? 16.f : n;   // a rotated N(0,1) chunk row has length ~16
+          float m = chunk ? 16.f : rawn;   // the V norm (a rotated N(0,1) chunk row has length ~16)
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
           if (lane == 0) vmax_slot[wq - 2] = m;   // read by the issuer after v_full
@@ -759,12 +766,13 @@ inline cudaError_t prefill_tc_set_attrs() {
   return cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPfSmem));
 }
 
-// rotate prologue, then the tcgen05 attention kernel (clusters of two CTAs)
+// rotate prologue (and, with reconstruct, the prefix's dense rows), then the
+// tcgen05 attention kernel (clusters of two CTAs)
 inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,
                                      int32_t prefix_len, const uint16_t* q, const uint16_t* kc,
                                      const uint16_t* vc, int32_t n_tok, float scale, void* out, int out_dtype,
                                      void* workspace, const Signs& signs, int* status, uint32_t spin_limit,
-                                     int test_withhold, cudaStream_t stream) {
+                                     int test_withhold, cudaStream_t stream, bool reconstruct = false) {
   __half* qr = static_cast<__half*>(workspace);
   __half* qlo = qr + size_t(n_tok) * kHq * kD;
   __half* kr = qlo + size_t(n_tok) * kHq * kD;
@@ -776,6 +784,18 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
                              n_tok, scale, qr, qlo, kr, krlo, vr, vrlo, signs);
   if (e != cudaSuccess) return e;
   PrefillParams p{};
+  if (reconstruct && prefix_len > 0) {   // rows after the chunk's: [prefix_len][4][256] each
+    __half* rows = vrlo + size_t(n_tok) * kHkv * kD;
+    const size_t n = size_t(prefix_len) * kHkv * kD;
+    p.pkr = rows;
+    p.pkrlo = rows + n;
+    p.pvr = rows + 2 * n;
+    p.pvrlo = rows + 3 * n;
+    const int64_t rvecs = int64_t(prefix_len) * kHkv * 2;
+    e = launch_pdl(prefill_reconstruct_rows_kernel, dim3(unsigned((rvecs + 7) / 8)), dim3(256), 0, stream, pool,
+                   num_pages, page_table, prefix_len, rows, rows + n, rows + 2 * n, rows + 3 * n, status);
+    if (e != cudaSuccess) return e;
+  }
   p.pool = pool;
   p.num_pages = num_pages;
   p.page_table = page_table;

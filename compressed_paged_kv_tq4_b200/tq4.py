@@ -45,6 +45,7 @@ EXPORTS = (
     "tq4_prefill_attention", "tq4_get_status", "tq4_status_string", "tq4_decode_attention_noalloc",
     "tq4_decode_append_attention", "tq4_ctx_set_wait_limit", "tq4_int8_encode_append", "tq4_int8_decode_attention",
     "tq4_decode_shared_workspace_bytes", "tq4_decode_attention_shared",
+    "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -94,6 +95,9 @@ _sig = {
     "tq4_decode_shared_workspace_bytes": ([_p, _i32, _i32, _i64, _i32, _p, _p], _sz),
     "tq4_decode_attention_shared": ([_p, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32, _i32, _i64, _p, _p,
                                      _f, _p, ctypes.c_int, _p, _sz, _p], ctypes.c_int),
+    "tq4_prefill_reconstructed_workspace_bytes": ([_i32, _i32], _sz),
+    "tq4_prefill_attention_reconstructed": ([_p, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p, ctypes.c_int,
+                                             _p, _sz, _p], ctypes.c_int),
     "tq4_pages_create": ([_i32, ctypes.POINTER(_p)], ctypes.c_int),
     "tq4_pages_destroy": ([_p], ctypes.c_int),
     "tq4_pages_reservation": ([_i64, _i64], _i64),
@@ -229,6 +233,19 @@ def tq4_prefill_attention(ctx, pool, num_pages, page_table, table_len, prefix_le
     return _lib.tq4_prefill_attention(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len, prefix_len,
                                       _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale, _ptr(out), out_dtype,
                                       _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_prefill_reconstructed_workspace_bytes(prefix_len, n_tok) -> int:
+    return _lib.tq4_prefill_reconstructed_workspace_bytes(prefix_len, n_tok)
+
+
+def tq4_prefill_attention_reconstructed(ctx, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk,
+                                        v_chunk, n_tok, scale, out, out_dtype, workspace, workspace_bytes,
+                                        stream=None) -> int:
+    return _lib.tq4_prefill_attention_reconstructed(ctx, _ptr(pool), num_pages, _ptr(page_table), table_len,
+                                                    prefix_len, _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale,
+                                                    _ptr(out), out_dtype, _ptr(workspace), workspace_bytes,
+                                                    _stream(stream))
 
 
 def tq4_int8_encode_append(ctx, pool, num_pages, page_table, table_len, start_pos, n_tok, k_new, v_new,
@@ -529,19 +546,22 @@ class Context:
         return out
 
     def prefill_attention(self, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,
-                          out_dtype=torch.bfloat16, workspace=None, stream=None):
-        """q: bf16 [n_tok, 24, 256]; k_chunk/v_chunk bf16 [n_tok, 4, 256]; out bf16 or float32."""
+                          out_dtype=torch.bfloat16, workspace=None, stream=None, reconstruct=False):
+        """q: bf16 [n_tok, 24, 256]; k_chunk/v_chunk bf16 [n_tok, 4, 256]; out bf16 or float32.
+        reconstruct=True: the direct-inverse-reconstruction variant (the prefix rebuilt as
+        dense rows first)."""
         _need_cuda(q, k_chunk, v_chunk)
         n_tok = q.shape[0]
         if out is None:
             out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
         od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
         if workspace is None:
-            workspace = torch.empty(max(tq4_prefill_workspace_bytes(n_tok), 256), dtype=torch.uint8,
-                                    device=q.device)
+            nbytes = (tq4_prefill_reconstructed_workspace_bytes(prefix_len, n_tok) if reconstruct
+                      else tq4_prefill_workspace_bytes(n_tok))
+            workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
         num_pages = pool.numel() // PAGE_BYTES if pool is not None else 0
         tlen = page_table.numel() if page_table is not None else 0
-        _check(tq4_prefill_attention(self.handle, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk,
-                                     v_chunk, n_tok, scale, out, od, workspace, workspace.numel(), stream),
-               "tq4_prefill_attention")
+        fn = tq4_prefill_attention_reconstructed if reconstruct else tq4_prefill_attention
+        _check(fn(self.handle, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk, v_chunk, n_tok, scale, out,
+                  od, workspace, workspace.numel(), stream), fn.__name__)
         return out

@@ -236,6 +236,24 @@ int tq4_prefill_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                           int32_t n_tok, float scale, void* out, int out_dtype,
                           void* workspace, size_t workspace_bytes, void* stream);
 
+/* The same prefill by direct inverse reconstruction ([KVEXEC]: multi-query
+ * prefill reconstructs the history directly, with the packed path as the
+ * alternative): a prologue kernel rebuilds every prefix K/V vector as a dense
+ * rotated-domain row n * c[idx] (f16 hi + lo) in the workspace, and the attention
+ * kernel then reads prefix positions as rows, like the chunk's own, instead of
+ * expanding packed words. Same arguments, results (up to fp32 rounding order) and
+ * errors as tq4_prefill_attention; the prefix rows cost
+ * prefix_len * 8 KiB of workspace and their write and re-reads in HBM.
+ *   workspace device scratch of tq4_prefill_reconstructed_workspace_bytes(
+ *             prefix_len, n_tok) bytes, 256-B aligned. */
+size_t tq4_prefill_reconstructed_workspace_bytes(int32_t prefix_len, int32_t n_tok);
+int tq4_prefill_attention_reconstructed(tq4_ctx* ctx, const void* pool, int32_t num_pages,
+                                        const int32_t* page_table, int32_t table_len,
+                                        int32_t prefix_len, const uint16_t* q,
+                                        const uint16_t* k_chunk, const uint16_t* v_chunk,
+                                        int32_t n_tok, float scale, void* out, int out_dtype,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bounded device-side waits (a tile's copy, a tensor-core step, the fused
  * append) give up after a number of polls, record TQ4_ERR_TIMEOUT in the status
  * word and let the kernel finish without the rest of its work: it drains the

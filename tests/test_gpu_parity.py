@@ -255,11 +255,14 @@ def test_decode_page_table_permutation_invariance():
 
 # (prefix_len, n_tok, outlier_frac): one or several 128-row blocks per KV head with a
 # ragged last block; prefixes that end inside a 64-position tile and cross pages;
-# 5% x8 outlier norms, whose large scores raise the softmax reference mid-walk
+# 5% x8 outlier norms, whose large scores raise the softmax reference mid-walk. Both
+# prefill paths: the prefix expanded from packed words inside the attention kernel,
+# and rebuilt as dense rows first (direct inverse reconstruction)
+@pytest.mark.parametrize("reconstruct", [False, True])
 @pytest.mark.parametrize("prefix_len,n_tok,outliers", [(300, 70, 0.0), (0, 5, 0.0), (512, 64, 0.0), (1, 1, 0.0),
                                                        (777, 130, 0.0), (1000, 200, 0.0), (600, 43, 0.05),
                                                        (2048, 22, 0.05), (1500, 90, 0.05), (64, 300, 0.0)])
-def test_prefill_parity(codebook, prefix_len, n_tok, outliers):
+def test_prefill_parity(codebook, prefix_len, n_tok, outliers, reconstruct):
     c, _ = codebook
     signs = I.signs(4)
     ctx = tq4.Context(signs)
@@ -275,7 +278,8 @@ def test_prefill_parity(codebook, prefix_len, n_tok, outliers):
         O.encode_append(opool, table, 0, k, v, signs, c)
     qb = I.queries(4, 0, (n_tok, 24, 256))
     kb, vb = I.chunk_kv(4, 0, n_tok)
-    out = ctx.prefill_attention(pool, tt, prefix_len, _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE)
+    out = ctx.prefill_attention(pool, tt, prefix_len, _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE,
+                                reconstruct=reconstruct)
     torch.cuda.synchronize()
     assert ctx.status() == tq4.TQ4_OK
     exp = O.prefill_attention(opool, table, prefix_len, I.bf16_bits_to_f32(qb), I.bf16_bits_to_f32(kb),
@@ -283,11 +287,17 @@ def test_prefill_parity(codebook, prefix_len, n_tok, outliers):
     H.assert_bf16_close(out.float().cpu().numpy(), exp, f"prefill {prefix_len}+{n_tok} outliers {outliers}")
     # fp32 output on the oracle's own pool bytes: the attention arithmetic alone, every row
     out32 = ctx.prefill_attention(torch.from_numpy(opool).cuda(), tt, prefix_len, _bf16_tensor(qb), _bf16_tensor(kb),
-                                  _bf16_tensor(vb), SCALE, out_dtype=torch.float32)
+                                  _bf16_tensor(vb), SCALE, out_dtype=torch.float32, reconstruct=reconstruct)
     torch.cuda.synchronize()
     assert ctx.status() == tq4.TQ4_OK
     err = np.abs(out32.cpu().numpy().astype(np.float64) - exp).max()
     assert err <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), (prefix_len, n_tok, outliers, err)
+    if reconstruct:   # the two paths compute the same values (fp32, up to rounding order)
+        other = ctx.prefill_attention(torch.from_numpy(opool).cuda(), tt, prefix_len, _bf16_tensor(qb),
+                                      _bf16_tensor(kb), _bf16_tensor(vb), SCALE, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        diff = (out32 - other).abs().max().item()
+        assert diff <= 2e-5 * max(1.0, other.abs().max().item()), diff
 
 
 # ------------------------------------------------------------------ failure paths (no GPU fault)
