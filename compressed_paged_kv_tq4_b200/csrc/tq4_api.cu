@@ -587,7 +587,8 @@ int prefill_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int32_
   return cuda_status(tq4::launch_prefill_tc(static_cast<const uint8_t*>(pool), num_pages, page_table,
                                             prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, out_dtype,
                                             workspace, ctx->signs, ctx->d_status, ctx->wait_polls,
-                                            ctx->withhold, static_cast<cudaStream_t>(stream), reconstruct));
+                                            ctx->withhold, static_cast<cudaStream_t>(stream), ctx->num_sms,
+                                            reconstruct));
 }
 
 }  // namespace

@@ -36,11 +36,21 @@ struct PrefillParams {
   const __half* pkrlo;
   const __half* pvr;
   const __half* pvrlo;
+  // KV segments per row block (1: none); with several, each segment's pair writes its
+  // partial rows ws_po [unit][4][256][256] and (m, l) ws_pml [unit][4][256], merged by
+  // the combine pass (unit = row block * n_seg + segment)
+  int n_seg;
+  float* ws_po;
+  float2* ws_pml;
 };
 
-// q' hi, q' lo, R k hi, R k lo, R v hi, R v lo
+constexpr int kPfMaxSegments = 3;
+
+// q' hi, q' lo, R k hi, R k lo, R v hi, R v lo, then room for the segment partials
 inline size_t prefill_workspace_bytes(int32_t n_tok) {
-  return size_t(n_tok) * (2 * kHq + 4 * kHkv) * kD * sizeof(__half);
+  const size_t pairs = (size_t(6) * n_tok + 255) / 256;
+  return size_t(n_tok) * (2 * kHq + 4 * kHkv) * kD * sizeof(__half) +
+         pairs * kPfMaxSegments * kHkv * 256 * (kD * sizeof(float) + sizeof(float2));
 }
 // the reconstructed prefix's K hi, K lo, V hi, V lo rows
 inline size_t prefill_prefix_rows_bytes(int32_t prefix_len) {

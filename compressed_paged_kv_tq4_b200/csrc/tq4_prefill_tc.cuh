@@ -233,12 +233,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
   const uint32_t rank = cluster_rank();
   const uint32_t peer = rank ^ 1u;
   const int h = blockIdx.y;
-  const int pair_row0 = (blockIdx.x >> 1) * (2 * kPfRows);
+  // pair unit u = row block rb, KV segment seg: segment seg of n_seg covers tiles
+  // [t0, t0 + n_tiles) of the row block's range (one segment: the whole range)
+  const int unit = int(blockIdx.x >> 1), rb = unit / p.n_seg, seg = unit % p.n_seg;
+  const int pair_row0 = rb * (2 * kPfRows);
   const int row0 = pair_row0 + int(rank) * kPfRows;
   const int m_total = 6 * p.n_tok;
   const int last_row = min(pair_row0 + 2 * kPfRows, m_total) - 1;   // the pair's last row
   const int kv_end = p.prefix_len + last_row / 6 + 1;
-  const int n_tiles = (kv_end + kPfTile - 1) / kPfTile;
+  const int n_all = (kv_end + kPfTile - 1) / kPfTile;
+  const int t0 = int(int64_t(seg) * n_all / p.n_seg);
+  const int n_tiles = int(int64_t(seg + 1) * n_all / p.n_seg) - t0;   // local tile j is tile t0 + j
   const bool exact = p.out_dtype == TQ4_DTYPE_F32;
 
   auto bar = [sbase](int i) -> uint32_t { return sbase + kPfBarOff + 8u * uint32_t(i); };
@@ -354,7 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       tc_fence_after();
       const float4* kn4 = reinterpret_cast<const float4*>(norms + b * 2 * kPfTile);   // K norm * log2(e)
       const float4* vn4 = kn4 + kPfTile / 4;                                          // V norm / 256
-      const int pos0 = j * kPfTile;
+      const int pos0 = (t0 + j) * kPfTile;
       uint32_t sr[2][32];
       tm_ld32(lane_addr + kTmS0 + 64 * b, sr[0]);
       tm_ld32(lane_addr + kTmS0 + 64 * b + 32, sr[1]);
@@ -451,7 +456,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     const bool ok = __all_sync(0xffffffffu, misc[1] == 0) && warp_wait(bar(kBVEmpty + ((n_tiles - 1) & 1)), ((n_tiles - 1) >> 1) & 1);
     tc_fence_after();
     float* os = reinterpret_cast<float*>(smem) + r_local * kPfOsStride;
-    const float inv = (ok && l_sum > 0.f) ? (0.0625f / kPfPScale) / l_sum : 0.f;   // the scale of P and 1/16 of R^T
+    // one segment: o' / l with the scale of P and 1/16 of R^T; several: the raw partial,
+    // with (m, l) beside it for the combine pass
+    const bool split = p.n_seg > 1;
+    const float inv = split ? (ok ? 1.f : 0.f) : (ok && l_sum > 0.f) ? (0.0625f / kPfPScale) / l_sum : 0.f;
+    if (split && row_ok)
+      p.ws_pml[(int64_t(unit) * kHkv + h) * (2 * kPfRows) + int(rank) * kPfRows + r_local] =
+          make_float2(ok ? m_ref : -INFINITY, ok ? l_sum : 0.f);
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
       uint32_t ov[32];
@@ -503,10 +514,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     uint4 raw[4];
     float rawn = 0.f;
     auto page_of = [=](int j) -> int32_t {
-      return (j < n_tiles && j * kPfTile < prefix_end) ? __ldg(page_table + ((j * kPfTile) >> 8)) : 0;
+      return (j < n_tiles && (t0 + j) * kPfTile < prefix_end) ? __ldg(page_table + (((t0 + j) * kPfTile) >> 8)) : 0;
     };
-    auto fetch = [&raw, prefix_end, dense, pool, num_pages, h, status, &unit_pos, &unit_grp](int j, int u, int32_t page) {
-      const int pos = j * kPfTile + unit_pos(u);
+    auto fetch = [&raw, t0, prefix_end, dense, pool, num_pages, h, status, &unit_pos, &unit_grp](int j, int u,
+                                                                                             int32_t page) {
+      const int pos = (t0 + j) * kPfTile + unit_pos(u);
       raw[u] = make_uint4(0, 0, 0, 0);
       if (pos < prefix_end && !dense) {
         if (page >= 0 && page < num_pages) {
@@ -518,8 +530,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
         }
       }
     };
-    auto fetch_norm = [&rawn, gt, prefix_end, pool, num_pages, h](int j, int32_t page) {
-      const int pos = j * kPfTile + (gt & 63);
+    auto fetch_norm = [&rawn, t0, gt, prefix_end, pool, num_pages, h](int j, int32_t page) {
+      const int pos = (t0 + j) * kPfTile + (gt & 63);
       rawn = 0.f;
       if (pos < prefix_end && page >= 0 && page < num_pages)
         rawn = ldg_half(pool + int64_t(page) * kPageBytes + (gt < 64 ? kKNorms : kVNorms) +
@@ -529,7 +541,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     // position, asynchronous copies of the prologue's hi and lo rows for a chunk
     // position, zeros past the pair's last visible position
     auto expand = [&](int j, int u) {
-      const int pl = unit_pos(u), pos = j * kPfTile + pl;
+      const int pl = unit_pos(u), pos = (t0 + j) * kPfTile + pl;
       const int g = u < 2 ? kgrp : vgrp;   // word group within the panels of this CTA
       const int sw = pl & 7, c0 = (g & 1) * 4;
       const int prow = (u < 2 ? pl - int(rank) * kPfKPos : pl) * 128;
@@ -606,8 +618,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
       expand(j, 3);
       {
         const int pl = gt & 63;
-        const bool chunk = j * kPfTile + pl >= prefix_end && j * kPfTile + pl < kv_end;
-        const bool row = chunk || (dense && j * kPfTile + pl < prefix_end);
+        const int pos = (t0 + j) * kPfTile + pl;
+        const bool chunk = pos >= prefix_end && pos < kv_end;
+        const bool row = chunk || (dense && pos < prefix_end);
         const float n = row ? 1.f : rawn;   // dense rows (chunk or reconstructed) carry their own length
         if (gt < 64) {
           nb[pl] = n * kLog2e;
@@ -739,6 +752,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
     float v[8];
     const float4 a = *reinterpret_cast<const float4*>(os + rl * kPfOsStride + lane * 8);
     const float4 c = *reinterpret_cast<const float4*>(os + rl * kPfOsStride + lane * 8 + 4);
+    if (p.n_seg > 1) {   // the segment's partial row; the combine pass merges, rotates and stores
+      float* dst = p.ws_po + ((int64_t(unit) * kHkv + h) * (2 * kPfRows) + int(rank) * kPfRows + rl) * kD + lane * 8;
+      reinterpret_cast<float4*>(dst)[0] = a;
+      reinterpret_cast<float4*>(dst)[1] = c;
+      continue;
+    }
     v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
     v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
     warp_fwht256(v);
@@ -762,6 +781,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
   }
 }
 
+// Merge of a row's KV segments (several segments per row block): one warp per
+// (row, KV head): m = max m_s, o' = sum 2^(m_s - m) o'_s, l = sum 2^(m_s - m) l_s
+// (m in log2 units), then o = R^T (o' / l) with the scale of P, as the attention
+// kernel's own epilogue does with one segment.
+__global__ void __launch_bounds__(256) prefill_combine_kernel(const PrefillParams p) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int m_total = 6 * p.n_tok;
+  pdl_wait();
+  pdl_launch_dependents();
+  if (wid >= int64_t(m_total) * kHkv) return;
+  const int h = int(wid % kHkv), row = int(wid / kHkv);
+  const int rb = row / (2 * kPfRows), rr = row % (2 * kPfRows);
+  float M = -INFINITY;
+  for (int s = 0; s < p.n_seg; ++s)
+    M = fmaxf(M, p.ws_pml[(int64_t(rb * p.n_seg + s) * kHkv + h) * (2 * kPfRows) + rr].x);
+  float L = 0.f, o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < p.n_seg; ++s) {
+      const int64_t rec = (int64_t(rb * p.n_seg + s) * kHkv + h) * (2 * kPfRows) + rr;
+      const float2 ml = p.ws_pml[rec];
+      const float wgt = fast_exp2(ml.x - M);   // 0 for a segment that saw nothing of this row
+      L = fmaf(wgt, ml.y, L);
+      const float4* src = reinterpret_cast<const float4*>(p.ws_po + rec * kD + lane * 8);
+      const float4 a = src[0], c = src[1];
+      o[0] = fmaf(wgt, a.x, o[0]); o[1] = fmaf(wgt, a.y, o[1]); o[2] = fmaf(wgt, a.z, o[2]);
+      o[3] = fmaf(wgt, a.w, o[3]); o[4] = fmaf(wgt, c.x, o[4]); o[5] = fmaf(wgt, c.y, o[5]);
+      o[6] = fmaf(wgt, c.z, o[6]); o[7] = fmaf(wgt, c.w, o[7]);
+    }
+  }
+  warp_fwht256(o);
+  const float inv = (L > 0.f) ? (0.0625f / kPfPScale) / L : 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] *= inv * sign_of(p.signs, lane * 8 + i);
+  const int tok = row / 6, jh = row % 6;
+  const int64_t off = (int64_t(tok) * kHq + h * kGroup + jh) * kD + lane * 8;
+  if (p.out_dtype == TQ4_DTYPE_F32) {
+    float* dst = static_cast<float*>(p.out) + off;
+    reinterpret_cast<float4*>(dst)[0] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4*>(dst)[1] = make_float4(o[4], o[5], o[6], o[7]);
+  } else {
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+      pk[i] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+}
+
+// KV segments per row block: the fewest that fill the SMs' pair slots (one pair per
+// two SMs) to within a few percent over the waves the units take; several only when
+// every segment keeps at least 8 prefix tiles.
+inline int prefill_segments(int n_tok, int prefix_len, int num_sms) {
+  const int64_t pairs = int64_t((6 * n_tok + 2 * kPfRows - 1) / (2 * kPfRows)) * kHkv;
+  const int64_t slots = std::max(num_sms / 2, 1);
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= kPfMaxSegments; ++s) {
+    if (s > 1 && prefix_len < s * 8 * kPfTile) break;
+    const int64_t units = pairs * s;
+    const double eff = double(units) / double(((units + slots - 1) / slots) * slots) - 0.02 * (s - 1);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
 inline cudaError_t prefill_tc_set_attrs() {
   return cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPfSmem));
 }
@@ -772,7 +864,7 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
                                      int32_t prefix_len, const uint16_t* q, const uint16_t* kc,
                                      const uint16_t* vc, int32_t n_tok, float scale, void* out, int out_dtype,
                                      void* workspace, const Signs& signs, int* status, uint32_t spin_limit,
-                                     int test_withhold, cudaStream_t stream, bool reconstruct = false) {
+                                     int test_withhold, cudaStream_t stream, int num_sms, bool reconstruct = false) {
   __half* qr = static_cast<__half*>(workspace);
   __half* qlo = qr + size_t(n_tok) * kHq * kD;
   __half* kr = qlo + size_t(n_tok) * kHq * kD;
@@ -784,8 +876,13 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
                              n_tok, scale, qr, qlo, kr, krlo, vr, vrlo, signs);
   if (e != cudaSuccess) return e;
   PrefillParams p{};
-  if (reconstruct && prefix_len > 0) {   // rows after the chunk's: [prefix_len][4][256] each
-    __half* rows = vrlo + size_t(n_tok) * kHkv * kD;
+  // segment partials after the chunk's rows, then (with reconstruct) the prefix rows
+  const int64_t pairs = (6 * n_tok + 2 * kPfRows - 1) / (2 * kPfRows);
+  p.n_seg = prefill_segments(n_tok, prefix_len, num_sms);
+  p.ws_po = reinterpret_cast<float*>(vrlo + size_t(n_tok) * kHkv * kD);
+  p.ws_pml = reinterpret_cast<float2*>(p.ws_po + size_t(pairs) * kPfMaxSegments * kHkv * (2 * kPfRows) * kD);
+  if (reconstruct && prefix_len > 0) {   // rows after the partials: [prefix_len][4][256] each
+    __half* rows = reinterpret_cast<__half*>(p.ws_pml + size_t(pairs) * kPfMaxSegments * kHkv * (2 * kPfRows));
     const size_t n = size_t(prefix_len) * kHkv * kD;
     p.pkr = rows;
     p.pkrlo = rows + n;
@@ -813,8 +910,11 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
   p.status = status;
   p.spin_limit = spin_limit;
   p.test_withhold = test_withhold;
-  const unsigned pairs = unsigned((6 * n_tok + 2 * kPfRows - 1) / (2 * kPfRows));
-  return launch_pdl(prefill_tc_kernel, dim3(2 * pairs, kHkv), dim3(kPfThreads), size_t(kPfSmem), stream, p);
+  e = launch_pdl(prefill_tc_kernel, dim3(unsigned(2 * pairs * p.n_seg), kHkv), dim3(kPfThreads), size_t(kPfSmem),
+                 stream, p);
+  if (e != cudaSuccess || p.n_seg == 1) return e;
+  const int64_t warps = int64_t(6) * n_tok * kHkv;
+  return launch_pdl(prefill_combine_kernel, dim3(unsigned((warps + 7) / 8)), dim3(256), 0, stream, p);
 }
 
 }  // namespace tq4

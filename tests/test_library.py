@@ -74,7 +74,11 @@ def test_status_strings():
 def test_workspace_sizes_are_host_arithmetic():
     assert tq4.tq4_prefill_workspace_bytes(0) == 0
     # q' hi + lo ([n][24][256] f16 each) and the rotated chunk K, V as hi + lo ([n][4][256] f16 each)
-    assert tq4.tq4_prefill_workspace_bytes(2048) == 2048 * (2 * 24 + 4 * 4) * 256 * 2
+    # rotated q' and chunk rows (hi + lo f16), then room for up to 3 KV segments of
+    # partial rows per 256-row block and KV head: 256 x (256 fp32 + (m, l))
+    assert tq4.tq4_prefill_workspace_bytes(2048) == 2048 * (2 * 24 + 4 * 4) * 256 * 2 + 48 * 3 * 4 * 256 * (1024 + 8)
+    assert (tq4.tq4_prefill_reconstructed_workspace_bytes(32768, 2048)
+            == tq4.tq4_prefill_workspace_bytes(2048) + 32768 * 4 * 4 * 256 * 2)
     assert tq4.tq4_decode_workspace_bytes(None, 1, 1, 32768) == 0   # no context: no plan
 
 
