@@ -102,26 +102,43 @@ def workload_config(name, world):
 
 
 # ---------------------------------------------------------------------------- measured DRAM traffic
-# DRAM bytes (read + write) per launch of the dominant kernel, from one ncu capture
-# (summarised under profiles/), per unit of work. A figure counts only while the
-# kernel's source file hashes to the value it had when the counters were taken.
-MEASURED_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
+# ncu capture of that workload (summarised under profiles/). The figures count only
+# while the kernel sources hash to the value they had when the counters were taken.
+MEASURED_TRAFFIC_SOURCES = "1671b6d78773d5c15b7f864e51596ddf4d6f591a47920f515bb80698d3a5ce37"
+MEASURED_TRAFFIC = {
+    "decode_32k": 34_212_352,              # decode_q1_kernel: 34,181,632 read + 30,720 written
+    "decode_213k_outliers": 225_921_536,   # decode_q1_kernel: 221,920,256 + 4,001,280
+    "verify_2req_229k": 226_206_976,       # decode_splitk_kernel<3,3>: 221,701,120 + 4,505,856
+    "shared_prefix_8req_33k": 43_047_680,  # decode_splitk_kernel<1,6> (grouped): 42,840,320 + 207,360
+    "int8_decode_32k": 69_583_104,         # decode_splitk_kernel<1,1,INT8>: 67,694,848 + 1,888,256
+    "prefill_2k_on_32k": 204_666_112,      # prefill_tc_kernel: 101,673,984 + 102,992,128 (segment partials)
+}
 
 
-def measured_traffic(key, units):
-    """Bytes per launch for ``units`` units of work, or None if the kernel changed since the capture."""
-    if key not in MEASURED_TRAFFIC:
-        return None
+def sources_digest():
+    import glob
     import hashlib
-    fname, digest, per_unit = MEASURED_TRAFFIC[key]
-    path = os.path.join(ROOT, "compressed_paged_kv_tq4_b200", "csrc", fname)
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "compressed_paged_kv_tq4_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(csrc, "*.cuh")) + glob.glob(os.path.join(csrc, "*.cu"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic(workload):
+    """DRAM bytes per launch of the workload's dominant kernel, or None if the kernel
+    sources changed since the capture."""
+    if workload not in MEASURED_TRAFFIC:
+        return None
     try:
-        with open(path, "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != digest:
-                return None
+        if sources_digest() != MEASURED_TRAFFIC_SOURCES:
+            return None
     except OSError:
         return None
-    return per_unit * units
+    return MEASURED_TRAFFIC[workload]
 
 
 # ---------------------------------------------------------------------------- replicas (host side)
@@ -328,7 +345,7 @@ class DecodeSetup:
                   "tq4_decode_append_attention (split-K decode with the append inside it for one query token "
                   "+ combine)")
         return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": measured_traffic("decode_q1" if self.w.n_q == 1 else "decode_splitk", distinct),
+                "traffic": measured_traffic(self.w.name),
                 "kernel": kernel,
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms,
                 "peak_source": f"{peaks_[3]} hbm_gbs"}
@@ -403,7 +420,8 @@ class Int8DecodeSetup(DecodeSetup):
         nbytes = self.total * I.H_KV * 2 * 258
         ach = nbytes / (att_ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                "traffic": None, "kernel": "tq4_int8_encode_append + tq4_int8_decode_attention (split-K + combine)",
+                "traffic": measured_traffic(self.w.name),
+                "kernel": "tq4_int8_encode_append + tq4_int8_decode_attention (split-K + combine)",
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms, "peak_source": f"{peaks_[3]} hbm_gbs"}
 
 
@@ -495,7 +513,7 @@ class PrefillSetup:
         sus, burst = peaks_[2], peaks_[1]
         return {"bound": "tensor", "achieved": ach, "peak": sus, "unit": "TFLOP/s", "frac": ach / sus,
                 "frac_of_burst_peak": ach / burst, "peak_burst": burst,
-                "traffic": measured_traffic("prefill_tc", 1) if self.w.name == "prefill_2k_on_32k" else None,
+                "traffic": measured_traffic(self.w.name),
                 "kernel": "tq4_prefill_attention (rotate prologue + tcgen05 attention kernel)",
                 "algorithmic_flops_per_launch": flops, "launch_ms": att_ms,
                 "peak_source": f"{peaks_[3]} bf16_tflops_sustained (f16 operands: same nominal rate)"}
