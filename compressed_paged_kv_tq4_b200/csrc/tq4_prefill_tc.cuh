@@ -706,7 +706,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1) prefi
           }
           tc_fence_after();
           const volatile float* vm = reinterpret_cast<const volatile float*>(misc) + 8 + 2 * bp;
-          const bool vlo = exact || fmaxf(vm[0], vm[1]) > kVloNorm;
+          // reconstructed prefix rows carry each value's own f16 rounding (not one fixed
+          // residual per centroid), so that path takes the V lo product on every tile
+          const bool vlo = exact || p.pkr != nullptr || fmaxf(vm[0], vm[1]) > kVloNorm;
           const uint32_t vb = sbase + bp * kPfStage;
           const uint32_t p_t = tmem + kTmS0 + 64 * bp;
           const uint64_t vhi0 = tc_sdesc(vb + kPfVHi, kPfVPanel, 1024), vlo0 = tc_sdesc(vb + kPfVLo, kPfVPanel, 1024);

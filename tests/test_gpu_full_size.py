@@ -1,9 +1,11 @@
 """Parity at the workloads' full sizes, in the launch configuration bench.py times.
 
-Decode over 32,768 positions, over 212,992 positions with 5% x8 norms, and over
-two requests of 163,840 + 65,536 positions (4 causal query tokens each, 64 shared
-pages); prefill of 2,048 tokens on a 32,768-position prefix; the prefill's
-2,048-token append. For attention the pool is filled with seeded random codes and
+Decode over 32,768 positions, over 212,992 positions with 5% x8 norms, over two
+requests of 163,840 + 65,536 positions (4 causal query tokens each, 64 shared
+pages) and over eight one-token requests sharing 32,768 of their 33,792
+positions, the last two both ungrouped and grouped (shared pages read once);
+prefill of 2,048 tokens on a 32,768-position prefix, on the packed path and by
+direct inverse reconstruction; the prefill's 2,048-token append. For attention the pool is filled with seeded random codes and
 norms (every 4-bit value occurs; norms follow the workloads' scale mix), so both
 sides read the same bytes and the oracle needs no encoding pass. Decode outputs
 are compared in full (fp32 and bf16 outputs); prefill outputs on sampled chunk
@@ -47,7 +49,7 @@ def codebook():
     return O.codebook()
 
 
-@pytest.mark.parametrize("name", ["decode_32k", "decode_213k_outliers", "verify_2req_229k"])
+@pytest.mark.parametrize("name", ["decode_32k", "decode_213k_outliers", "verify_2req_229k", "shared_prefix_8req_33k"])
 def test_decode_full_size(codebook, name):
     c, _ = codebook
     w = I.WORKLOADS[name]
@@ -67,9 +69,21 @@ def test_decode_full_size(codebook, name):
     g32 = got32.cpu().numpy().astype(np.float64)
     assert np.abs(g32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), name
     H.assert_bf16_close(got16.float().cpu().numpy(), exp, name)
+    if w.shared_prefix_pages:   # the grouped decode: every request led by request 0
+        leader, pages = [0] * w.n_req, [w.shared_prefix_pages] * w.n_req
+        sh32 = ctx.decode_attention_shared(dpool, q, dtab, dseq, int(seq.sum()), SCALE, leader, pages,
+                                           out_dtype=torch.float32)
+        sh16 = ctx.decode_attention_shared(dpool, q, dtab, dseq, int(seq.sum()), SCALE, leader, pages,
+                                           out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        assert ctx.status() == tq4.TQ4_OK
+        s32 = sh32.cpu().numpy().astype(np.float64)
+        assert np.abs(s32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), name + " grouped"
+        H.assert_bf16_close(sh16.float().cpu().numpy(), exp, name + " grouped")
 
 
-def test_prefill_full_size(codebook):
+@pytest.mark.parametrize("reconstruct", [False, True])
+def test_prefill_full_size(codebook, reconstruct):
     c, _ = codebook
     w = I.WORKLOADS["prefill_2k_on_32k"]
     signs = I.signs(w.config)
@@ -79,12 +93,12 @@ def test_prefill_full_size(codebook):
     qb = I.queries(w.config, 0, (w.n_q, 24, 256))
     kb, vb = I.chunk_kv(w.config, 0, w.n_q)
     out = ctx.prefill_attention(torch.from_numpy(pool).cuda(), torch.from_numpy(tab).cuda(), w.prefix_len,
-                                _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE)
+                                _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE, reconstruct=reconstruct)
     torch.cuda.synchronize()
     assert ctx.status() == tq4.TQ4_OK
     out32 = ctx.prefill_attention(torch.from_numpy(pool).cuda(), torch.from_numpy(tab).cuda(), w.prefix_len,
                                   _bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE,
-                                  out_dtype=torch.float32)
+                                  out_dtype=torch.float32, reconstruct=reconstruct)
     torch.cuda.synchronize()
     assert ctx.status() == tq4.TQ4_OK
     # 64 chunk tokens: first and last, both sides of every 256-row CTA pair boundary, and a seeded draw
