@@ -325,6 +325,18 @@ class DecodeSetup:
     def alt_name(self):   # the path not timed as the workload's
         return "ungrouped (tq4_decode_append_attention)" if self.shared else "grouped (tq4_decode_attention_shared)"
 
+    def alternatives(self):
+        """The workload's other paths on the same inputs: (name, enter, leave)."""
+        alts = []
+        if self.n_q > 1 and not self.shared:   # 2-4 tokens: the tensor-memory kernel beside the default one
+            tq4 = self.tq4
+            alts.append(("tcgen05 tensor-memory split-K kernel (decode path TQ4_DECODE_PATH_TENSOR_MEMORY)",
+                         lambda: self.ctx.set_decode_path(tq4.DECODE_PATH_TENSOR_MEMORY),
+                         lambda: self.ctx.set_decode_path(tq4.DECODE_PATH_WARP_MMA)))
+        if self.has_groups:
+            alts.append((self.alt_name(), self.flip, self.flip))
+        return alts
+
     def units_per_step(self):
         return self.total * self.w.layers  # attended KV positions x layers
 
@@ -397,6 +409,9 @@ class Int8DecodeSetup(DecodeSetup):
         torch.cuda.synchronize()
         if self.ctx.status() != tq4.TQ4_OK:
             raise RuntimeError("INT8 cache build failed")
+
+    def alternatives(self):   # the INT8 arm has one kernel path
+        return []
 
     def attend(self, layer):
         """The step's append and decode of one layer: two calls on the INT8 arm."""
@@ -482,6 +497,9 @@ class PrefillSetup:
         return ("packed prefix (tq4_prefill_attention)" if self.reconstruct else
                 "direct inverse reconstruction (tq4_prefill_attention_reconstructed: dense prefix rows, then "
                 "the same attention kernel)")
+
+    def alternatives(self):
+        return [(self.alt_name(), self.flip, self.flip)]
 
     def append(self, layer):
         tq4, w = self.tq4, self.w
@@ -707,8 +725,9 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
     torch.cuda.synchronize()
     att_ms = ev0.elapsed_time(ev1) / (reps * w.layers)
     res["roofline"] = S.roofline(att_ms, peaks())
-    if getattr(S, "has_alt", False):   # the workload's other path on the same inputs, timed the same way
-        S.flip()
+    others = []
+    for name, enter, leave in (S.alternatives() if hasattr(S, "alternatives") else []):
+        enter()   # the workload's other path on the same inputs, timed the same way
         g3 = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
             torch.cuda.synchronize()
@@ -723,8 +742,12 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
             ev1.record(stream)
         torch.cuda.synchronize()
         del g3
-        S.flip()
-        res["roofline"]["other_path"] = {"path": S.alt_name(), "launch_ms": ev0.elapsed_time(ev1) / (reps * w.layers)}
+        leave()
+        others.append({"path": name, "launch_ms": ev0.elapsed_time(ev1) / (reps * w.layers)})
+    if others:
+        res["roofline"]["other_path"] = others[0]
+        if len(others) > 1:
+            res["roofline"]["other_paths"] = others
 
     # end to end through the public API: pinned host inputs in, every layer's output out, each step
     h2d, d2h = S.h2d_d2h()

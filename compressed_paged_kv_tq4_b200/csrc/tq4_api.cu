@@ -16,6 +16,7 @@
 #include "tq4_decode_q1.cuh"
 #include "tq4_prefill.cuh"
 #include "tq4_prefill_tc.cuh"
+#include "tq4_decode_tc.cuh"
 
 struct tq4_ctx {
   int device;
@@ -27,6 +28,7 @@ struct tq4_ctx {
   uint32_t wait_polls;   // bounded device waits give up after this many polls
   int withhold;          // test hook: kernels withhold one producer signal (see tq4_ctx_set_wait_limit)
   void* noalloc_scratch; // device address of the library's fixed split-K array on this device
+  int decode_path;       // TQ4_DECODE_PATH_*: which kernel decodes 2-4 query tokens
 };
 
 namespace {
@@ -86,6 +88,27 @@ cudaError_t set_decode_attrs() {
     e = cudaFuncSetAttribute(tq4::decode_splitk_kernel<NT, NTG, kI8, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, int(tq4::decode_smem_bytes<NT, NTG, kI8>()));
   return e;
+}
+
+template <int NT>
+cudaError_t set_decode_tc_attrs() {
+  cudaError_t e = cudaFuncSetAttribute(tq4::decode_tc_kernel<NT, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(tq4::kDtSmem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(tq4::decode_tc_kernel<NT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(tq4::kDtSmem));
+  return e;
+}
+// the tensor-memory decode of 2-4 query tokens (n-tiles 2 or 3)
+cudaError_t launch_decode_tc(int nt, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  const bool exact = p.out_dtype == TQ4_DTYPE_F32;
+  const dim3 block(tq4::kDtThreads);
+  const size_t smem = tq4::kDtSmem;
+  if (nt == 2)
+    return exact ? tq4::launch_pdl(tq4::decode_tc_kernel<2, true>, grid, block, smem, st, p)
+                 : tq4::launch_pdl(tq4::decode_tc_kernel<2, false>, grid, block, smem, st, p);
+  return exact ? tq4::launch_pdl(tq4::decode_tc_kernel<3, true>, grid, block, smem, st, p)
+               : tq4::launch_pdl(tq4::decode_tc_kernel<3, false>, grid, block, smem, st, p);
 }
 
 // one split-K decode launch with the output precision chosen at run time
@@ -291,6 +314,7 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   if (!ctx) return TQ4_ERR_ARG;
   ctx->signs = sb;
   ctx->wait_polls = TQ4_DEFAULT_WAIT_POLLS;
+  ctx->decode_path = TQ4_DECODE_PATH_WARP_MMA;
   // the fp64 Lloyd-Max solution is the codebook: encode compares against its
   // midpoints (rounded to fp32), reconstruction reads the centroids rounded to
   // fp32, and the attention kernels read each centroid as an f16 hi + lo pair
@@ -323,6 +347,8 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   if (e == cudaSuccess) e = set_decode_attrs<2, 2, true>();
   if (e == cudaSuccess) e = set_decode_attrs<3, 3, true>();
   if (e == cudaSuccess) e = tq4::prefill_tc_set_attrs();
+  if (e == cudaSuccess) e = set_decode_tc_attrs<2>();
+  if (e == cudaSuccess) e = set_decode_tc_attrs<3>();
   if (e == cudaSuccess) e = cudaGetSymbolAddress(&ctx->noalloc_scratch, g_noalloc_scratch);
   if (e == cudaSuccess && !ctx->noalloc_scratch) e = cudaErrorInvalidSymbol;
   if (e == cudaSuccess) e = cudaMalloc(&ctx->d_status, sizeof(int));
@@ -348,6 +374,12 @@ int tq4_ctx_set_wait_limit(tq4_ctx* ctx, uint32_t polls, int withhold_signal) {
   if (!ctx) return TQ4_ERR_ARG;
   ctx->wait_polls = polls ? polls : TQ4_DEFAULT_WAIT_POLLS;
   ctx->withhold = withhold_signal ? 1 : 0;
+  return TQ4_OK;
+}
+
+int tq4_ctx_set_decode_path(tq4_ctx* ctx, int path) {
+  if (!ctx || (path != TQ4_DECODE_PATH_TENSOR_MEMORY && path != TQ4_DECODE_PATH_WARP_MMA)) return TQ4_ERR_ARG;
+  ctx->decode_path = path;
   return TQ4_OK;
 }
 
@@ -493,7 +525,10 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
                               tq4::decode_q1_smem_bytes(), st, p, map);
         break;
       }
-      default: e = launch_splitk_nt<false>(tq4::decode_nt(n_q), false, grid, st, p); break;
+      default:
+        e = ctx->decode_path == TQ4_DECODE_PATH_TENSOR_MEMORY ? launch_decode_tc(tq4::decode_nt(n_q), grid, st, p)
+                                                             : launch_splitk_nt<false>(tq4::decode_nt(n_q), false, grid, st, p);
+        break;
     }
   }
   if (e != cudaSuccess) return TQ4_ERR_CUDA;

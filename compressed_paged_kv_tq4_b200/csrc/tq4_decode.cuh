@@ -727,6 +727,42 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem
   }
 }
 
+// Warp-collective (one warp; lane 0 writes): the description of private item x
+// of the grid (items [0, share.n_gitems) are group items) in s_item, with
+// kItNMem = 0 when x is no item. Records TQ4_ERR_SEQ when the device lengths make
+// more items than the grid holds.
+__device__ __forceinline__ void describe_private_item(const DecodeParams& p, int x, int h, int* s_item) {
+  const int lane = threadIdx.x & 31;
+  int req = 0, sp = 0, total = 0;
+  const bool ok = find_item(p, x - p.share.n_gitems, req, sp, total);
+  int first = 0, P = 0, nsh = 0, own = 0;
+  if (ok) {
+    first = request_first_record(p, req);
+    P = shared_pos(p, req);
+    request_records(p, req, __ldg(p.seq_lens + req), nsh, own);
+  }
+  if (lane == 0) {
+    s_item[kItNMem] = ok ? 1 : 0;
+    s_item[kItReq] = req;
+    s_item[kItRec] = first + nsh + sp;
+    s_item[kItTable] = req;
+    s_item[kItPosB] = P + sp * p.split_len;
+    s_item[kItPosE] = min(P + (sp + 1) * p.split_len, ok ? __ldg(p.seq_lens + req) : 0);
+    if (x == p.share.n_gitems && h == 0 && p.share.n_gitems + total > p.items_ub)
+      record_error(p.status, TQ4_ERR_SEQ);
+  }
+}
+// (one thread) every record the item writes must lie inside the workspace; an
+// item that would write outside it records TQ4_ERR_SEQ and is dropped
+__device__ __forceinline__ void check_item_records(const DecodeParams& p, int* s_item) {
+  bool in = true;
+  for (int k = 0; k < s_item[kItNMem]; ++k) in = in && s_item[kItRec + k] < p.records_ub;
+  if (!in) {
+    record_error(p.status, TQ4_ERR_SEQ);
+    s_item[kItNMem] = 0;
+  }
+}
+
 // Split-K decode: grid (items, 4 KV heads). Items [0, share.n_gitems) are group
 // items (NTG n-tiles), the rest the requests' own items (NT n-tiles).
 template <int NT, int NTG, bool kI8, bool kExact>
@@ -761,34 +797,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
         s_item[kItNMem] = nm;
       }
     } else {       // request req, split sp of its own positions
-      int req = 0, sp = 0, total = 0;
-      const bool ok = find_item(p, x - p.share.n_gitems, req, sp, total);
-      int first = 0, P = 0, nsh = 0, own = 0;
-      if (ok) {
-        first = request_first_record(p, req);
-        P = shared_pos(p, req);
-        request_records(p, req, __ldg(p.seq_lens + req), nsh, own);
-      }
-      if (lane == 0) {
-        s_item[kItNMem] = ok ? 1 : 0;
-        s_item[kItReq] = req;
-        s_item[kItRec] = first + nsh + sp;
-        s_item[kItTable] = req;
-        s_item[kItPosB] = P + sp * p.split_len;
-        s_item[kItPosE] = min(P + (sp + 1) * p.split_len, ok ? __ldg(p.seq_lens + req) : 0);
-        if (x == p.share.n_gitems && h == 0 && p.share.n_gitems + total > p.items_ub)
-          record_error(p.status, TQ4_ERR_SEQ);
-      }
+      describe_private_item(p, x, h, s_item);
     }
   }
-  if (w == 0 && lane == 0) {   // every record this item writes must lie inside the workspace
-    bool in = true;
-    for (int k = 0; k < s_item[kItNMem]; ++k) in = in && s_item[kItRec + k] < p.records_ub;
-    if (!in) {
-      record_error(p.status, TQ4_ERR_SEQ);
-      s_item[kItNMem] = 0;
-    }
-  }
+  if (w == 0 && lane == 0) check_item_records(p, s_item);
   __syncthreads();
   if (s_item[kItNMem] == 0 || x >= p.items_ub) return;
   if constexpr (NTG != NT) {

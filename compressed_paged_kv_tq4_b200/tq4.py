@@ -39,6 +39,9 @@ INT8_POSITION_BYTES = 2064
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
 
+DECODE_PATH_TENSOR_MEMORY = 0   # tcgen05 kernel for 2-4 query tokens
+DECODE_PATH_WARP_MMA = 1        # warp-level mma.sync kernel (default)
+
 EXPORTS = (
     "tq4_ctx_create", "tq4_ctx_destroy", "tq4_codebook", "tq4_encode_append", "tq4_reconstruct",
     "tq4_decode_workspace_bytes", "tq4_decode_attention", "tq4_prefill_workspace_bytes",
@@ -46,6 +49,7 @@ EXPORTS = (
     "tq4_decode_append_attention", "tq4_ctx_set_wait_limit", "tq4_int8_encode_append", "tq4_int8_decode_attention",
     "tq4_decode_shared_workspace_bytes", "tq4_decode_attention_shared",
     "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
+    "tq4_ctx_set_decode_path",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -83,6 +87,7 @@ _sig = {
     "tq4_prefill_attention": ([_p, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p, ctypes.c_int, _p, _sz,
                                _p], ctypes.c_int),
     "tq4_ctx_set_wait_limit": ([_p, ctypes.c_uint32, ctypes.c_int], ctypes.c_int),
+    "tq4_ctx_set_decode_path": ([_p, ctypes.c_int], ctypes.c_int),
     "tq4_int8_encode_append": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p], ctypes.c_int),
     "tq4_int8_decode_attention": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int,
                                    _p, _sz, _p], ctypes.c_int),
@@ -266,6 +271,10 @@ def tq4_ctx_set_wait_limit(ctx, polls, withhold_signal=0) -> int:
     return _lib.tq4_ctx_set_wait_limit(ctx, polls, withhold_signal)
 
 
+def tq4_ctx_set_decode_path(ctx, path) -> int:
+    return _lib.tq4_ctx_set_decode_path(ctx, path)
+
+
 def tq4_decode_attention_noalloc(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
                                  total_seq_len, scale, out, out_dtype, stream=None) -> int:
     """Decode attention whose split-K scratch is the library's fixed device array
@@ -415,6 +424,10 @@ class Context:
         """Polls a bounded device wait makes before it gives up (0 = the default);
         withhold_signal makes later calls withhold one producer signal (testing)."""
         _check(tq4_ctx_set_wait_limit(self.handle, polls, int(withhold_signal)), "tq4_ctx_set_wait_limit")
+
+    def set_decode_path(self, path: int) -> None:
+        """Kernel for 2-4 query tokens: DECODE_PATH_TENSOR_MEMORY or DECODE_PATH_WARP_MMA (default)."""
+        _check(tq4_ctx_set_decode_path(self.handle, path), "tq4_ctx_set_decode_path")
 
     # -- pool helpers
     @staticmethod

@@ -265,13 +265,30 @@ int tq4_prefill_attention_reconstructed(tq4_ctx* ctx, const void* pool, int32_t 
  *   withhold_signal  nonzero: later calls withhold one producer signal so that
  *                    a wait is sure to run out (the one-token decode kernel
  *                    does not issue the copy of each warp's first tile; the
- *                    prefill kernel does not signal the tensor-core issuer that
- *                    P of tile min(1, tiles - 1) is ready); their results are
+ *                    tensor-memory decode of 2-4 tokens does not signal the
+ *                    tensor-core issuer that the first key chunk is ready; the
+ *                    prefill kernel does not signal it that P of tile
+ *                    min(1, tiles - 1) is ready); their results are
  *                    then undefined and the status is TQ4_ERR_TIMEOUT. 0 (the
  *                    default) restores normal operation.
  * Returns TQ4_ERR_ARG for a NULL context. */
 #define TQ4_DEFAULT_WAIT_POLLS (1u << 24)
 int tq4_ctx_set_wait_limit(tq4_ctx* ctx, uint32_t polls, int withhold_signal);
+
+/* Which kernel decodes requests of 2 to 4 query tokens (the tq4_decode_attention
+ * family, without shared-prefix groups; the arithmetic is the same, see
+ * tq4_decode_attention):
+ *   TQ4_DECODE_PATH_TENSOR_MEMORY  tcgen05 MMAs with tensor-memory
+ *        accumulators: tile positions are the MMA's rows, the keys are expanded
+ *        into tensor memory and the values into shared memory;
+ *   TQ4_DECODE_PATH_WARP_MMA       (default) the warp-level mma.sync kernel that
+ *        also serves one-token groups, shared-prefix groups and the INT8 arm.
+ * The two give the same results up to fp32 summation order. The choice holds
+ * for later calls on the context.
+ * Returns TQ4_ERR_ARG for a NULL context or an unknown path. */
+#define TQ4_DECODE_PATH_TENSOR_MEMORY 0
+#define TQ4_DECODE_PATH_WARP_MMA      1
+int tq4_ctx_set_decode_path(tq4_ctx* ctx, int path);
 
 /* Decode attention for callers that cannot allocate device memory.
  * The pages have no counterpart to this call; it exists for the library's users.

@@ -94,5 +94,6 @@ def test_argument_errors_return_before_any_launch():
     assert lib.tq4_prefill_attention(None, None, 0, None, 0, 0, None, None, None, 1, 0.0625, None, 1, None, 0,
                                      None) == E
     assert lib.tq4_ctx_set_wait_limit(None, 4, 0) == E
+    assert lib.tq4_ctx_set_decode_path(None, 0) == E
     assert lib.tq4_reconstruct(None, None, 0, None, 0, 0, 1, None, None, None) == E
     assert lib.tq4_get_status(None, None) == E
