@@ -57,6 +57,8 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="launch without a CUDA graph (profiling)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (profiling only)")
+    ap.add_argument("--decode-path", default="default", choices=["default", "warp", "tensor"],
+                    help="kernel for 2-4 query tokens (tq4_ctx_set_decode_path); default: the library's")
     ap.add_argument("--profile", action="store_true",
                     help="eager steps of the one workload only: no roofline replay, e2e or CPU leg (ncu captures)")
     return ap.parse_args(argv)
@@ -662,6 +664,8 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
         import dataclasses
         w = dataclasses.replace(w, layers=args.layers)
     S = {"decode": DecodeSetup, "decode_int8": Int8DecodeSetup, "prefill": PrefillSetup}[w.kind](w, torch, tq4, device)
+    if args.decode_path != "default":
+        S.ctx.set_decode_path(tq4.DECODE_PATH_WARP_MMA if args.decode_path == "warp" else tq4.DECODE_PATH_TENSOR_MEMORY)
     stream = torch.cuda.Stream(device)
     graph = None
     with torch.cuda.stream(stream):
