@@ -107,14 +107,14 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
 # ncu capture of that workload (summarised under profiles/). The figures count only
 # while the kernel sources hash to the value they had when the counters were taken.
-MEASURED_TRAFFIC_SOURCES = "1671b6d78773d5c15b7f864e51596ddf4d6f591a47920f515bb80698d3a5ce37"
+MEASURED_TRAFFIC_SOURCES = "38f42d63ea1a05e90a569162c85af6919e200690f40e6cc1c0d7b44ca5ed3b7b"
 MEASURED_TRAFFIC = {
-    "decode_32k": 34_212_352,              # decode_q1_kernel: 34,181,632 read + 30,720 written
-    "decode_213k_outliers": 225_921_536,   # decode_q1_kernel: 221,920,256 + 4,001,280
-    "verify_2req_229k": 226_206_976,       # decode_splitk_kernel<3,3>: 221,701,120 + 4,505,856
-    "shared_prefix_8req_33k": 43_047_680,  # decode_splitk_kernel<1,6> (grouped): 42,840,320 + 207,360
-    "int8_decode_32k": 69_583_104,         # decode_splitk_kernel<1,1,INT8>: 67,694,848 + 1,888,256
-    "prefill_2k_on_32k": 204_666_112,      # prefill_tc_kernel: 101,673,984 + 102,992,128 (segment partials)
+    "decode_32k": 34_221_056,              # decode_q1_kernel: 34,184,192 read + 36,864 written
+    "decode_213k_outliers": 225_458_944,   # decode_q1_kernel: 221,923,840 + 3,535,104
+    "verify_2req_229k": 224_921_088,       # decode_splitk_kernel<3,3>: 221,703,680 + 3,217,408
+    "shared_prefix_8req_33k": 43_076_864,  # decode_splitk_kernel<1,6> (grouped): 42,842,880 + 233,984
+    "int8_decode_32k": 68_667_136,         # decode_splitk_kernel<1,1,INT8>: 67,694,336 + 972,800
+    "prefill_2k_on_32k": 202_866_688,      # prefill_tc_kernel: 101,581,824 + 101,284,864 (segment partials)
 }
 
 
