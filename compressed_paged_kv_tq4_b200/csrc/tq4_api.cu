@@ -29,6 +29,8 @@ struct tq4_ctx {
   int withhold;          // test hook: kernels withhold one producer signal (see tq4_ctx_set_wait_limit)
   void* noalloc_scratch; // device address of the library's fixed split-K array on this device
   int decode_path;       // TQ4_DECODE_PATH_*: which kernel decodes 2-4 query tokens
+  double centroids_b[2][8];   // the 2- and 3-bit variants' fp64 codebooks (4 and 8 levels)
+  double boundaries_b[2][7];
 };
 
 namespace {
@@ -42,25 +44,26 @@ namespace {
 // ---------------------------------------------------------------------------
 double std_normal_pdf(double z) { return std::isinf(z) ? 0.0 : std::exp(-0.5 * z * z) / std::sqrt(2.0 * M_PI); }
 
-void lloyd_max_16(double sigma, double c[16], double b[15]) {
-  for (int j = 0; j < 16; ++j) c[j] = sigma * (-2.5 + 5.0 * j / 15.0);
+void lloyd_max_levels(int levels, double sigma, double* c, double* b) {
+  for (int j = 0; j < levels; ++j) c[j] = sigma * (-2.5 + 5.0 * j / double(levels - 1));
   for (int it = 0; it < 200000; ++it) {
-    for (int j = 0; j < 15; ++j) b[j] = 0.5 * (c[j] + c[j + 1]);
+    for (int j = 0; j + 1 < levels; ++j) b[j] = 0.5 * (c[j] + c[j + 1]);
     double moved = 0.0;
     double cn[16];
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < levels; ++j) {
       const double lo = j == 0 ? -INFINITY : b[j - 1] / sigma;
-      const double hi = j == 15 ? INFINITY : b[j] / sigma;
+      const double hi = j == levels - 1 ? INFINITY : b[j] / sigma;
       // P(lo < Z < hi) = (erfc(lo/sqrt2) - erfc(hi/sqrt2)) / 2
       const double mass = 0.5 * (std::erfc(lo / M_SQRT2) - std::erfc(hi / M_SQRT2));
       cn[j] = sigma * (std_normal_pdf(lo) - std_normal_pdf(hi)) / mass;
       moved = std::fmax(moved, std::fabs(cn[j] - c[j]));
     }
-    std::memcpy(c, cn, sizeof(cn));
+    std::memcpy(c, cn, sizeof(double) * levels);
     if (moved < 1e-19) break;
   }
-  for (int j = 0; j < 15; ++j) b[j] = 0.5 * (c[j] + c[j + 1]);
+  for (int j = 0; j + 1 < levels; ++j) b[j] = 0.5 * (c[j] + c[j + 1]);
 }
+void lloyd_max_16(double sigma, double c[16], double b[15]) { lloyd_max_levels(16, sigma, c, b); }
 
 uint16_t half_bits(double x) {
   const __half h = __double2half(x);
@@ -109,6 +112,43 @@ cudaError_t launch_decode_tc(int nt, dim3 grid, cudaStream_t st, const tq4::Deco
                  : tq4::launch_pdl(tq4::decode_tc_kernel<2, false>, grid, block, smem, st, p);
   return exact ? tq4::launch_pdl(tq4::decode_tc_kernel<3, true>, grid, block, smem, st, p)
                : tq4::launch_pdl(tq4::decode_tc_kernel<3, false>, grid, block, smem, st, p);
+}
+
+template <int kBits>
+cudaError_t set_decode_bits_attrs() {
+  cudaError_t e = cudaSuccess;
+  auto set = [&e](auto kernel, size_t bytes) {
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
+  };
+  set(tq4::decode_bits_kernel<1, false, kBits>, tq4::decode_item_smem_bytes<1, false, kBits>());
+  set(tq4::decode_bits_kernel<1, true, kBits>, tq4::decode_item_smem_bytes<1, false, kBits>());
+  set(tq4::decode_bits_kernel<2, false, kBits>, tq4::decode_item_smem_bytes<2, false, kBits>());
+  set(tq4::decode_bits_kernel<2, true, kBits>, tq4::decode_item_smem_bytes<2, false, kBits>());
+  set(tq4::decode_bits_kernel<3, false, kBits>, tq4::decode_item_smem_bytes<3, false, kBits>());
+  set(tq4::decode_bits_kernel<3, true, kBits>, tq4::decode_item_smem_bytes<3, false, kBits>());
+  return e;
+}
+template <int NT, int kBits>
+cudaError_t launch_bits_nt(dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  const size_t smem = tq4::decode_item_smem_bytes<NT, false, kBits>();
+  if (p.out_dtype == TQ4_DTYPE_F32)
+    return tq4::launch_pdl(tq4::decode_bits_kernel<NT, true, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
+  return tq4::launch_pdl(tq4::decode_bits_kernel<NT, false, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
+}
+// a 2- or 3-bit pool's split-K decode
+cudaError_t launch_decode_bits(int bits, int nt, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  if (bits == 2) {
+    switch (nt) {
+      case 1: return launch_bits_nt<1, 2>(grid, st, p);
+      case 2: return launch_bits_nt<2, 2>(grid, st, p);
+      default: return launch_bits_nt<3, 2>(grid, st, p);
+    }
+  }
+  switch (nt) {
+    case 1: return launch_bits_nt<1, 3>(grid, st, p);
+    case 2: return launch_bits_nt<2, 3>(grid, st, p);
+    default: return launch_bits_nt<3, 3>(grid, st, p);
+  }
 }
 
 // one split-K decode launch with the output precision chosen at run time
@@ -328,9 +368,25 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
     cb.r16[j] = half_bits(ctx->centroids[j] - double(__half2float(hh)));
   }
   for (int j = 0; j < 15; ++j) cb.b[j] = float(ctx->boundaries[j]);
+  tq4::CodebookB cbb[2]{};   // the 2- and 3-bit variants, stored the same way
+  for (int v = 0; v < 2; ++v) {
+    const int levels = 4 << v;
+    lloyd_max_levels(levels, 1.0 / 16.0, ctx->centroids_b[v], ctx->boundaries_b[v]);
+    for (int j = 0; j < levels; ++j) {
+      cbb[v].c[j] = float(ctx->centroids_b[v][j]);
+      cbb[v].c16[j] = half_bits(ctx->centroids_b[v][j]);
+      __half hh;
+      std::memcpy(&hh, &cbb[v].c16[j], 2);
+      cbb[v].r16[j] = half_bits(ctx->centroids_b[v][j] - double(__half2float(hh)));
+    }
+    for (int j = 0; j + 1 < levels; ++j) cbb[v].b[j] = float(ctx->boundaries_b[v][j]);
+  }
   cudaError_t e = cudaGetDevice(&ctx->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, ctx->device);
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(tq4::g_codebook, &cb, sizeof(cb));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(tq4::g_codebook_b, cbb, sizeof(cbb));
+  if (e == cudaSuccess) e = set_decode_bits_attrs<2>();
+  if (e == cudaSuccess) e = set_decode_bits_attrs<3>();
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(tq4::decode_q1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              int(tq4::decode_q1_smem_bytes()));
@@ -449,7 +505,7 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
                 int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q, int64_t total_seq_len,
                 float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream,
                 const AppendArgs* app, bool int8 = false, const int32_t* prefix_leader = nullptr,
-                const int32_t* prefix_pages = nullptr) {
+                const int32_t* prefix_pages = nullptr, int bits = 4) {
   if (!ctx || n_req < 0) return TQ4_ERR_ARG;
   if (n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS) return TQ4_ERR_UNSUPPORTED;
   if (n_req == 0) return TQ4_OK;
@@ -508,7 +564,9 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
     if (e != cudaSuccess) return TQ4_ERR_CUDA;
   }
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
-  if (int8) {
+  if (bits != 4) {
+    e = launch_decode_bits(bits, tq4::decode_nt(n_q), grid, st, p);
+  } else if (int8) {
     e = launch_splitk_nt<true>(tq4::decode_nt(n_q), false, grid, st, p);
   } else if (groups) {     // group items and the requests' own items in one launch
     e = launch_splitk_nt<false>(tq4::decode_nt(n_q), true, grid, st, p);
@@ -591,6 +649,42 @@ int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                               int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
   return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
                      out, out_dtype, workspace, workspace_bytes, stream, nullptr, true);
+}
+
+int tq4_tqb_codebook(const tq4_ctx* ctx, int bits, double* centroids, double* boundaries) {
+  if (!ctx || !centroids || !boundaries || (bits != 2 && bits != 3)) return TQ4_ERR_ARG;
+  const int v = bits - 2, levels = 4 << v;
+  std::memcpy(centroids, ctx->centroids_b[v], sizeof(double) * levels);
+  std::memcpy(boundaries, ctx->boundaries_b[v], sizeof(double) * (levels - 1));
+  return TQ4_OK;
+}
+
+int tq4_tqb_encode_append(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages, const int32_t* page_table,
+                          int32_t table_len, int32_t start_pos, int32_t n_tok, const void* k_new, const void* v_new,
+                          int dtype, void* stream) {
+  if (!ctx || n_tok < 0 || start_pos < 0) return TQ4_ERR_ARG;
+  if (bits != 2 && bits != 3) return TQ4_ERR_UNSUPPORTED;
+  if (n_tok == 0) return TQ4_OK;
+  if (!pool || !page_table || !k_new || !v_new || num_pages <= 0 || table_len <= 0) return TQ4_ERR_ARG;
+  if (dtype != TQ4_DTYPE_F32 && dtype != TQ4_DTYPE_BF16) return TQ4_ERR_ARG;
+  if ((int64_t(start_pos) + n_tok + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
+  if (!aligned(pool, 16) || !aligned(k_new, 16) || !aligned(v_new, 16)) return TQ4_ERR_ARG;
+  if (int rc = check_device(ctx)) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto* pl = static_cast<uint8_t*>(pool);
+  return cuda_status(bits == 2 ? tq4::launch_encode_bits<2>(pl, num_pages, page_table, start_pos, n_tok, k_new, v_new,
+                                                            dtype, ctx->signs, ctx->d_status, st)
+                               : tq4::launch_encode_bits<3>(pl, num_pages, page_table, start_pos, n_tok, k_new, v_new,
+                                                            dtype, ctx->signs, ctx->d_status, st));
+}
+
+int tq4_tqb_decode_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t num_pages, const uint16_t* q,
+                             const int32_t* page_tables, int32_t max_pages, const int32_t* seq_lens, int32_t n_req,
+                             int32_t n_q, int64_t total_seq_len, float scale, void* out, int out_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  if (bits != 2 && bits != 3) return ctx ? TQ4_ERR_UNSUPPORTED : TQ4_ERR_ARG;
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, nullptr, false, nullptr, nullptr, bits);
 }
 
 size_t tq4_prefill_workspace_bytes(int32_t n_tok) {

@@ -113,9 +113,19 @@ __host__ __device__ constexpr int decode_nt(int n_q) { return (6 * n_q + 7) / 8;
 // ring stages: three, two for the wide group items (shared memory)
 template <int NT, bool kI8>
 constexpr int decode_stages() { return kI8 ? kI8Stages : (NT >= 4 ? 2 : kStages); }
-template <int NT, bool kI8>
+// 2- and 3-bit pools: a chunk's rows are staged as they are in the page (K and V
+// packed words, then K and V norms) and widened to the four-bit stage layout in
+// one work stage
+template <int kBits>
+constexpr size_t tqb_raw_stage_bytes() { return size_t(2) * kChunk * tqb_row_bytes<kBits>() + size_t(2) * kChunk * 2; }
+template <int NT, bool kI8, int kBits>
+constexpr size_t decode_ring_bytes() {
+  return kBits != 4 ? size_t(decode_stages<NT, kI8>()) * tqb_raw_stage_bytes<kBits>() + kStageBytes
+                    : size_t(decode_stages<NT, kI8>()) * (kI8 ? kI8StageBytes : kStageBytes);
+}
+template <int NT, bool kI8, int kBits = 4>
 constexpr size_t decode_item_smem_bytes() {
-  return (kI8 ? size_t(kI8Stages) * kI8StageBytes : size_t(kLutBytes) + size_t(decode_stages<NT, kI8>()) * kStageBytes) +
+  return (kI8 ? 0 : size_t(kLutBytes)) + decode_ring_bytes<NT, kI8, kBits>() +
          2 * size_t(8 * NT) * kQvStride * 2 + 2 * size_t(8 * NT) * kPsStride * 2 + size_t(kDecWarps) * 8 * NT * 4;
 }
 template <int NT, int NTG, bool kI8>
@@ -124,6 +134,7 @@ constexpr size_t decode_smem_bytes() {
                                                                                 : decode_item_smem_bytes<NTG, kI8>();
 }
 static_assert(decode_item_smem_bytes<kShareNT, false>() <= 227u * 1024u, "group items fit shared memory");
+static_assert(decode_item_smem_bytes<3, false, 3>() <= 227u * 1024u, "3-bit items fit shared memory");
 
 __device__ __forceinline__ int warp_incl_scan(int v) {
   const int lane = threadIdx.x & 31;
@@ -251,14 +262,19 @@ constexpr int kItPosB = 0, kItPosE = 1, kItTable = 2, kItNMem = 3, kItReq = 4,
 // table, scored against the query rows of item[kItNMem] requests (request
 // item[kItReq + k], partial record item[kItRec + k]); NT n-tiles hold their
 // n_mem * 6 * n_q rows (member-major, then token, then head).
-template <int NT, bool kI8, bool kExact>   // kExact: fp32 outputs, C_lo P' on every chunk (see kVloNorm)
+// kExact: fp32 outputs, C_lo P' on every chunk (see kVloNorm). kBits: 4 (TQ4), or 2
+// or 3 for the narrower variants, whose codes are widened to nibbles per chunk.
+template <int NT, bool kI8, bool kExact, int kBits = 4>
 __device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem, const int* item) {
+  static_assert(kBits == 4 || (!kI8 && (kBits == 2 || kBits == 3)), "bit width");
+  constexpr bool kTQB = kBits != 4;
   constexpr int kRB = kI8 ? 256 : 128;                 // bytes of one staged K or V row
   constexpr int kNS = decode_stages<NT, kI8>();        // ring stages; chunks prefetched kNS - 1 ahead
-  constexpr int kSB = kI8 ? kI8StageBytes : kStageBytes;
+  constexpr int kSB = kTQB ? int(tqb_raw_stage_bytes<kBits>()) : (kI8 ? kI8StageBytes : kStageBytes);
   const uint32_t lut = smem_u32(smem);                 // the centroid table (TQ4 only)
   uint8_t* ring = smem + (kI8 ? 0 : kLutBytes);
-  __half* qv_hi = reinterpret_cast<__half*>(ring + kNS * kSB);
+  uint8_t* work = ring + kNS * kSB;                    // the widened chunk (2- and 3-bit pools)
+  __half* qv_hi = reinterpret_cast<__half*>(smem + (kI8 ? 0 : kLutBytes) + decode_ring_bytes<NT, kI8, kBits>());
   __half* qv_lo = qv_hi + 8 * NT * kQvStride;
   __half* ps_hi = qv_lo + 8 * NT * kQvStride;
   __half* ps_lo = ps_hi + 8 * NT * kPsStride;   // P' = hi + lo, both f16
@@ -283,6 +299,24 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem
       const int32_t page = __ldg(table + (c >> 8));
       if (page < 0 || page >= p.num_pages) {
         if (tid == 0) record_error(p.status, TQ4_ERR_PAGE_RANGE);
+      } else if constexpr (kTQB) {
+        constexpr int kRBb = tqb_row_bytes<kBits>(), kSegB = kRBb / 16;
+        const uint8_t* pg = p.pool + int64_t(page) * tqb_page_bytes<kBits>();
+        const int64_t slot0 = head_slot0 + (c & (kPage - 1));
+        uint8_t* st = ring + (i % kNS) * kSB;
+        const int nvalid = min(kChunk, pos_e - c);
+        for (int e = tid; e < 2 * kChunk * kSegB; e += kDecThreads) {
+          const int kv = e / (kChunk * kSegB), pl = (e / kSegB) % kChunk, sg = e % kSegB;
+          if (pl < nvalid)
+            cp_async16(smem_u32(st + (kv * kChunk + pl) * kRBb + sg * 16),
+                       pg + (kv ? tqb_v_words<kBits>() : 0) + (slot0 + pl) * kRBb + sg * 16);
+        }
+        if (tid < 2 * (kChunk / 8)) {
+          const int kv = tid / (kChunk / 8), sg = tid % (kChunk / 8);
+          if (sg * 8 < nvalid)
+            cp_async16(smem_u32(st + 2 * kChunk * kRBb + kv * kChunk * 2 + sg * 16),
+                       pg + (kv ? tqb_v_norms<kBits>() : tqb_k_norms<kBits>()) + (slot0 + sg * 8) * 2);
+        }
       } else {
         constexpr int64_t kPB = kI8 ? kI8PageBytes : kPageBytes;
         constexpr int64_t kKR = kI8 ? kI8KCodes : kKWords, kVR = kI8 ? kI8VCodes : kVWords;
@@ -365,7 +399,8 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem
   }
   // centroid table: row b holds each lane's 8-byte slot {c16 pair, r16 pair} at +8*lane
   if constexpr (!kI8)
-    for (int e = tid; e < 256 * 32; e += kDecThreads) reinterpret_cast<uint2*>(smem)[e] = lut_row(e >> 5);
+    for (int e = tid; e < 256 * 32; e += kDecThreads)
+      reinterpret_cast<uint2*>(smem)[e] = kTQB ? lut_row_bits<kBits>(e >> 5) : lut_row(e >> 5);
   __syncthreads();
 
   // ---- B fragments of Q' (hi, lo) for the K phase, in registers when they fit
@@ -411,6 +446,28 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem
     issue_chunk(i + kNS - 1);
     const int c = pos_b + i * kChunk;
     const uint8_t* st = ring + (i % kNS) * kSB;
+    if constexpr (kTQB) {
+      // widen the staged chunk into the four-bit layout: thread -> (K or V, position,
+      // 16-byte segment of four nibble words = dims 32 sg .. 32 sg + 31)
+      constexpr int kRBb = tqb_row_bytes<kBits>();
+      for (int e = tid; e < 2 * kChunk * 8; e += kDecThreads) {
+        const int kv = e / (kChunk * 8), pl = (e >> 3) % kChunk, sg = e & 7;
+        const uint8_t* r = st + (kv * kChunk + pl) * kRBb;
+        const uint2 lo = lds64(r + sg * 8);                    // plane 0: words 2 sg, 2 sg + 1
+        const uint32_t hb = kBits == 3 ? lds32(r + 64 + sg * 4) : 0u;   // plane 1: word sg
+        uint4 o;
+        o.x = widen2(lo.x) | (widen1(hb) << 2);
+        o.y = widen2(lo.x >> 16) | (widen1(hb >> 8) << 2);
+        o.z = widen2(lo.y) | (widen1(hb >> 16) << 2);
+        o.w = widen2(lo.y >> 16) | (widen1(hb >> 24) << 2);
+        *reinterpret_cast<uint4*>(work + (kv * kChunk + pl) * 128 + ((sg ^ seg_swz(pl)) << 4)) = o;
+      }
+      if (tid < 2 * kChunk * 2 / 16)   // the norms, unchanged
+        reinterpret_cast<uint4*>(work + 2 * kChunk * 128)[tid] =
+            reinterpret_cast<const uint4*>(st + 2 * kChunk * kRBb)[tid];
+      __syncthreads();
+      st = work;
+    }
     const uint8_t* kst = st;
     const uint8_t* vst = st + kChunk * kRB;
     const __half* knr = reinterpret_cast<const __half*>(st + 2 * kChunk * kRB);
@@ -810,6 +867,24 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
     }
   }
   decode_item<NT, kI8, kExact>(p, smem, s_item);
+}
+
+// Split-K decode over a 2- or 3-bit pool: grid (items, 4 KV heads), the requests'
+// own items only (no shared-prefix groups).
+template <int NT, bool kExact, int kBits>
+__global__ void __launch_bounds__(kDecThreads, 1) decode_bits_kernel(const DecodeParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int s_item[kItWords];
+  const int w = threadIdx.x >> 5;
+  const int h = blockIdx.y;
+  const int x = int(blockIdx.x);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (w == 0) describe_private_item(p, x, h, s_item);
+  if (threadIdx.x == 0) check_item_records(p, s_item);
+  __syncthreads();
+  if (s_item[kItNMem] == 0 || x >= p.items_ub) return;
+  decode_item<NT, false, kExact, kBits>(p, smem, s_item);
 }
 
 // One CTA of 8 warps per output row (request, token, query head). Warp w

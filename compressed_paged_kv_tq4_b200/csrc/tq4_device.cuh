@@ -41,6 +41,16 @@ struct Codebook {
 };
 __constant__ Codebook g_codebook;  // one translation unit (tq4_api.cu) includes every kernel header
 
+// Codebooks of the 2- and 3-bit variants (entry 0: 4 levels, entry 1: 8 levels),
+// written by the host from its fp64 Lloyd-Max solutions like the 16-level one.
+struct CodebookB {
+  float c[8];         // centroids rounded to fp32
+  float b[7];         // decision boundaries (fp64 midpoints, rounded to fp32)
+  uint16_t c16[8];    // f16 bits of the centroids
+  uint16_t r16[8];    // f16 bits of the rounding residuals
+};
+__constant__ CodebookB g_codebook_b[2];
+
 // 256 sign bits: bit i set <=> s_i = -1. Passed by value to kernels.
 struct Signs {
   uint32_t bits[8];
@@ -136,6 +146,49 @@ __device__ __forceinline__ void lut_decode(uint32_t lut_s, uint32_t w, uint32_t 
 __device__ __forceinline__ uint2 lut_row(int b) {
   return make_uint2(uint32_t(g_codebook.c16[b & 15]) | (uint32_t(g_codebook.c16[b >> 4]) << 16),
                     uint32_t(g_codebook.r16[b & 15]) | (uint32_t(g_codebook.r16[b >> 4]) << 16));
+}
+
+// The same slot for a 2- or 3-bit pool whose codes have been widened to nibbles
+// (an index never exceeds 2^kBits - 1).
+template <int kBits>
+__device__ __forceinline__ uint2 lut_row_bits(int b) {
+  const CodebookB& cb = g_codebook_b[kBits - 2];
+  constexpr int m = (1 << kBits) - 1;
+  return make_uint2(uint32_t(cb.c16[b & m]) | (uint32_t(cb.c16[(b >> 4) & m]) << 16),
+                    uint32_t(cb.r16[b & m]) | (uint32_t(cb.r16[(b >> 4) & m]) << 16));
+}
+
+// Page layout of the 2- and 3-bit variants: per 256-dim vector 8 kBits u32 words
+// (plane 0: the low two bits of every index, coordinate 16w + i in bits 2i..2i+1 of
+// word w; plane 1, 3 bits only: bit 2, coordinate 32w + i in bit i of word 16 + w)
+// plus one fp16 norm; per page K words [4][256][8 kBits], V words, K norms [4][256],
+// V norms.
+template <int kBits>
+constexpr int tqb_row_bytes() { return 32 * kBits; }
+template <int kBits>
+constexpr int64_t tqb_page_bytes() { return int64_t(2) * kHkv * kPage * (tqb_row_bytes<kBits>() + 2); }
+template <int kBits>
+constexpr int64_t tqb_v_words() { return int64_t(kHkv) * kPage * tqb_row_bytes<kBits>(); }
+template <int kBits>
+constexpr int64_t tqb_k_norms() { return 2 * tqb_v_words<kBits>(); }
+template <int kBits>
+constexpr int64_t tqb_v_norms() { return tqb_k_norms<kBits>() + int64_t(kHkv) * kPage * 2; }
+static_assert(tqb_page_bytes<2>() == TQ4_TQB2_PAGE_BYTES && tqb_page_bytes<3>() == TQ4_TQB3_PAGE_BYTES,
+              "page sizes of the header");
+
+// Widen 8 two-bit fields (bits 2i..2i+1 of x) to the low bits of 8 nibbles, and 8
+// single bits (bit i of h) to bit 0 of 8 nibbles.
+__device__ __forceinline__ uint32_t widen2(uint32_t x) {
+  x &= 0xFFFFu;
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  return (x | (x << 2)) & 0x33333333u;
+}
+__device__ __forceinline__ uint32_t widen1(uint32_t h) {
+  h &= 0xFFu;
+  h = (h | (h << 12)) & 0x000F000Fu;
+  h = (h | (h << 6)) & 0x03030303u;
+  return (h | (h << 3)) & 0x11111111u;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

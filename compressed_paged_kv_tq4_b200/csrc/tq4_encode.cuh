@@ -224,7 +224,85 @@ __global__ void __launch_bounds__(256) int8_encode_kernel(
   if (lane == 0) reinterpret_cast<__half*>(base + (kv ? kVS : kKS))[slot] = __double2half(sc);
 }
 
+// The 2- and 3-bit variants: the four-bit encode with a 2^kBits-level codebook
+// (g_codebook_b) and the bit-plane packing of tqb_row_bytes: lane l's indices of
+// coordinates 8l .. 8l + 7 give the 16 low bits (plane 0) of word l / 2 and the 8
+// bits at 8 (l & 3) of plane-1 word 16 + l / 4. One warp per vector.
+template <typename T, int kBits>
+__global__ void __launch_bounds__(256) encode_bits_kernel(
+    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table, int32_t start_pos,
+    int32_t n_tok, const T* __restrict__ k_new, const T* __restrict__ v_new, Signs signs, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (vec >= int64_t(n_tok) * 2 * kHkv) return;
+  const int tok = int(vec / (2 * kHkv));
+  const int kv = int(vec / kHkv) & 1;
+  const int head = int(vec % kHkv);
+  float x[8];
+  load8<T>((kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8, x);
+  const CodebookB& cb = g_codebook_b[kBits - 2];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+  const float n = sqrtf(ss);
+  uint32_t lo16 = 0, hi8 = 0;
+  if (n > 0.f) {
+    const uint32_t sb = lane_sign_bits(signs);
+    float y[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[i] = apply_sign(x[i] / n, sb, i);
+    warp_fwht256(y);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float yi = y[i] * 0.0625f;
+      uint32_t idx = 0;
+#pragma unroll
+      for (int j = 0; j < (1 << kBits) - 1; ++j) idx += (yi > cb.b[j]) ? 1u : 0u;
+      lo16 |= (idx & 3u) << (2 * i);
+      hi8 |= ((idx >> 2) & 1u) << i;
+    }
+  }
+  // plane 0: word w = lanes 2w (low half) and 2w + 1; plane 1: word w = lanes 4w .. 4w + 3
+  const uint32_t w0 = lo16 | (__shfl_down_sync(0xffffffffu, lo16, 1) << 16);
+  uint32_t w1 = hi8 << (8 * (lane & 3));
+  w1 |= __shfl_xor_sync(0xffffffffu, w1, 1);
+  w1 |= __shfl_xor_sync(0xffffffffu, w1, 2);
+  const int32_t pos = start_pos + tok;
+  const int32_t page = __ldg(page_table + (pos >> 8));
+  if (page < 0 || page >= num_pages) {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+    return;
+  }
+  const int slot = head * kPage + (pos & (kPage - 1));
+  uint8_t* base = pool + int64_t(page) * tqb_page_bytes<kBits>();
+  uint32_t* words = reinterpret_cast<uint32_t*>(base + (kv ? tqb_v_words<kBits>() : 0) +
+                                                int64_t(slot) * tqb_row_bytes<kBits>());
+  if ((lane & 1) == 0) words[lane >> 1] = w0;
+  if (kBits == 3 && (lane & 3) == 0) words[16 + (lane >> 2)] = w1;
+  if (lane == 0)
+    reinterpret_cast<__half*>(base + (kv ? tqb_v_norms<kBits>() : tqb_k_norms<kBits>()))[slot] = __float2half_rn(n);
+}
+
 // ---------------------------------------------------------------- launchers
+template <int kBits>
+cudaError_t launch_encode_bits(uint8_t* pool, int32_t num_pages, const int32_t* page_table, int32_t start_pos,
+                               int32_t n_tok, const void* k_new, const void* v_new, int dtype, const Signs& signs,
+                               int* status, cudaStream_t stream) {
+  const int threads = 256, wpb = threads / 32;
+  const unsigned blocks = unsigned((int64_t(n_tok) * 2 * kHkv + wpb - 1) / wpb);
+  if (dtype == TQ4_DTYPE_F32)
+    return launch_pdl(encode_bits_kernel<float, kBits>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                      page_table, start_pos, n_tok, static_cast<const float*>(k_new),
+                      static_cast<const float*>(v_new), signs, status);
+  return launch_pdl(encode_bits_kernel<uint16_t, kBits>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+                    page_table, start_pos, n_tok, static_cast<const uint16_t*>(k_new),
+                    static_cast<const uint16_t*>(v_new), signs, status);
+}
+
 cudaError_t launch_int8_encode_append(uint8_t* pool, int32_t num_pages, const int32_t* page_table,
                                       int32_t start_pos, int32_t n_tok, const void* k_new, const void* v_new,
                                       int dtype, int* status, cudaStream_t stream) {

@@ -34,6 +34,7 @@ Q_HEADS = 24
 PAGE_BYTES = 266240
 POSITION_BYTES = 1040
 INT8_PAGE_BYTES = 528384
+TQB_PAGE_BYTES = {2: 135168, 3: 200704}   # the 2- and 3-bit variants
 INT8_POSITION_BYTES = 2064
 
 DTYPE_F32 = 0
@@ -49,7 +50,7 @@ EXPORTS = (
     "tq4_decode_append_attention", "tq4_ctx_set_wait_limit", "tq4_int8_encode_append", "tq4_int8_decode_attention",
     "tq4_decode_shared_workspace_bytes", "tq4_decode_attention_shared",
     "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
-    "tq4_ctx_set_decode_path",
+    "tq4_ctx_set_decode_path", "tq4_tqb_codebook", "tq4_tqb_encode_append", "tq4_tqb_decode_attention",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -88,6 +89,11 @@ _sig = {
                                _p], ctypes.c_int),
     "tq4_ctx_set_wait_limit": ([_p, ctypes.c_uint32, ctypes.c_int], ctypes.c_int),
     "tq4_ctx_set_decode_path": ([_p, ctypes.c_int], ctypes.c_int),
+    "tq4_tqb_codebook": ([_p, ctypes.c_int, _p, _p], ctypes.c_int),
+    "tq4_tqb_encode_append": ([_p, ctypes.c_int, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p],
+                              ctypes.c_int),
+    "tq4_tqb_decode_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p,
+                                  ctypes.c_int, _p, _sz, _p], ctypes.c_int),
     "tq4_int8_encode_append": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p], ctypes.c_int),
     "tq4_int8_decode_attention": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int,
                                    _p, _sz, _p], ctypes.c_int),
@@ -265,6 +271,27 @@ def tq4_int8_decode_attention(ctx, pool, num_pages, q, page_tables, max_pages, s
     return _lib.tq4_int8_decode_attention(ctx, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
                                           _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out),
                                           out_dtype, _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_tqb_codebook(ctx: int, bits: int):
+    c = (ctypes.c_double * 8)()
+    b = (ctypes.c_double * 7)()
+    _check(_lib.tq4_tqb_codebook(ctx, bits, ctypes.cast(c, _p), ctypes.cast(b, _p)), "tq4_tqb_codebook")
+    levels = 1 << bits
+    return list(c)[:levels], list(b)[:levels - 1]
+
+
+def tq4_tqb_encode_append(ctx, bits, pool, num_pages, page_table, table_len, start_pos, n_tok, k_new, v_new,
+                          dtype, stream=None) -> int:
+    return _lib.tq4_tqb_encode_append(ctx, bits, _ptr(pool), num_pages, _ptr(page_table), table_len, start_pos,
+                                      n_tok, _ptr(k_new), _ptr(v_new), dtype, _stream(stream))
+
+
+def tq4_tqb_decode_attention(ctx, bits, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q,
+                             total_seq_len, scale, out, out_dtype, workspace, workspace_bytes, stream=None) -> int:
+    return _lib.tq4_tqb_decode_attention(ctx, bits, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
+                                         _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out), out_dtype,
+                                         _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def tq4_ctx_set_wait_limit(ctx, polls, withhold_signal=0) -> int:
@@ -556,6 +583,40 @@ class Context:
         _check(tq4_int8_decode_attention(self.handle, pool, pool.numel() // INT8_PAGE_BYTES, q, page_tables,
                                          page_tables.shape[1], seq_lens, n_req, n_q, total_seq_len, scale, out,
                                          od, workspace, workspace.numel(), stream), "tq4_int8_decode_attention")
+        return out
+
+    # -- the 2- and 3-bit variants
+    @staticmethod
+    def new_tqb_pool(bits: int, num_pages: int, device="cuda") -> torch.Tensor:
+        return torch.zeros(num_pages * TQB_PAGE_BYTES[bits], dtype=torch.uint8, device=device)
+
+    def tqb_codebook(self, bits: int):
+        return tq4_tqb_codebook(self.handle, bits)
+
+    def tqb_encode_append(self, bits, pool, page_table, start_pos, k_new, v_new, stream=None):
+        _need_cuda(pool, page_table, k_new, v_new)
+        dtype = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(k_new.dtype)
+        if dtype is None or v_new.dtype != k_new.dtype:
+            raise ValueError("k_new/v_new must both be float32 or bfloat16")
+        _check(tq4_tqb_encode_append(self.handle, bits, pool, pool.numel() // TQB_PAGE_BYTES[bits], page_table,
+                                     page_table.numel(), start_pos, k_new.shape[0], k_new, v_new, dtype, stream),
+               "tq4_tqb_encode_append")
+
+    def tqb_decode_attention(self, bits, pool, q, page_tables, seq_lens, total_seq_len, scale, out=None,
+                             out_dtype=torch.bfloat16, workspace=None, stream=None):
+        _need_cuda(pool, q, page_tables, seq_lens)
+        if q.dtype != torch.bfloat16:
+            raise ValueError("q must be bfloat16")
+        n_req, n_q = q.shape[0], q.shape[1]
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        if workspace is None:
+            workspace = self.decode_workspace(n_req, n_q, total_seq_len, q.device)
+        _check(tq4_tqb_decode_attention(self.handle, bits, pool, pool.numel() // TQB_PAGE_BYTES[bits], q,
+                                        page_tables, page_tables.shape[1], seq_lens, n_req, n_q, total_seq_len,
+                                        scale, out, od, workspace, workspace.numel(), stream),
+               "tq4_tqb_decode_attention")
         return out
 
     def prefill_attention(self, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,

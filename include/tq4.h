@@ -88,6 +88,8 @@ extern "C" {
 #define TQ4_MAX_QUERY_TOKENS 4
 #define TQ4_INT8_POSITION_BYTES 2064      /* INT8 arm: 4 heads x (K+V) x (256 + 2) B    */
 #define TQ4_INT8_PAGE_BYTES     528384    /* INT8 arm: 256 layer-positions             */
+#define TQ4_TQB2_PAGE_BYTES     135168    /* 2-bit variant: 256 x 528 B                */
+#define TQ4_TQB3_PAGE_BYTES     200704    /* 3-bit variant: 256 x 784 B                */
 
 #define TQ4_DTYPE_F32   0
 #define TQ4_DTYPE_BF16  1
@@ -349,6 +351,36 @@ int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
                               int64_t total_seq_len, float scale,
                               void* out, int out_dtype,
                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* The 2- and 3-bit variants of the format. The pages describe the four-bit
+ * encoding only ([KVEXEC] simpleprog.com, "Fitting a 27B-Parameter LLM into
+ * 24 GiB of Laptop Memory", section "KVExec"); this library's reading keeps every
+ * step of it (norm, rotation R = H diag(s) / 16, nearest-centroid quantiser with
+ * ties low, fp16 norm, rotated-domain attention) with b = bits per coordinate and
+ * a 2^b-level Lloyd-Max codebook for N(0, 1/256) computed in fp64 by the library.
+ * Per 256-dim vector: 8 b u32 words and one fp16 norm. Plane 0, words 0..15: the
+ * low two bits of every index, coordinate 16w + i in bits 2i..2i+1 of word w;
+ * plane 1 (b = 3 only), words 16..23: bit 2, coordinate 32w + i in bit i of word
+ * 16 + w. A pool is num_pages pages of TQ4_TQB2_PAGE_BYTES (b = 2) or
+ * TQ4_TQB3_PAGE_BYTES (b = 3) bytes:
+ *   [0, 4*256*32b)          K words [4 heads][256 slots][8b u32]
+ *   [.., 2*4*256*32b)       V words (same shape)
+ *   then K norms [4][256] fp16, then V norms [4][256] fp16.
+ * Page tables, lengths, queries, outputs, workspaces (tq4_decode_workspace_bytes)
+ * and errors are as for the four-bit calls of the same shape; bits other than 2
+ * and 3 return TQ4_ERR_UNSUPPORTED.
+ * tq4_tqb_codebook copies the fp64 centroids (2^b) and boundaries (2^b - 1). */
+int tq4_tqb_codebook(const tq4_ctx* ctx, int bits, double* centroids, double* boundaries);
+int tq4_tqb_encode_append(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
+                          const int32_t* page_table, int32_t table_len,
+                          int32_t start_pos, int32_t n_tok,
+                          const void* k_new, const void* v_new, int dtype, void* stream);
+int tq4_tqb_decode_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t num_pages,
+                             const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                             const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                             int64_t total_seq_len, float scale,
+                             void* out, int out_dtype,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise the stream, return the first device-side error recorded since
  * the last call (TQ4_OK if none) and clear it. */

@@ -1,0 +1,161 @@
+"""GPU parity of the 2- and 3-bit variants against their fp64 oracle
+(oracle/tqb_oracle.py), through the C ABI: the library's codebooks equal the
+oracle's; the encode is bit-exact apart from coordinates within 1e-6 of a decision
+boundary (the GPU rotates in fp32); decode attention meets the bf16 tolerance on the
+GPU-encoded pool and 1e-4 (fp32 output) on the oracle's own pool bytes, for one to
+four query tokens, ragged lengths, shared pages, outliers and a 32,768-position
+history."""
+import numpy as np
+import pytest
+
+from compressed_paged_kv_tq4_b200 import inputs as I
+from oracle import tqb_oracle as OB
+import _helpers as H
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+from compressed_paged_kv_tq4_b200 import tq4  # noqa: E402
+
+SCALE = 1.0 / 16.0
+
+
+def _bf16_tensor(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_tqb_codebook_matches_oracle(bits):
+    ctx = tq4.Context(I.signs(0))
+    c, b = ctx.tqb_codebook(bits)
+    oc, ob = OB.codebook(bits)
+    assert np.max(np.abs(np.array(c) - oc)) < 1e-15
+    assert np.max(np.abs(np.array(b) - ob)) < 1e-15
+
+
+def _pool_regions(pool_bytes, bits):
+    return OB._regions(np.ascontiguousarray(pool_bytes), bits)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_tqb_encode_bit_exact(bits, dtype):
+    signs = I.signs(0)
+    ctx = tq4.Context(signs)
+    c, b = OB.codebook(bits)
+    table = I.page_table_scattered(41, 5, 7)
+    k, v = I.kv_vectors(41, 0, 1200, outlier_frac=0.05)
+    k[17] = 0.0                                        # a zero vector
+    if dtype == "bf16":
+        kb, vb = I.to_bf16_bits(k), I.to_bf16_bits(v)
+        k, v = I.bf16_bits_to_f32(kb), I.bf16_bits_to_f32(vb)
+        kt, vt = _bf16_tensor(kb), _bf16_tensor(vb)
+    else:
+        kt, vt = torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda()
+    pool = tq4.Context.new_tqb_pool(bits, 7)
+    tt = torch.from_numpy(table).cuda()
+    for a, e in ((0, 333), (333, 1000), (1000, 1200)):   # appends that start mid-page
+        ctx.tqb_encode_append(bits, pool, tt, a, kt[a:e], vt[a:e])
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    opool = OB.new_pool(7, bits)
+    yk, yv = OB.encode_append(opool, table, 0, k, v, signs, c, bits)
+    g = _pool_regions(pool.cpu().numpy(), bits)
+    o = _pool_regions(opool, bits)
+    pos = np.arange(1200)
+    pg, sl = table[pos // 256], pos % 256
+    exempt = 0
+    for gw, ow, y, what in ((g[0], o[0], yk, "K"), (g[1], o[1], yv, "V")):
+        gi = OB.unpack_indices(gw[pg, :, sl], bits).astype(np.int64)
+        oi = OB.unpack_indices(ow[pg, :, sl], bits).astype(np.int64)
+        diff = gi != oi
+        if diff.any():
+            dist = np.min(np.abs(np.asarray(y)[diff][:, None] - b[None, :]), axis=1)
+            ok = (dist < H.BOUNDARY_EXEMPT) & (np.abs(gi[diff] - oi[diff]) == 1)
+            assert ok.all(), f"{what}: {int((~ok).sum())} indices differ away from a boundary"
+            exempt += int(diff.sum())
+        # every word bit outside the differing indices is identical: repack the oracle's
+        # indices with the GPU's exempt ones and compare the words
+        fixed = np.where(diff, gi, oi).astype(np.uint8)
+        assert np.array_equal(OB.pack_indices(fixed, bits), gw[pg, :, sl])
+    assert exempt <= 20
+    H.check_norms_against_oracle(g[2][pg, :, sl], o[2][pg, :, sl], k, "K norms")
+    H.check_norms_against_oracle(g[3][pg, :, sl], o[3][pg, :, sl], v, "V norms")
+
+
+class TqbCase:
+    def __init__(self, bits, config, seq_lens, n_q, shared_pages=0, outliers=0.05):
+        self.bits = bits
+        self.signs = I.signs(config)
+        self.ctx = tq4.Context(self.signs)
+        self.c, _ = OB.codebook(bits)
+        npg = [(s + 255) // 256 for s in seq_lens]
+        total = npg[0] + sum(n - shared_pages for n in npg[1:]) + 2
+        ids = I.page_table_scattered(config, total, total)
+        tab = np.full((len(seq_lens), max(npg)), -1, np.int32)
+        tab[0, :npg[0]] = ids[:npg[0]]
+        off = npg[0]
+        for r in range(1, len(seq_lens)):
+            tab[r, :shared_pages] = tab[0, :shared_pages]
+            f = npg[r] - shared_pages
+            tab[r, shared_pages:npg[r]] = ids[off:off + f]
+            off += f
+        self.tab, self.n_q = tab, n_q
+        self.seq = np.array(seq_lens, np.int32)
+        self.pool = tq4.Context.new_tqb_pool(bits, total)
+        self.opool = OB.new_pool(total, bits)
+        for r, s in enumerate(seq_lens):
+            first = shared_pages * 256 if r > 0 else 0
+            k, v = I.kv_vectors(config, 0, s - first, first_pos=first, request=r, outlier_frac=outliers)
+            self.ctx.tqb_encode_append(bits, self.pool, torch.from_numpy(tab[r]).cuda(), first,
+                                       torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+            OB.encode_append(self.opool, tab[r], first, k, v, self.signs, self.c, bits)
+        torch.cuda.synchronize()
+        assert self.ctx.status() == tq4.TQ4_OK
+
+    def decode(self, qb, pool, out_dtype):
+        out = self.ctx.tqb_decode_attention(self.bits, pool, _bf16_tensor(qb), torch.from_numpy(self.tab).cuda(),
+                                            torch.from_numpy(self.seq).cuda(), int(self.seq.sum()), SCALE,
+                                            out_dtype=out_dtype)
+        torch.cuda.synchronize()
+        assert self.ctx.status() == tq4.TQ4_OK
+        return out.float().cpu().numpy().astype(np.float64)
+
+    def oracle(self, qb):
+        return OB.decode_attention(self.opool, self.tab, self.seq, I.bf16_bits_to_f32(qb), SCALE, self.signs,
+                                   self.c, self.bits)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("seq_lens,n_q,shared", [
+    ([1], 1, 0), ([255], 1, 0), ([257], 1, 0), ([1000, 63, 2047], 1, 0), ([300], 2, 0),
+    ([513, 40], 3, 0), ([2048, 700], 4, 2), ([4], 4, 0), ([5000], 4, 0),
+])
+def test_tqb_decode_parity(bits, seq_lens, n_q, shared):
+    case = TqbCase(bits, 43, seq_lens, n_q, shared_pages=shared)
+    qb = I.queries(43, 1, (len(seq_lens), n_q, 24, 256))
+    exp = case.oracle(qb)
+    H.assert_bf16_close(case.decode(qb, case.pool, torch.bfloat16), exp, f"{bits}-bit decode {seq_lens} n_q={n_q}")
+    got32 = case.decode(qb, torch.from_numpy(case.opool).cuda(), torch.float32)
+    assert np.abs(got32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max())
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_tqb_decode_32k_history(bits):
+    """The decode_32k shape (one request, 32,768 positions, one query token)."""
+    case = TqbCase(bits, 44, [32768], 1, outliers=0.0)
+    qb = I.queries(44, 0, (1, 1, 24, 256))
+    exp = case.oracle(qb)
+    got32 = case.decode(qb, torch.from_numpy(case.opool).cuda(), torch.float32)
+    assert np.abs(got32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max())
+    H.assert_bf16_close(case.decode(qb, case.pool, torch.bfloat16), exp, f"{bits}-bit decode 32k")
+
+
+def test_tqb_argument_checks():
+    ctx = tq4.Context(I.signs(0))
+    assert tq4.tq4_tqb_encode_append(ctx.handle, 4, None, 1, None, 1, 0, 1, None, None, 1) == tq4.TQ4_ERR_UNSUPPORTED
+    assert tq4.tq4_tqb_decode_attention(ctx.handle, 5, None, 1, None, None, 1, None, 1, 1, 1, SCALE, None, 1,
+                                        None, 0) == tq4.TQ4_ERR_UNSUPPORTED
