@@ -41,7 +41,8 @@ from compressed_paged_kv_tq4_b200 import inputs as I  # noqa: E402
 METRIC = "TQ4 fused attention KV positions/s & HBM GB/s (% of roofline) at 32K–229K ctx"
 UNIT = "KV positions/s"
 SCALE = 1.0 / 16.0
-EXTRA_DEFAULT = "decode_213k_outliers,verify_2req_229k,shared_prefix_8req_33k,prefill_2k_on_32k,int8_decode_32k"
+EXTRA_DEFAULT = ("decode_213k_outliers,verify_2req_229k,shared_prefix_8req_33k,prefill_2k_on_32k,int8_decode_32k,"
+                 "tqb3_decode_32k,tqb2_decode_32k")
 
 
 def parse(argv=None):
@@ -89,13 +90,17 @@ WORKLOAD_DESC = {
     "single_layer_2k": "1 layer, 2,048 TQ4 positions, 1 query token",
     "int8_decode_32k": "uniform INT8 comparison arm: 16 layers x 32,768 INT8 positions (2,064 B per "
                        "layer-position), 1 request, 1 bf16 query token, append of 1 position per layer",
+    "tqb3_decode_32k": "3-bit variant: 16 layers x 32,768 positions (784 B per layer-position), 1 request, "
+                       "1 bf16 query token, append of 1 position per layer",
+    "tqb2_decode_32k": "2-bit variant: 16 layers x 32,768 positions (528 B per layer-position), 1 request, "
+                       "1 bf16 query token, append of 1 position per layer",
 }
 
 
 def workload_config(name, world):
     """The `config` object of the JSON line (the same for both arms)."""
     w = I.WORKLOADS[name]
-    per_pos = 2064 if w.kind == "decode_int8" else 1040
+    per_pos = {"decode_int8": 2064, "decode_tqb2": 528, "decode_tqb3": 784}.get(w.kind, 1040)
     return {"workload": f"{name}: {WORKLOAD_DESC[name]}", "append_per_layer": w.append_per_step,
             "pool_pages": w.pool_pages, "page_positions": 256,
             "l2": "inputs larger than L2: packed KV read per step is "
@@ -442,6 +447,72 @@ class Int8DecodeSetup(DecodeSetup):
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms, "peak_source": f"{peaks_[3]} hbm_gbs"}
 
 
+class TqbDecodeSetup(Int8DecodeSetup):
+    """The 2- or 3-bit variant on a decode workload: each layer's pool holds the
+    history in the narrower format; a step appends the new position with
+    tq4_tqb_encode_append and runs tq4_tqb_decode_attention, per layer."""
+
+    def __init__(self, w, torch, tq4, device):
+        self.w, self.torch, self.tq4 = w, torch, tq4
+        self.bits = 2 if w.kind == "decode_tqb2" else 3
+        self.ctx = tq4.Context(I.signs(w.config))
+        self.tables_np = I.request_tables(w)
+        self.tables = torch.from_numpy(self.tables_np).to(device)
+        self.seq_np = np.array(w.seq_lens, np.int32)
+        self.seq = torch.from_numpy(self.seq_np).to(device)
+        self.total = int(self.seq_np.sum())
+        self.start = int(self.seq_np[0]) - w.n_q
+        if w.n_req != 1:
+            raise ValueError("the variants' bench workloads have one request")
+        self.pools = []
+        self.ws = self.ctx.decode_workspace(w.n_req, w.n_q, self.total, device)
+        ain, aout = Arena(torch, device), Arena(torch, device)
+        qi, ki, vi, oi = [], [], [], []
+        for layer in range(w.layers):
+            pool = tq4.Context.new_tqb_pool(self.bits, w.pool_pages, device)
+            k, v = I.kv_vectors_device(w.config, layer, self.total, outlier_frac=w.outlier_frac, device=device)
+            self.ctx.tqb_encode_append(self.bits, pool, self.tables[0], 0, k[:self.start], v[:self.start])
+            ki.append(ain.add(k[self.start:].cpu().numpy(), torch.float32, (w.n_q, 4, 256)))
+            vi.append(ain.add(v[self.start:].cpu().numpy(), torch.float32, (w.n_q, 4, 256)))
+            del k, v
+            qb = I.queries(w.config, layer, (1, w.n_q, 24, 256))
+            qi.append(ain.add(qb, torch.bfloat16, (1, w.n_q, 24, 256)))
+            oi.append(aout.add(np.zeros((1, w.n_q, 24, 256), np.uint16), torch.bfloat16, (1, w.n_q, 24, 256)))
+            self.pools.append(pool)
+        vin, vout = ain.finalize(), aout.finalize()
+        self.arena_in, self.arena_out = ain, aout
+        self.qs = [vin[i] for i in qi]
+        self.knew = [vin[i] for i in ki]
+        self.vnew = [vin[i] for i in vi]
+        self.outs = [vout[i] for i in oi]
+        torch.cuda.synchronize()
+        if self.ctx.status() != tq4.TQ4_OK:
+            raise RuntimeError(f"{self.bits}-bit cache build failed")
+
+    def attend(self, layer):
+        """The step's append and decode of one layer: two calls on the variant."""
+        tq4, w = self.tq4, self.w
+        rc = tq4.tq4_tqb_encode_append(self.ctx.handle, self.bits, self.pools[layer], w.pool_pages, self.tables[0],
+                                       self.tables.shape[1], self.start, w.n_q, self.knew[layer], self.vnew[layer],
+                                       tq4.DTYPE_F32)
+        assert rc == 0, rc
+        rc = tq4.tq4_tqb_decode_attention(self.ctx.handle, self.bits, self.pools[layer], w.pool_pages, self.qs[layer],
+                                          self.tables, self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total,
+                                          SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
+        assert rc == 0, rc
+
+    def roofline(self, att_ms, peaks_):
+        """Dominant call: one layer's append + decode of the variant; algorithmic bytes =
+        the packed history it must read (528 B or 784 B per attended layer-position)."""
+        hbm = peaks_[0]
+        nbytes = self.total * I.H_KV * 2 * (32 * self.bits + 2)
+        ach = nbytes / (att_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                "traffic": measured_traffic(self.w.name),
+                "kernel": f"tq4_tqb_encode_append + tq4_tqb_decode_attention, {self.bits} bits (split-K + combine)",
+                "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms, "peak_source": f"{peaks_[3]} hbm_gbs"}
+
+
 class PrefillSetup:
     """The prefill workload on the device: every layer's pool holds the TQ4 prefix
     (encoded from K/V drawn on the device); the chunk's queries and K/V are seeded
@@ -663,7 +734,8 @@ def measure_workload(name, args, torch, tq4, device, dist, world, steps, headlin
     if args.layers:
         import dataclasses
         w = dataclasses.replace(w, layers=args.layers)
-    S = {"decode": DecodeSetup, "decode_int8": Int8DecodeSetup, "prefill": PrefillSetup}[w.kind](w, torch, tq4, device)
+    S = {"decode": DecodeSetup, "decode_int8": Int8DecodeSetup, "decode_tqb2": TqbDecodeSetup,
+         "decode_tqb3": TqbDecodeSetup, "prefill": PrefillSetup}[w.kind](w, torch, tq4, device)
     if args.decode_path != "default":
         S.ctx.set_decode_path(tq4.DECODE_PATH_WARP_MMA if args.decode_path == "warp" else tq4.DECODE_PATH_TENSOR_MEMORY)
     stream = torch.cuda.Stream(device)

@@ -171,7 +171,8 @@ class Workload:
     pool_pages: int
     seq_lens: tuple          # attended positions per request (new positions included)
     n_q: int                 # query tokens per request (decode) or chunk length (prefill)
-    kind: str                # "decode", "decode_int8" (the INT8 comparison arm) or "prefill"
+    kind: str                # "decode", "decode_int8" (the INT8 comparison arm), "decode_tqb2" /
+                             # "decode_tqb3" (the 2- and 3-bit variants) or "prefill"
     outlier_frac: float = 0.0
     append_per_step: int = 0  # positions appended by tq4_encode_append per layer per step
     shared_prefix_pages: int = 0
@@ -201,6 +202,11 @@ WORKLOADS = {
                                        shared_prefix_pages=128, grouped=True, append_per_step=1),
     # the uniform INT8 comparison arm on the decode_32k shape (same config, same law of K/V)
     "int8_decode_32k": Workload("int8_decode_32k", 1, 16, POOL_PAGES, (32768,), 1, "decode_int8",
+                                append_per_step=1),
+    # the 3- and 2-bit variants on the decode_32k shape (same config, same law of K/V)
+    "tqb3_decode_32k": Workload("tqb3_decode_32k", 1, 16, POOL_PAGES, (32768,), 1, "decode_tqb3",
+                                append_per_step=1),
+    "tqb2_decode_32k": Workload("tqb2_decode_32k", 1, 16, POOL_PAGES, (32768,), 1, "decode_tqb2",
                                 append_per_step=1),
     # prefill: 2,048 causal query tokens against a 32,768-position TQ4 prefix + the chunk
     "prefill_2k_on_32k": Workload("prefill_2k_on_32k", 4, 16, POOL_PAGES, (32_768 + 2048,), 2048,
