@@ -112,14 +112,16 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
 # ncu capture of that workload (summarised under profiles/). The figures count only
 # while the kernel sources hash to the value they had when the counters were taken.
-MEASURED_TRAFFIC_SOURCES = "38f42d63ea1a05e90a569162c85af6919e200690f40e6cc1c0d7b44ca5ed3b7b"
+MEASURED_TRAFFIC_SOURCES = "f80e9e2edbc9bc7f32a43c323c31e5185b2c780b8cedd393c7956d824d4cb279"
 MEASURED_TRAFFIC = {
-    "decode_32k": 34_221_056,              # decode_q1_kernel: 34,184,192 read + 36,864 written
-    "decode_213k_outliers": 225_458_944,   # decode_q1_kernel: 221,923,840 + 3,535,104
-    "verify_2req_229k": 224_921_088,       # decode_splitk_kernel<3,3>: 221,703,680 + 3,217,408
-    "shared_prefix_8req_33k": 43_076_864,  # decode_splitk_kernel<1,6> (grouped): 42,842,880 + 233,984
-    "int8_decode_32k": 68_667_136,         # decode_splitk_kernel<1,1,INT8>: 67,694,336 + 972,800
-    "prefill_2k_on_32k": 202_866_688,      # prefill_tc_kernel: 101,581,824 + 101,284,864 (segment partials)
+    "decode_32k": 34_188_032,              # decode_q1_kernel: 34,184,448 read + 3,584 written
+    "decode_213k_outliers": 226_268_416,   # decode_q1_kernel: 221,949,952 + 4,318,464
+    "verify_2req_229k": 225_352_704,       # decode_splitk_kernel<3,3>: 221,706,752 + 3,645,952
+    "shared_prefix_8req_33k": 42_972_672,  # decode_splitk_kernel<1,6> (grouped): 42,843,136 + 129,536
+    "int8_decode_32k": 68_470_272,         # decode_splitk_kernel<1,1,INT8>: 67,694,336 + 775,936
+    "prefill_2k_on_32k": 204_016_640,      # prefill_tc_kernel: 101,828,096 + 102,188,544 (segment partials)
+    "tqb3_decode_32k": 25_765_888,         # decode_bits_kernel<1,0,3>: 25,765,632 + 256
+    "tqb2_decode_32k": 17_377_536,         # decode_bits_kernel<1,0,2>: 17,377,536 + 0
 }
 
 
