@@ -3,7 +3,8 @@
 Decode over 32,768 positions, over 212,992 positions with 5% x8 norms, over two
 requests of 163,840 + 65,536 positions (4 causal query tokens each, 64 shared
 pages) and over eight one-token requests sharing 32,768 of their 33,792
-positions, the last two both ungrouped and grouped (shared pages read once);
+positions, the last two both ungrouped and grouped (shared pages read once), and
+the two-request verify also on the tensor-memory (tcgen05) kernel;
 prefill of 2,048 tokens on a 32,768-position prefix, on the packed path and by
 direct inverse reconstruction; the prefill's 2,048-token append. For attention the pool is filled with seeded random codes and
 norms (every 4-bit value occurs; norms follow the workloads' scale mix), so both
@@ -69,6 +70,16 @@ def test_decode_full_size(codebook, name):
     g32 = got32.cpu().numpy().astype(np.float64)
     assert np.abs(g32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), name
     H.assert_bf16_close(got16.float().cpu().numpy(), exp, name)
+    if w.n_q > 1:   # the tensor-memory kernel (tcgen05) on the same full-size call
+        ctx.set_decode_path(tq4.DECODE_PATH_TENSOR_MEMORY)
+        tm32 = ctx.decode_attention(dpool, q, dtab, dseq, int(seq.sum()), SCALE, out_dtype=torch.float32)
+        tm16 = ctx.decode_attention(dpool, q, dtab, dseq, int(seq.sum()), SCALE, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        ctx.set_decode_path(tq4.DECODE_PATH_WARP_MMA)
+        assert ctx.status() == tq4.TQ4_OK
+        t32 = tm32.cpu().numpy().astype(np.float64)
+        assert np.abs(t32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), name + " tensor memory"
+        H.assert_bf16_close(tm16.float().cpu().numpy(), exp, name + " tensor memory")
     if w.shared_prefix_pages:   # the grouped decode: every request led by request 0
         leader, pages = [0] * w.n_req, [w.shared_prefix_pages] * w.n_req
         sh32 = ctx.decode_attention_shared(dpool, q, dtab, dseq, int(seq.sum()), SCALE, leader, pages,
