@@ -69,7 +69,7 @@ extern "C" {
 
 #define TQ4_OK                 0
 #define TQ4_ERR_ARG           -1  /* bad pointer, size, count or dtype             */
-#define TQ4_ERR_UNSUPPORTED   -2  /* shape this build is not specialised for       */
+#define TQ4_ERR_UNSUPPORTED   -2  /* shape the library is not specialised for     */
 #define TQ4_ERR_PAGE_RANGE    -3  /* page id outside [0, num_pages) (device check) */
 #define TQ4_ERR_CUDA          -4  /* a CUDA runtime call failed                    */
 #define TQ4_ERR_WORKSPACE     -5  /* workspace missing or smaller than required    */
