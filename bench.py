@@ -451,8 +451,8 @@ class Int8DecodeSetup(DecodeSetup):
 
 class TqbDecodeSetup(Int8DecodeSetup):
     """The 2- or 3-bit variant on a decode workload: each layer's pool holds the
-    history in the narrower format; a step appends the new position with
-    tq4_tqb_encode_append and runs tq4_tqb_decode_attention, per layer."""
+    history in the narrower format; a step is tq4_tqb_decode_append_attention per
+    layer (the new position appended inside the one-token decode kernel)."""
 
     def __init__(self, w, torch, tq4, device):
         self.w, self.torch, self.tq4 = w, torch, tq4
@@ -491,16 +491,18 @@ class TqbDecodeSetup(Int8DecodeSetup):
         if self.ctx.status() != tq4.TQ4_OK:
             raise RuntimeError(f"{self.bits}-bit cache build failed")
 
+    def kernels_per_step(self):
+        # decode (append fused) + combine per layer; with n_q > 1 a tail-encode kernel as well
+        return self.w.layers * (2 if self.w.n_q == 1 else 3)
+
     def attend(self, layer):
-        """The step's append and decode of one layer: two calls on the variant."""
+        """The step's append and decode of one layer: one fused call on the variant."""
         tq4, w = self.tq4, self.w
-        rc = tq4.tq4_tqb_encode_append(self.ctx.handle, self.bits, self.pools[layer], w.pool_pages, self.tables[0],
-                                       self.tables.shape[1], self.start, w.n_q, self.knew[layer], self.vnew[layer],
-                                       tq4.DTYPE_F32)
-        assert rc == 0, rc
-        rc = tq4.tq4_tqb_decode_attention(self.ctx.handle, self.bits, self.pools[layer], w.pool_pages, self.qs[layer],
-                                          self.tables, self.tables.shape[1], self.seq, w.n_req, w.n_q, self.total,
-                                          SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws, self.ws.numel())
+        rc = tq4.tq4_tqb_decode_append_attention(self.ctx.handle, self.bits, self.pools[layer], w.pool_pages,
+                                                 self.knew[layer], self.vnew[layer], tq4.DTYPE_F32, self.qs[layer],
+                                                 self.tables, self.tables.shape[1], self.seq, w.n_req, w.n_q,
+                                                 self.total, SCALE, self.outs[layer], tq4.DTYPE_BF16, self.ws,
+                                                 self.ws.numel())
         assert rc == 0, rc
 
     def roofline(self, att_ms, peaks_):
@@ -511,7 +513,8 @@ class TqbDecodeSetup(Int8DecodeSetup):
         ach = nbytes / (att_ms * 1e-3) / 1e9
         return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                 "traffic": measured_traffic(self.w.name),
-                "kernel": f"tq4_tqb_encode_append + tq4_tqb_decode_attention, {self.bits} bits (split-K + combine)",
+                "kernel": f"tq4_tqb_decode_append_attention, {self.bits} bits (decode_q1_kernel<0,{self.bits}> with the "
+                          "append fused + combine)",
                 "algorithmic_bytes_per_launch": nbytes, "launch_ms": att_ms, "peak_source": f"{peaks_[3]} hbm_gbs"}
 
 

@@ -136,6 +136,18 @@ cudaError_t launch_bits_nt(dim3 grid, cudaStream_t st, const tq4::DecodeParams& 
   return tq4::launch_pdl(tq4::decode_bits_kernel<NT, false, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
 }
 // a 2- or 3-bit pool's split-K decode
+// One query token over a b-bit pool: the one-token kernel (tiles by bulk copies,
+// so the tensor map argument is unused).
+template <int kBits>
+cudaError_t launch_q1_bits(bool exact, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  const CUtensorMap unused{};
+  if (exact)
+    return tq4::launch_pdl(tq4::decode_q1_kernel<true, kBits>, grid, dim3(tq4::kQ1Threads),
+                           tq4::decode_q1_smem_bytes(), st, p, unused);
+  return tq4::launch_pdl(tq4::decode_q1_kernel<false, kBits>, grid, dim3(tq4::kQ1Threads),
+                         tq4::decode_q1_smem_bytes(), st, p, unused);
+}
+
 cudaError_t launch_decode_bits(int bits, int nt, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
   if (bits == 2) {
     switch (nt) {
@@ -387,12 +399,14 @@ int tq4_ctx_create(const int8_t* signs, tq4_ctx** out) {
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(tq4::g_codebook_b, cbb, sizeof(cbb));
   if (e == cudaSuccess) e = set_decode_bits_attrs<2>();
   if (e == cudaSuccess) e = set_decode_bits_attrs<3>();
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(tq4::decode_q1_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(tq4::decode_q1_smem_bytes()));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(tq4::decode_q1_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             int(tq4::decode_q1_smem_bytes()));
+  for (const void* fn : {reinterpret_cast<const void*>(tq4::decode_q1_kernel<false, 4>),
+                         reinterpret_cast<const void*>(tq4::decode_q1_kernel<true, 4>),
+                         reinterpret_cast<const void*>(tq4::decode_q1_kernel<false, 2>),
+                         reinterpret_cast<const void*>(tq4::decode_q1_kernel<true, 2>),
+                         reinterpret_cast<const void*>(tq4::decode_q1_kernel<false, 3>),
+                         reinterpret_cast<const void*>(tq4::decode_q1_kernel<true, 3>)})
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(tq4::decode_q1_smem_bytes()));
   if (e == cudaSuccess) e = set_decode_attrs<1, 1, false>();
   if (e == cudaSuccess) e = set_decode_attrs<2, 2, false>();
   if (e == cudaSuccess) e = set_decode_attrs<3, 3, false>();
@@ -560,12 +574,16 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
     p.new_dtype = app->dtype;
   } else if (app) {        // a tail-encode kernel ahead of the decode
     e = tq4::launch_encode_tail(static_cast<uint8_t*>(app->pool), num_pages, page_tables, max_pages, seq_lens,
-                                n_req, n_q, app->k_new, app->v_new, app->dtype, ctx->signs, ctx->d_status, st);
+                                n_req, n_q, app->k_new, app->v_new, app->dtype, ctx->signs, ctx->d_status, st, bits);
     if (e != cudaSuccess) return TQ4_ERR_CUDA;
   }
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   if (bits != 4) {
-    e = launch_decode_bits(bits, tq4::decode_nt(n_q), grid, st, p);
+    const bool exact = out_dtype == TQ4_DTYPE_F32;
+    if (tq4::decode_nt(n_q) == 1)
+      e = bits == 2 ? launch_q1_bits<2>(exact, grid, st, p) : launch_q1_bits<3>(exact, grid, st, p);
+    else
+      e = launch_decode_bits(bits, tq4::decode_nt(n_q), grid, st, p);
   } else if (int8) {
     e = launch_splitk_nt<true>(tq4::decode_nt(n_q), false, grid, st, p);
   } else if (groups) {     // group items and the requests' own items in one launch
@@ -685,6 +703,17 @@ int tq4_tqb_decode_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t n
   if (bits != 2 && bits != 3) return ctx ? TQ4_ERR_UNSUPPORTED : TQ4_ERR_ARG;
   return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
                      out, out_dtype, workspace, workspace_bytes, stream, nullptr, false, nullptr, nullptr, bits);
+}
+
+int tq4_tqb_decode_append_attention(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages, const void* k_new,
+                                    const void* v_new, int new_dtype, const uint16_t* q, const int32_t* page_tables,
+                                    int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                    int64_t total_seq_len, float scale, void* out, int out_dtype, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (bits != 2 && bits != 3) return ctx ? TQ4_ERR_UNSUPPORTED : TQ4_ERR_ARG;
+  const AppendArgs app{pool, k_new, v_new, new_dtype};
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, &app, false, nullptr, nullptr, bits);
 }
 
 size_t tq4_prefill_workspace_bytes(int32_t n_tok) {

@@ -22,6 +22,12 @@
 //   * V phase: O'^T += C_v^T P'^T over all 256 dims (M = dims, K = positions);
 //   * at the end the 8 warp states (m, l, o') are merged through shared memory
 //     and written as one split-K partial for the combine pass.
+//   * 2- and 3-bit pools (kBits): the same kernel; lane 0 copies a tile's word rows
+//     (64 or 96 B per position) and norms with plain bulk copies, and each lane
+//     widens the plane words it loads into the nibble words of the four-bit layout,
+//     so the table lookups, MMAs and softmax below are shared; the table holds the
+//     b-bit codebook (codes never exceed 2^b - 1); the fused append encodes with
+//     the b-bit quantiser and packing;
 //   * fused append: in the CTA that owns a request's last position, warps 6 and 7
 //     encode the new K and V vectors of this KV head (the append kernel's
 //     arithmetic), store them in the pool and fence them for the tensor-copy
@@ -76,6 +82,14 @@ constexpr size_t decode_q1_smem_bytes() { return kQ1DynBytes; }
 // and V-phase shared loads conflict-free.
 __host__ __device__ constexpr int q1_sigma(int m) {
   return ((0x37156240u >> (4 * (m & 7))) & 7) + (m & 8);
+}
+// The b-bit pools' rows are 64 or 96 B (no swizzle): with sigma = [0,1,2,3,5,4,7,6]
+// the 8-byte plane-0 loads of both phases are conflict-free for 96-B rows (each
+// half warp meets four rows whose bank offsets 24 r mod 32 differ) and 2-way for
+// 64-B rows (two offsets only).
+template <int kBits>
+__host__ __device__ constexpr int q1_sigma_b(int m) {
+  return kBits == 4 ? q1_sigma(m) : ((0x67453210u >> (4 * (m & 7))) & 7) + (m & 8);
 }
 
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -163,9 +177,33 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // K words (4 heads x 256 slots), V words, then 32 rows of norms.
 constexpr int kRowsPerPage = int(kPageBytes / 128);   // 2,080
 
-template <bool kExact>   // fp32 outputs: C_lo P' on every tile (see kVloNorm)
+// Nibble words 4i .. 4i + 3 (dims 32i .. 32i + 31) of one position of a b-bit pool,
+// from its staged row at `row`: plane-0 words 2i, 2i + 1 widened to the low two
+// bits of each nibble and, with 3 bits, byte m of plane-1 word 16 + i as bit 2 of
+// nibble word 4i + m.
+template <int kBits>
+__device__ __forceinline__ uint4 widen_words32(uint32_t row, int i) {
+  uint32_t a, b;
+  ld_shared_v2(row + 8 * i, a, b);
+  uint4 r = make_uint4(widen2(a), widen2(a >> 16), widen2(b), widen2(b >> 16));
+  if constexpr (kBits == 3) {
+    const uint32_t hb = ld_shared_u32(row + 64 + 4 * i);
+    r.x |= widen1(hb) << 2;
+    r.y |= widen1(hb >> 8) << 2;
+    r.z |= widen1(hb >> 16) << 2;
+    r.w |= widen1(hb >> 24) << 2;
+  }
+  return r;
+}
+
+// kExact: fp32 outputs, C_lo P' on every tile (see kVloNorm). kBits: 4 (TQ4 pool,
+// tiles by tensor copies through tmap), or 2 / 3 (b-bit pools, tmap unused).
+template <bool kExact, int kBits = 4>
 __global__ void __launch_bounds__(kQ1Threads, 1)
     decode_q1_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmap) {
+  static_assert(kBits == 4 || kBits == 2 || kBits == 3, "bit width");
+  constexpr uint32_t kRB = uint32_t(tqb_row_bytes<kBits>());   // bytes of a staged word row: 32 b
+  static_assert(kQ1Tile * kRB <= uint32_t(kQ1KV), "a tile's word rows fit their half of the buffer");
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t base = smem_u32(smem);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -189,7 +227,9 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   // table rows: 32 copies of the c16 pair, then 32 copies of the r16 pair (16-B stores of 4 copies)
   for (int e = tid; e < 256 * 16; e += kQ1Threads) {
-    const uint2 v = lut_row(e >> 4);
+    uint2 v;
+    if constexpr (kBits == 4) v = lut_row(e >> 4);
+    else v = lut_row_bits<kBits>(e >> 4);
     const uint32_t x = (e & 8) ? v.y : v.x;
     asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};\n" ::"r"(kQ1Lut + (e >> 4) * 256 + (e & 15) * 16), "r"(x)
                  : "memory");
@@ -264,8 +304,14 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
   auto fused_encode = [&]() {
     const int kv = w - (kQ1Warps - 2);
     float nrm;
-    const uint32_t word = encode_vector_warp(x_new, p.signs, nrm);
-    store_packed_warp(p.pool_w, p.num_pages, table, seq_len - 1, h, kv, word, nrm, p.status);
+    if constexpr (kBits == 4) {
+      const uint32_t word = encode_vector_warp(x_new, p.signs, nrm);
+      store_packed_warp(p.pool_w, p.num_pages, table, seq_len - 1, h, kv, word, nrm, p.status);
+    } else {
+      uint32_t w0, w1;
+      encode_bits_warp<kBits>(x_new, p.signs, w0, w1, nrm);
+      store_bits_warp<kBits>(p.pool_w, p.num_pages, table, seq_len - 1, h, kv, w0, w1, nrm, p.status);
+    }
     asm volatile("fence.proxy.async.global;\n" ::: "memory");   // generic stores -> the TMA reads below
     __syncwarp();
     if (lane == 0) mbar_arrive_q1(bar_new);
@@ -307,18 +353,30 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         page = 0;   // still complete the barrier (reading page 0); the tile is masked below
       }
       const int slot0 = h * kPage + (c & (kPage - 1));
-      const int row = page * kRowsPerPage + slot0;
-      const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
       const uint32_t kdst = buf_addr(b), ndst = base + kQ1NrmOff + b * 128;
-      // A half tile still takes 32-row word boxes (the extra rows stay inside the
-      // page: at most row 2,063 of its 2,080) but only its own 16 norms, since the
-      // V norms end the page.
       const uint32_t nbytes = tile_half(k) ? kQ1Tile : 2 * kQ1Tile;
-      mbar_expect_tx(bar, 2 * kQ1KV + 2 * nbytes);
-      tma_load_2d(kdst, &tmap, 0, row, bar);                       // K words of 32 positions
-      tma_load_2d(kdst + kQ1KV, &tmap, 0, row + 4 * kPage, bar);   // V words
-      bulk_load(ndst, pg + kKNorms + slot0 * 2, nbytes, bar);
-      bulk_load(ndst + 64, pg + kVNorms + slot0 * 2, nbytes, bar);
+      if constexpr (kBits == 4) {
+        const int row = page * kRowsPerPage + slot0;
+        const uint8_t* pg = p.pool + int64_t(page) * kPageBytes;
+        // A half tile still takes 32-row word boxes (the extra rows stay inside the
+        // page: at most row 2,063 of its 2,080) but only its own 16 norms, since the
+        // V norms end the page.
+        mbar_expect_tx(bar, 2 * kQ1KV + 2 * nbytes);
+        tma_load_2d(kdst, &tmap, 0, row, bar);                       // K words of 32 positions
+        tma_load_2d(kdst + kQ1KV, &tmap, 0, row + 4 * kPage, bar);   // V words
+        bulk_load(ndst, pg + kKNorms + slot0 * 2, nbytes, bar);
+        bulk_load(ndst + 64, pg + kVNorms + slot0 * 2, nbytes, bar);
+      } else {
+        // b-bit pool: a tile's rows are contiguous (slot0 is a multiple of 16, so
+        // every source is 16-byte aligned); a half tile copies its 16 rows only
+        const uint8_t* pg = p.pool + int64_t(page) * tqb_page_bytes<kBits>();
+        const uint32_t wbytes = (tile_half(k) ? kQ1Tile / 2 : kQ1Tile) * kRB;
+        mbar_expect_tx(bar, 2 * wbytes + 2 * nbytes);
+        bulk_load(kdst, pg + int64_t(slot0) * kRB, wbytes, bar);
+        bulk_load(kdst + kQ1KV, pg + tqb_v_words<kBits>() + int64_t(slot0) * kRB, wbytes, bar);
+        bulk_load(ndst, pg + tqb_k_norms<kBits>() + slot0 * 2, nbytes, bar);
+        bulk_load(ndst + 64, pg + tqb_v_norms<kBits>() + slot0 * 2, nbytes, bar);
+      }
     }
   };
   if (encoder) fused_load();
@@ -376,8 +434,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
     for (int i = 0; i < 4; ++i) o[mt][i] = 0.f;
 
   // positions of this lane: K phase rows g, g+8 -> sigma; V phase k-indices 2t, 2t+1 (+8)
-  const int pk = q1_sigma(g);                        // and pk + 8 (same swizzle phase)
-  const int pv0 = q1_sigma(2 * t), pv1 = q1_sigma(2 * t + 1);
+  const int pk = q1_sigma_b<kBits>(g);               // and pk + 8 (same swizzle phase)
+  const int pv0 = q1_sigma_b<kBits>(2 * t), pv1 = q1_sigma_b<kBits>(2 * t + 1);
   const uint32_t k_off0 = pk * 128 + ((t ^ (pk & 7)) << 4);          // words 4t..4t+3
   const uint32_t k_off1 = pk * 128 + (((4 + t) ^ (pk & 7)) << 4);    // words 16+4t..16+4t+3
   const uint32_t v_off0 = pv0 * 128 + ((g ^ (pv0 & 7)) << 4);        // words 4g..4g+3 of position pv0
@@ -414,11 +472,19 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
         ka[1] = kb4[1] = kc[1] = kd[1] = make_uint4(0, 0, 0, 0);
         break;
       }
-      const uint32_t mrow = kst + j * 16 * 128;
-      ka[j] = ld_shared_v4(mrow + k_off0);
-      kb4[j] = ld_shared_v4(mrow + k_off1);
-      kc[j] = ld_shared_v4(mrow + 8 * 128 + k_off0);
-      kd[j] = ld_shared_v4(mrow + 8 * 128 + k_off1);
+      if constexpr (kBits == 4) {
+        const uint32_t mrow = kst + j * 16 * 128;
+        ka[j] = ld_shared_v4(mrow + k_off0);
+        kb4[j] = ld_shared_v4(mrow + k_off1);
+        kc[j] = ld_shared_v4(mrow + 8 * 128 + k_off0);
+        kd[j] = ld_shared_v4(mrow + 8 * 128 + k_off1);
+      } else {   // the same nibble words, widened from positions pk, pk + 8
+        const uint32_t r0 = kst + (16 * j + pk) * kRB, r8 = r0 + 8 * kRB;
+        ka[j] = widen_words32<kBits>(r0, t);
+        kb4[j] = widen_words32<kBits>(r0, 4 + t);
+        kc[j] = widen_words32<kBits>(r8, t);
+        kd[j] = widen_words32<kBits>(r8, 4 + t);
+      }
     }
     // S = (C_hi + C_lo)(q'_hi + q'_lo) less C_lo q'_lo: sc = C_hi q'_hi, sd = C_hi q'_lo,
     // se = C_lo q'_hi (three accumulators: three independent chains of 16 MMAs)
@@ -534,11 +600,20 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       if (j == 1 && !two) break;   // a half tile's positions 16-31 carry P' = 0
-      const uint32_t vrow = vst + j * 16 * 128;
-      const uint4 x0 = ld_shared_v4(vrow + v_off0);              // position sigma(2t)
-      const uint4 x1 = ld_shared_v4(vrow + v_off1);              // position sigma(2t+1)
-      const uint4 y0 = ld_shared_v4(vrow + 8 * 128 + v_off0);    // +8
-      const uint4 y1 = ld_shared_v4(vrow + 8 * 128 + v_off1);
+      uint4 x0, x1, y0, y1;
+      if constexpr (kBits == 4) {
+        const uint32_t vrow = vst + j * 16 * 128;
+        x0 = ld_shared_v4(vrow + v_off0);              // position sigma(2t)
+        x1 = ld_shared_v4(vrow + v_off1);              // position sigma(2t+1)
+        y0 = ld_shared_v4(vrow + 8 * 128 + v_off0);    // +8
+        y1 = ld_shared_v4(vrow + 8 * 128 + v_off1);
+      } else {   // nibble words 4g .. 4g + 3 of the same positions
+        const uint32_t vrow = vst + 16 * j * kRB;
+        x0 = widen_words32<kBits>(vrow + pv0 * kRB, g);
+        x1 = widen_words32<kBits>(vrow + pv1 * kRB, g);
+        y0 = widen_words32<kBits>(vrow + (pv0 + 8) * kRB, g);
+        y1 = widen_words32<kBits>(vrow + (pv1 + 8) * kRB, g);
+      }
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t lo01, hi01, lo89, hi89;

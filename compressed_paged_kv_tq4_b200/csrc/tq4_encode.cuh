@@ -108,34 +108,6 @@ __global__ void __launch_bounds__(256) encode_append_kernel(
   store_packed_warp(pool, num_pages, page_table, start_pos + tok, head, kv, word, n, status);
 }
 
-// The last n_q positions of every request, with positions taken from the device
-// lengths: new token t of request r goes to position seq_lens[r] - n_q + t.
-// grid: ceil(n_req * n_q * 8 / warps_per_block); inputs [n_req][n_q][4][256].
-template <typename T>
-__global__ void __launch_bounds__(256) encode_tail_kernel(
-    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_tables, int32_t max_pages,
-    const int32_t* __restrict__ seq_lens, int32_t n_req, int32_t n_q, const T* __restrict__ k_new,
-    const T* __restrict__ v_new, Signs signs, int* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  pdl_wait();
-  pdl_launch_dependents();
-  if (vec >= int64_t(n_req) * n_q * 2 * kHkv) return;
-  const int64_t tok = vec / (2 * kHkv);       // request-major token index
-  const int r = int(tok / n_q), t = int(tok % n_q);
-  const int kv = int(vec / kHkv) & 1;
-  const int head = int(vec % kHkv);
-  const int32_t len = __ldg(seq_lens + r);
-  if (len < n_q || len > max_pages * kPage) {   // the decode kernels record TQ4_ERR_SEQ for it
-    return;
-  }
-  float x[8];
-  load8<T>((kv ? v_new : k_new) + (tok * kHkv + head) * kD + lane * 8, x);
-  float n;
-  const uint32_t word = encode_vector_warp(x, signs, n);
-  store_packed_warp(pool, num_pages, page_tables + int64_t(r) * max_pages, len - n_q + t, head, kv, word, n, status);
-}
-
 // grid: ceil(n * 8 / warps_per_block); writes fp32 [n][4][256] for K and V
 __global__ void __launch_bounds__(256) reconstruct_kernel(
     const uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table,
@@ -227,28 +199,20 @@ __global__ void __launch_bounds__(256) int8_encode_kernel(
 // The 2- and 3-bit variants: the four-bit encode with a 2^kBits-level codebook
 // (g_codebook_b) and the bit-plane packing of tqb_row_bytes: lane l's indices of
 // coordinates 8l .. 8l + 7 give the 16 low bits (plane 0) of word l / 2 and the 8
-// bits at 8 (l & 3) of plane-1 word 16 + l / 4. One warp per vector.
-template <typename T, int kBits>
-__global__ void __launch_bounds__(256) encode_bits_kernel(
-    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table, int32_t start_pos,
-    int32_t n_tok, const T* __restrict__ k_new, const T* __restrict__ v_new, Signs signs, int* status) {
+// bits at 8 (l & 3) of plane-1 word 16 + l / 4. One warp per vector: w0 receives
+// plane-0 word l / 2 (meaningful in even lanes), w1 plane-1 word 16 + l / 4
+// (meaningful in lanes 4w), n the norm.
+template <int kBits>
+__device__ __forceinline__ void encode_bits_warp(const float x[8], const Signs& signs, uint32_t& w0, uint32_t& w1,
+                                                 float& n) {
   const int lane = threadIdx.x & 31;
-  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  pdl_wait();
-  pdl_launch_dependents();
-  if (vec >= int64_t(n_tok) * 2 * kHkv) return;
-  const int tok = int(vec / (2 * kHkv));
-  const int kv = int(vec / kHkv) & 1;
-  const int head = int(vec % kHkv);
-  float x[8];
-  load8<T>((kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8, x);
   const CodebookB& cb = g_codebook_b[kBits - 2];
   float ss = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) ss = fmaf(x[i], x[i], ss);
 #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-  const float n = sqrtf(ss);
+  n = sqrtf(ss);
   uint32_t lo16 = 0, hi8 = 0;
   if (n > 0.f) {
     const uint32_t sb = lane_sign_bits(signs);
@@ -267,15 +231,23 @@ __global__ void __launch_bounds__(256) encode_bits_kernel(
     }
   }
   // plane 0: word w = lanes 2w (low half) and 2w + 1; plane 1: word w = lanes 4w .. 4w + 3
-  const uint32_t w0 = lo16 | (__shfl_down_sync(0xffffffffu, lo16, 1) << 16);
-  uint32_t w1 = hi8 << (8 * (lane & 3));
+  w0 = lo16 | (__shfl_down_sync(0xffffffffu, lo16, 1) << 16);
+  w1 = hi8 << (8 * (lane & 3));
   w1 |= __shfl_xor_sync(0xffffffffu, w1, 1);
   w1 |= __shfl_xor_sync(0xffffffffu, w1, 2);
-  const int32_t pos = start_pos + tok;
-  const int32_t page = __ldg(page_table + (pos >> 8));
+}
+
+// Store a b-bit vector at position pos of a request (page table `table`), head
+// `head`, K (kv = 0) or V. A page id outside [0, num_pages) records
+// TQ4_ERR_PAGE_RANGE and writes nothing; returns false then.
+template <int kBits>
+__device__ __forceinline__ bool store_bits_warp(uint8_t* pool, int32_t num_pages, const int32_t* table, int32_t pos,
+                                                int head, int kv, uint32_t w0, uint32_t w1, float n, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int32_t page = __ldg(table + (pos >> 8));
   if (page < 0 || page >= num_pages) {
     if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
-    return;
+    return false;
   }
   const int slot = head * kPage + (pos & (kPage - 1));
   uint8_t* base = pool + int64_t(page) * tqb_page_bytes<kBits>();
@@ -285,6 +257,64 @@ __global__ void __launch_bounds__(256) encode_bits_kernel(
   if (kBits == 3 && (lane & 3) == 0) words[16 + (lane >> 2)] = w1;
   if (lane == 0)
     reinterpret_cast<__half*>(base + (kv ? tqb_v_norms<kBits>() : tqb_k_norms<kBits>()))[slot] = __float2half_rn(n);
+  return true;
+}
+
+// One warp per new b-bit vector: grid ceil(n_tok * 8 / warps_per_block)
+template <typename T, int kBits>
+__global__ void __launch_bounds__(256) encode_bits_kernel(
+    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table, int32_t start_pos,
+    int32_t n_tok, const T* __restrict__ k_new, const T* __restrict__ v_new, Signs signs, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (vec >= int64_t(n_tok) * 2 * kHkv) return;
+  const int tok = int(vec / (2 * kHkv));
+  const int kv = int(vec / kHkv) & 1;
+  const int head = int(vec % kHkv);
+  float x[8];
+  load8<T>((kv ? v_new : k_new) + (int64_t(tok) * kHkv + head) * kD + lane * 8, x);
+  uint32_t w0, w1;
+  float n;
+  encode_bits_warp<kBits>(x, signs, w0, w1, n);
+  store_bits_warp<kBits>(pool, num_pages, page_table, start_pos + tok, head, kv, w0, w1, n, status);
+}
+
+// The last n_q positions of every request, with positions taken from the device
+// lengths: new token t of request r goes to position seq_lens[r] - n_q + t.
+// grid: ceil(n_req * n_q * 8 / warps_per_block); inputs [n_req][n_q][4][256].
+// kBits: 4 (TQ4 pool) or 2 / 3 (b-bit pools).
+template <typename T, int kBits>
+__global__ void __launch_bounds__(256) encode_tail_kernel(
+    uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_tables, int32_t max_pages,
+    const int32_t* __restrict__ seq_lens, int32_t n_req, int32_t n_q, const T* __restrict__ k_new,
+    const T* __restrict__ v_new, Signs signs, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();
+  if (vec >= int64_t(n_req) * n_q * 2 * kHkv) return;
+  const int64_t tok = vec / (2 * kHkv);       // request-major token index
+  const int r = int(tok / n_q), t = int(tok % n_q);
+  const int kv = int(vec / kHkv) & 1;
+  const int head = int(vec % kHkv);
+  const int32_t len = __ldg(seq_lens + r);
+  if (len < n_q || len > max_pages * kPage) {   // the decode kernels record TQ4_ERR_SEQ for it
+    return;
+  }
+  float x[8];
+  load8<T>((kv ? v_new : k_new) + (tok * kHkv + head) * kD + lane * 8, x);
+  float n;
+  const int32_t* table = page_tables + int64_t(r) * max_pages;
+  if constexpr (kBits == 4) {
+    const uint32_t word = encode_vector_warp(x, signs, n);
+    store_packed_warp(pool, num_pages, table, len - n_q + t, head, kv, word, n, status);
+  } else {
+    uint32_t w0, w1;
+    encode_bits_warp<kBits>(x, signs, w0, w1, n);
+    store_bits_warp<kBits>(pool, num_pages, table, len - n_q + t, head, kv, w0, w1, n, status);
+  }
 }
 
 // ---------------------------------------------------------------- launchers
@@ -333,19 +363,34 @@ cudaError_t launch_encode_append(uint8_t* pool, int32_t num_pages, const int32_t
                     static_cast<const uint16_t*>(v_new), signs, status);
 }
 
-cudaError_t launch_encode_tail(uint8_t* pool, int32_t num_pages, const int32_t* page_tables, int32_t max_pages,
-                               const int32_t* seq_lens, int32_t n_req, int32_t n_q, const void* k_new,
-                               const void* v_new, int dtype, const Signs& signs, int* status, cudaStream_t stream) {
+template <int kBits>
+cudaError_t launch_encode_tail_b(uint8_t* pool, int32_t num_pages, const int32_t* page_tables, int32_t max_pages,
+                                 const int32_t* seq_lens, int32_t n_req, int32_t n_q, const void* k_new,
+                                 const void* v_new, int dtype, const Signs& signs, int* status, cudaStream_t stream) {
   const int threads = 256, wpb = threads / 32;
   const int64_t vecs = int64_t(n_req) * n_q * 2 * kHkv;
   const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
   if (dtype == TQ4_DTYPE_F32)
-    return launch_pdl(encode_tail_kernel<float>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+    return launch_pdl(encode_tail_kernel<float, kBits>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
                       page_tables, max_pages, seq_lens, n_req, n_q, static_cast<const float*>(k_new),
                       static_cast<const float*>(v_new), signs, status);
-  return launch_pdl(encode_tail_kernel<uint16_t>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
+  return launch_pdl(encode_tail_kernel<uint16_t, kBits>, dim3(blocks), dim3(threads), 0, stream, pool, num_pages,
                     page_tables, max_pages, seq_lens, n_req, n_q, static_cast<const uint16_t*>(k_new),
                     static_cast<const uint16_t*>(v_new), signs, status);
+}
+// bits: 4 (TQ4 pool), 2 or 3
+inline cudaError_t launch_encode_tail(uint8_t* pool, int32_t num_pages, const int32_t* page_tables,
+                                      int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                      const void* k_new, const void* v_new, int dtype, const Signs& signs,
+                                      int* status, cudaStream_t stream, int bits = 4) {
+  switch (bits) {
+    case 2: return launch_encode_tail_b<2>(pool, num_pages, page_tables, max_pages, seq_lens, n_req, n_q, k_new,
+                                           v_new, dtype, signs, status, stream);
+    case 3: return launch_encode_tail_b<3>(pool, num_pages, page_tables, max_pages, seq_lens, n_req, n_q, k_new,
+                                           v_new, dtype, signs, status, stream);
+    default: return launch_encode_tail_b<4>(pool, num_pages, page_tables, max_pages, seq_lens, n_req, n_q, k_new,
+                                            v_new, dtype, signs, status, stream);
+  }
 }
 
 cudaError_t launch_reconstruct(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,

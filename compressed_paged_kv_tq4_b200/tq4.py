@@ -51,6 +51,7 @@ EXPORTS = (
     "tq4_decode_shared_workspace_bytes", "tq4_decode_attention_shared",
     "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
     "tq4_ctx_set_decode_path", "tq4_tqb_codebook", "tq4_tqb_encode_append", "tq4_tqb_decode_attention",
+    "tq4_tqb_decode_append_attention",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -94,6 +95,8 @@ _sig = {
                               ctypes.c_int),
     "tq4_tqb_decode_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p,
                                   ctypes.c_int, _p, _sz, _p], ctypes.c_int),
+    "tq4_tqb_decode_append_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32,
+                                         _i32, _i64, _f, _p, ctypes.c_int, _p, _sz, _p], ctypes.c_int),
     "tq4_int8_encode_append": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p], ctypes.c_int),
     "tq4_int8_decode_attention": ([_p, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p, ctypes.c_int,
                                    _p, _sz, _p], ctypes.c_int),
@@ -292,6 +295,15 @@ def tq4_tqb_decode_attention(ctx, bits, pool, num_pages, q, page_tables, max_pag
     return _lib.tq4_tqb_decode_attention(ctx, bits, _ptr(pool), num_pages, _ptr(q), _ptr(page_tables), max_pages,
                                          _ptr(seq_lens), n_req, n_q, total_seq_len, scale, _ptr(out), out_dtype,
                                          _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_tqb_decode_append_attention(ctx, bits, pool, num_pages, k_new, v_new, new_dtype, q, page_tables, max_pages,
+                                    seq_lens, n_req, n_q, total_seq_len, scale, out, out_dtype, workspace,
+                                    workspace_bytes, stream=None) -> int:
+    return _lib.tq4_tqb_decode_append_attention(ctx, bits, _ptr(pool), num_pages, _ptr(k_new), _ptr(v_new),
+                                                new_dtype, _ptr(q), _ptr(page_tables), max_pages, _ptr(seq_lens),
+                                                n_req, n_q, total_seq_len, scale, _ptr(out), out_dtype,
+                                                _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def tq4_ctx_set_wait_limit(ctx, polls, withhold_signal=0) -> int:
@@ -617,6 +629,31 @@ class Context:
                                         page_tables, page_tables.shape[1], seq_lens, n_req, n_q, total_seq_len,
                                         scale, out, od, workspace, workspace.numel(), stream),
                "tq4_tqb_decode_attention")
+        return out
+
+    def tqb_decode_append_attention(self, bits, pool, k_new, v_new, q, page_tables, seq_lens, total_seq_len, scale,
+                                    out=None, out_dtype=torch.bfloat16, workspace=None, stream=None):
+        """decode_append_attention for a b-bit pool: k_new/v_new [n_req, n_q, 4, 256]
+        (float32 or bfloat16) encoded at the last n_q positions, then the decode."""
+        _need_cuda(pool, k_new, v_new, q, page_tables, seq_lens)
+        if q.dtype != torch.bfloat16:
+            raise ValueError("q must be bfloat16")
+        nd = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(k_new.dtype)
+        if nd is None or v_new.dtype != k_new.dtype:
+            raise ValueError("k_new/v_new must both be float32 or bfloat16")
+        n_req, n_q = q.shape[0], q.shape[1]
+        if tuple(k_new.shape) != (n_req, n_q, KV_HEADS, HEAD_DIM) or k_new.shape != v_new.shape:
+            raise ValueError("k_new/v_new must be [n_req, n_q, 4, 256]")
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        if workspace is None:
+            workspace = self.decode_workspace(n_req, n_q, total_seq_len, q.device)
+        _check(tq4_tqb_decode_append_attention(self.handle, bits, pool, pool.numel() // TQB_PAGE_BYTES[bits], k_new,
+                                               v_new, nd, q, page_tables, page_tables.shape[1], seq_lens, n_req,
+                                               n_q, total_seq_len, scale, out, od, workspace, workspace.numel(),
+                                               stream),
+               "tq4_tqb_decode_append_attention")
         return out
 
     def prefill_attention(self, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,

@@ -368,7 +368,12 @@ int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
  *   then K norms [4][256] fp16, then V norms [4][256] fp16.
  * Page tables, lengths, queries, outputs, workspaces (tq4_decode_workspace_bytes)
  * and errors are as for the four-bit calls of the same shape; bits other than 2
- * and 3 return TQ4_ERR_UNSUPPORTED.
+ * and 3 return TQ4_ERR_UNSUPPORTED. tq4_tqb_decode_append_attention is the fused
+ * step of tq4_decode_append_attention for a b-bit pool: the n_q new tokens' K and
+ * V are encoded into the last n_q positions of every request (one query token:
+ * inside the decode kernel; more: a tail-encode kernel ahead of it), then
+ * decoded as tq4_tqb_decode_attention does. k_new, v_new, new_dtype and the
+ * pool's ownership are as for tq4_decode_append_attention.
  * tq4_tqb_codebook copies the fp64 centroids (2^b) and boundaries (2^b - 1). */
 int tq4_tqb_codebook(const tq4_ctx* ctx, int bits, double* centroids, double* boundaries);
 int tq4_tqb_encode_append(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
@@ -381,6 +386,13 @@ int tq4_tqb_decode_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t n
                              int64_t total_seq_len, float scale,
                              void* out, int out_dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
+int tq4_tqb_decode_append_attention(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
+                                    const void* k_new, const void* v_new, int new_dtype,
+                                    const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                    const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                    int64_t total_seq_len, float scale,
+                                    void* out, int out_dtype,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise the stream, return the first device-side error recorded since
  * the last call (TQ4_OK if none) and clear it. */

@@ -87,7 +87,9 @@ def test_tqb_encode_bit_exact(bits, dtype):
 
 
 class TqbCase:
-    def __init__(self, bits, config, seq_lens, n_q, shared_pages=0, outliers=0.05):
+    def __init__(self, bits, config, seq_lens, n_q, shared_pages=0, outliers=0.05, hist=None):
+        """Pools (GPU-encoded and oracle-encoded) whose tables cover seq_lens; the
+        first hist[r] positions of request r are encoded (all of them by default)."""
         self.bits = bits
         self.signs = I.signs(config)
         self.ctx = tq4.Context(self.signs)
@@ -107,7 +109,7 @@ class TqbCase:
         self.seq = np.array(seq_lens, np.int32)
         self.pool = tq4.Context.new_tqb_pool(bits, total)
         self.opool = OB.new_pool(total, bits)
-        for r, s in enumerate(seq_lens):
+        for r, s in enumerate(seq_lens if hist is None else hist):
             first = shared_pages * 256 if r > 0 else 0
             k, v = I.kv_vectors(config, 0, s - first, first_pos=first, request=r, outlier_frac=outliers)
             self.ctx.tqb_encode_append(bits, self.pool, torch.from_numpy(tab[r]).cuda(), first,
@@ -152,6 +154,51 @@ def test_tqb_decode_32k_history(bits):
     got32 = case.decode(qb, torch.from_numpy(case.opool).cuda(), torch.float32)
     assert np.abs(got32 - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max())
     H.assert_bf16_close(case.decode(qb, case.pool, torch.bfloat16), exp, f"{bits}-bit decode 32k")
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("seq_lens,n_q,new_dtype", [
+    ([3000], 1, "f32"),                 # one token, fused into the one-token decode kernel
+    ([257, 1000, 64], 1, "bf16"),       # position 256 opens a page; three requests
+    ([2000, 700], 4, "f32"),            # four tokens: the tail-encode kernel, then the decode
+])
+def test_tqb_fused_append(bits, seq_lens, n_q, new_dtype):
+    """tq4_tqb_decode_append_attention writes the same pool bytes as a separate
+    tq4_tqb_encode_append and then returns the same output as tq4_tqb_decode_attention
+    (the same kernels on the same bytes: bit-identical); against the oracle, which
+    encodes the new tokens itself, within the bf16 tolerance."""
+    hist = [s - n_q for s in seq_lens]
+    case = TqbCase(bits, 45, seq_lens, n_q, hist=hist)
+    dt = torch.float32 if new_dtype == "f32" else torch.bfloat16
+    k_new, v_new = [], []
+    for r, s in enumerate(hist):
+        k, v = I.kv_vectors(45, 1, n_q, first_pos=s, request=r)
+        k_new.append(k)
+        v_new.append(v)
+    kn = np.stack(k_new)
+    vn = np.stack(v_new)
+    kt = torch.from_numpy(kn).cuda().to(dt)
+    vt = torch.from_numpy(vn).cuda().to(dt)
+    qb = I.queries(45, 2, (len(seq_lens), n_q, 24, 256))
+    tab = torch.from_numpy(case.tab).cuda()
+    seq = torch.from_numpy(case.seq).cuda()
+    pool_b = case.pool.clone()
+    fused = case.ctx.tqb_decode_append_attention(bits, case.pool, kt, vt, _bf16_tensor(qb), tab, seq,
+                                                 int(case.seq.sum()), SCALE, out_dtype=torch.float32)
+    for r, s in enumerate(hist):
+        case.ctx.tqb_encode_append(bits, pool_b, tab[r], s, kt[r], vt[r])
+    plain = case.ctx.tqb_decode_attention(bits, pool_b, _bf16_tensor(qb), tab, seq, int(case.seq.sum()), SCALE,
+                                          out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert case.ctx.status() == tq4.TQ4_OK
+    assert torch.equal(case.pool, pool_b)
+    assert torch.equal(fused, plain)
+    for r, s in enumerate(hist):   # the oracle's pool gets the new tokens as the GPU saw them
+        k = kt[r].float().cpu().numpy().astype(np.float64)
+        v = vt[r].float().cpu().numpy().astype(np.float64)
+        OB.encode_append(case.opool, case.tab[r], s, k, v, case.signs, case.c, bits)
+    H.assert_bf16_close(fused.cpu().numpy().astype(np.float64), case.oracle(qb),
+                        f"{bits}-bit fused append {seq_lens} n_q={n_q}")
 
 
 def test_tqb_argument_checks():
