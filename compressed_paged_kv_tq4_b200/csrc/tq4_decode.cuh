@@ -456,10 +456,10 @@ __device__ __forceinline__ void decode_item(const DecodeParams& p, uint8_t* smem
         const uint2 lo = lds64(r + sg * 8);                    // plane 0: words 2 sg, 2 sg + 1
         const uint32_t hb = kBits == 3 ? lds32(r + 64 + sg * 4) : 0u;   // plane 1: word sg
         uint4 o;
-        o.x = widen2(lo.x) | (widen1(hb) << 2);
-        o.y = widen2(lo.x >> 16) | (widen1(hb >> 8) << 2);
-        o.z = widen2(lo.y) | (widen1(hb >> 16) << 2);
-        o.w = widen2(lo.y >> 16) | (widen1(hb >> 24) << 2);
+        o.x = widen2(lo.x) | widen1_bit2<0>(hb);
+        o.y = widen2_hi(lo.x) | widen1_bit2<1>(hb);
+        o.z = widen2(lo.y) | widen1_bit2<2>(hb);
+        o.w = widen2_hi(lo.y) | widen1_bit2<3>(hb);
         *reinterpret_cast<uint4*>(work + (kv * kChunk + pl) * 128 + ((sg ^ seg_swz(pl)) << 4)) = o;
       }
       if (tid < 2 * kChunk * 2 / 16)   // the norms, unchanged

@@ -185,13 +185,13 @@ template <int kBits>
 __device__ __forceinline__ uint4 widen_words32(uint32_t row, int i) {
   uint32_t a, b;
   ld_shared_v2(row + 8 * i, a, b);
-  uint4 r = make_uint4(widen2(a), widen2(a >> 16), widen2(b), widen2(b >> 16));
+  uint4 r = make_uint4(widen2(a), widen2_hi(a), widen2(b), widen2_hi(b));
   if constexpr (kBits == 3) {
     const uint32_t hb = ld_shared_u32(row + 64 + 4 * i);
-    r.x |= widen1(hb) << 2;
-    r.y |= widen1(hb >> 8) << 2;
-    r.z |= widen1(hb >> 16) << 2;
-    r.w |= widen1(hb >> 24) << 2;
+    r.x |= widen1_bit2<0>(hb);
+    r.y |= widen1_bit2<1>(hb);
+    r.z |= widen1_bit2<2>(hb);
+    r.w |= widen1_bit2<3>(hb);
   }
   return r;
 }

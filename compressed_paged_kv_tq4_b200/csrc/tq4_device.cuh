@@ -176,19 +176,30 @@ constexpr int64_t tqb_v_norms() { return tqb_k_norms<kBits>() + int64_t(kHkv) * 
 static_assert(tqb_page_bytes<2>() == TQ4_TQB2_PAGE_BYTES && tqb_page_bytes<3>() == TQ4_TQB3_PAGE_BYTES,
               "page sizes of the header");
 
-// Widen 8 two-bit fields (bits 2i..2i+1 of x) to the low bits of 8 nibbles, and 8
-// single bits (bit i of h) to bit 0 of 8 nibbles.
-__device__ __forceinline__ uint32_t widen2(uint32_t x) {
-  x &= 0xFFFFu;
-  x = (x | (x << 8)) & 0x00FF00FFu;
+// Widen 8 two-bit fields (bits 2i..2i+1 of x) to the low bits of 8 nibbles, and the
+// 8 single bits of byte M of h (bit i) to bit 2 of 8 nibbles. A byte permute places the input
+// bytes; each spreading step then ORs a shifted copy under a mask. Where a shifted
+// copy cannot overlap the original, the step is a multiply (the sum equals the OR).
+__device__ __forceinline__ uint32_t spread_fields2(uint32_t x) {   // bytes 0 and 2 hold 4 fields each
   x = (x | (x << 4)) & 0x0F0F0F0Fu;
   return (x | (x << 2)) & 0x33333333u;
 }
-__device__ __forceinline__ uint32_t widen1(uint32_t h) {
-  h &= 0xFFu;
-  h = (h | (h << 12)) & 0x000F000Fu;
-  h = (h | (h << 6)) & 0x03030303u;
-  return (h | (h << 3)) & 0x11111111u;
+__device__ __forceinline__ uint32_t widen2(uint32_t x) {      // fields of bits 0..15
+  return spread_fields2(__byte_perm(x, 0u, 0x4140u));
+}
+__device__ __forceinline__ uint32_t widen2_hi(uint32_t x) {   // fields of bits 16..31
+  return spread_fields2(__byte_perm(x, 0u, 0x4342u));
+}
+// byte M of h -> its bit pairs 2k, 2k + 1 at bits 8k, 8k + 1
+template <int M>
+__device__ __forceinline__ uint32_t spread_bits_pairs(uint32_t h) {
+  uint32_t t = __byte_perm(h, 0u, 0x4440u | uint32_t(M));
+  t = (t * 0x1001u) & 0x000F000Fu;   // bits 4..7 -> 16..19
+  return (t * 0x41u) & 0x03030303u;  // bits 2..3 -> 8..9 (and 18..19 -> 24..25)
+}
+template <int M>
+__device__ __forceinline__ uint32_t widen1_bit2(uint32_t h) { // byte M of h -> bit 2 of 8 nibbles
+  return (spread_bits_pairs<M>(h) * 0x24u) & 0x44444444u;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
