@@ -112,16 +112,16 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
 # ncu capture of that workload (summarised under profiles/). The figures count only
 # while the kernel sources hash to the value they had when the counters were taken.
-MEASURED_TRAFFIC_SOURCES = "f80e9e2edbc9bc7f32a43c323c31e5185b2c780b8cedd393c7956d824d4cb279"
+MEASURED_TRAFFIC_SOURCES = "49b2151c2cdd75d9666a55d902d580e69d0ececba275d453fcb75d54b7bb8060"
 MEASURED_TRAFFIC = {
-    "decode_32k": 34_188_032,              # decode_q1_kernel: 34,184,448 read + 3,584 written
-    "decode_213k_outliers": 226_268_416,   # decode_q1_kernel: 221,949,952 + 4,318,464
-    "verify_2req_229k": 225_352_704,       # decode_splitk_kernel<3,3>: 221,706,752 + 3,645,952
-    "shared_prefix_8req_33k": 42_972_672,  # decode_splitk_kernel<1,6> (grouped): 42,843,136 + 129,536
-    "int8_decode_32k": 68_470_272,         # decode_splitk_kernel<1,1,INT8>: 67,694,336 + 775,936
-    "prefill_2k_on_32k": 204_016_640,      # prefill_tc_kernel: 101,828,096 + 102,188,544 (segment partials)
-    "tqb3_decode_32k": 25_765_888,         # decode_bits_kernel<1,0,3>: 25,765,632 + 256
-    "tqb2_decode_32k": 17_377_536,         # decode_bits_kernel<1,0,2>: 17,377,536 + 0
+    "decode_32k": 34_226_432,              # decode_q1_kernel<0,4>: 34,184,448 read + 41,984 written
+    "decode_213k_outliers": 225_446_400,   # decode_q1_kernel<0,4>: 221,980,416 read + 3,465,984 written
+    "verify_2req_229k": 225_414_400,       # decode_splitk_kernel<3,3>: 221,705,216 read + 3,709,184 written
+    "shared_prefix_8req_33k": 42_945_024,  # decode_splitk_kernel<1,6> (grouped): 42,843,904 read + 101,120 written
+    "int8_decode_32k": 68_662_016,         # decode_splitk_kernel<1,1,INT8>: 67,694,080 read + 967,936 written
+    "prefill_2k_on_32k": 203_337_984,      # prefill_tc_kernel: 101,502,976 read + 101,835,008 written (segment partials)
+    "tqb3_decode_32k": 25_802_240,         # decode_q1_kernel<0,3>: 25,802,240 read + 0 written
+    "tqb2_decode_32k": 17_409_024,         # decode_q1_kernel<0,2>: 17,409,024 read + 0 written
 }
 
 
