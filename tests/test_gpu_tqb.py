@@ -201,6 +201,30 @@ def test_tqb_fused_append(bits, seq_lens, n_q, new_dtype):
                         f"{bits}-bit fused append {seq_lens} n_q={n_q}")
 
 
+@pytest.mark.parametrize("bits", [2, 3])
+def test_tqb_bad_page_id(bits):
+    """A page id outside the pool is reported (TQ4_ERR_PAGE_RANGE) by the encode, the
+    one-token decode and the fused step, and nothing is written outside the pool's
+    valid pages: page 1, which the table never names, stays zero."""
+    ctx = tq4.Context(I.signs(0))
+    pool = tq4.Context.new_tqb_pool(bits, 2)
+    table = torch.tensor([0, 7], dtype=torch.int32, device="cuda")   # 7 is outside a 2-page pool
+    k = torch.randn(300, 4, 256, device="cuda")
+    ctx.tqb_encode_append(bits, pool, table, 0, k, k)
+    assert ctx.status() == tq4.TQ4_ERR_PAGE_RANGE
+    assert ctx.status() == tq4.TQ4_OK   # cleared by the read
+    page_bytes = tq4.TQB_PAGE_BYTES[bits]
+    assert int(pool[page_bytes:].sum()) == 0
+    q = torch.zeros(1, 1, 24, 256, dtype=torch.bfloat16, device="cuda")
+    seq = torch.tensor([300], dtype=torch.int32, device="cuda")
+    ctx.tqb_decode_attention(bits, pool, q, table[None], seq, 300, SCALE)
+    assert ctx.status() == tq4.TQ4_ERR_PAGE_RANGE
+    kn = torch.randn(1, 1, 4, 256, device="cuda")
+    ctx.tqb_decode_append_attention(bits, pool, kn, kn, q, table[None], seq, 300, SCALE)
+    assert ctx.status() == tq4.TQ4_ERR_PAGE_RANGE
+    assert int(pool[page_bytes:].sum()) == 0
+
+
 def test_tqb_argument_checks():
     ctx = tq4.Context(I.signs(0))
     assert tq4.tq4_tqb_encode_append(ctx.handle, 4, None, 1, None, 1, 0, 1, None, None, 1) == tq4.TQ4_ERR_UNSUPPORTED
