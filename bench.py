@@ -112,16 +112,16 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
 # ncu capture of that workload (summarised under profiles/). The figures count only
 # while the kernel sources hash to the value they had when the counters were taken.
-MEASURED_TRAFFIC_SOURCES = "49b2151c2cdd75d9666a55d902d580e69d0ececba275d453fcb75d54b7bb8060"
+MEASURED_TRAFFIC_SOURCES = "c55ea038a632a82a45a04e315fe82ab50fb31824d9444e21d1b8ebe0efe9e6bc"
 MEASURED_TRAFFIC = {
-    "decode_32k": 34_226_432,              # decode_q1_kernel<0,4>: 34,184,448 read + 41,984 written
-    "decode_213k_outliers": 225_446_400,   # decode_q1_kernel<0,4>: 221,980,416 read + 3,465,984 written
-    "verify_2req_229k": 225_414_400,       # decode_splitk_kernel<3,3>: 221,705,216 read + 3,709,184 written
-    "shared_prefix_8req_33k": 42_945_024,  # decode_splitk_kernel<1,6> (grouped): 42,843,904 read + 101,120 written
-    "int8_decode_32k": 68_662_016,         # decode_splitk_kernel<1,1,INT8>: 67,694,080 read + 967,936 written
-    "prefill_2k_on_32k": 203_337_984,      # prefill_tc_kernel: 101,502,976 read + 101,835,008 written (segment partials)
-    "tqb3_decode_32k": 25_802_240,         # decode_q1_kernel<0,3>: 25,802,240 read + 0 written
-    "tqb2_decode_32k": 17_409_024,         # decode_q1_kernel<0,2>: 17,409,024 read + 0 written
+    "decode_32k": 34_186_240,              # decode_q1_kernel<0,4>: 34,183,680 read + 2,560 written
+    "decode_213k_outliers": 225_153_024,   # decode_q1_kernel<0,4>: 221,978,880 read + 3,174,144 written
+    "verify_2req_229k": 224_915_968,       # decode_splitk_kernel<3,3>: 221,715,968 read + 3,200,000 written
+    "shared_prefix_8req_33k": 43_089_664,  # decode_splitk_kernel<1,6> (grouped): 42,842,880 read + 246,784 written
+    "int8_decode_32k": 68_684_288,         # decode_splitk_kernel<1,1,INT8>: 67,694,336 read + 989,952 written
+    "prefill_2k_on_32k": 203_094_528,      # prefill_tc_kernel: 101,441,792 read + 101,652,736 written (segment partials)
+    "tqb3_decode_32k": 25_805_056,         # decode_q1_kernel<0,3>: 25,803,008 read + 2,048 written
+    "tqb2_decode_32k": 17_409_024,         # decode_q1_kernel<0,2>: 17,408,512 read + 512 written
 }
 
 

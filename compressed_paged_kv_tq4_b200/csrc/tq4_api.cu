@@ -120,8 +120,6 @@ cudaError_t set_decode_bits_attrs() {
   auto set = [&e](auto kernel, size_t bytes) {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
   };
-  set(tq4::decode_bits_kernel<1, false, kBits>, tq4::decode_item_smem_bytes<1, false, kBits>());
-  set(tq4::decode_bits_kernel<1, true, kBits>, tq4::decode_item_smem_bytes<1, false, kBits>());
   set(tq4::decode_bits_kernel<2, false, kBits>, tq4::decode_item_smem_bytes<2, false, kBits>());
   set(tq4::decode_bits_kernel<2, true, kBits>, tq4::decode_item_smem_bytes<2, false, kBits>());
   set(tq4::decode_bits_kernel<3, false, kBits>, tq4::decode_item_smem_bytes<3, false, kBits>());
@@ -135,7 +133,6 @@ cudaError_t launch_bits_nt(dim3 grid, cudaStream_t st, const tq4::DecodeParams& 
     return tq4::launch_pdl(tq4::decode_bits_kernel<NT, true, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
   return tq4::launch_pdl(tq4::decode_bits_kernel<NT, false, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
 }
-// a 2- or 3-bit pool's split-K decode
 // One query token over a b-bit pool: the one-token kernel (tiles by bulk copies,
 // so the tensor map argument is unused).
 template <int kBits>
@@ -148,19 +145,10 @@ cudaError_t launch_q1_bits(bool exact, dim3 grid, cudaStream_t st, const tq4::De
                          tq4::decode_q1_smem_bytes(), st, p, unused);
 }
 
+// a 2- or 3-bit pool's split-K decode (two to four query tokens)
 cudaError_t launch_decode_bits(int bits, int nt, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
-  if (bits == 2) {
-    switch (nt) {
-      case 1: return launch_bits_nt<1, 2>(grid, st, p);
-      case 2: return launch_bits_nt<2, 2>(grid, st, p);
-      default: return launch_bits_nt<3, 2>(grid, st, p);
-    }
-  }
-  switch (nt) {
-    case 1: return launch_bits_nt<1, 3>(grid, st, p);
-    case 2: return launch_bits_nt<2, 3>(grid, st, p);
-    default: return launch_bits_nt<3, 3>(grid, st, p);
-  }
+  if (bits == 2) return nt == 2 ? launch_bits_nt<2, 2>(grid, st, p) : launch_bits_nt<3, 2>(grid, st, p);
+  return nt == 2 ? launch_bits_nt<2, 3>(grid, st, p) : launch_bits_nt<3, 3>(grid, st, p);
 }
 
 // one split-K decode launch with the output precision chosen at run time

@@ -869,8 +869,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   decode_item<NT, kI8, kExact>(p, smem, s_item);
 }
 
-// Split-K decode over a 2- or 3-bit pool: grid (items, 4 KV heads), the requests'
-// own items only (no shared-prefix groups).
+// Split-K decode of two to four query tokens over a 2- or 3-bit pool (one token
+// takes the one-token kernel): grid (items, 4 KV heads), the requests' own items
+// only (no shared-prefix groups).
 template <int NT, bool kExact, int kBits>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_bits_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];

@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       encode_bits_warp<kBits>(x_new, p.signs, w0, w1, nrm);
       store_bits_warp<kBits>(p.pool_w, p.num_pages, table, seq_len - 1, h, kv, w0, w1, nrm, p.status);
     }
-    asm volatile("fence.proxy.async.global;\n" ::: "memory");   // generic stores -> the TMA reads below
+    asm volatile("fence.proxy.async.global;\n" ::: "memory");   // generic stores -> the tile copies below
     __syncwarp();
     if (lane == 0) mbar_arrive_q1(bar_new);
   };
@@ -350,7 +350,8 @@ __global__ void __launch_bounds__(kQ1Threads, 1)
       }
       if (page < 0 || page >= p.num_pages) {
         record_error(p.status, TQ4_ERR_PAGE_RANGE);
-        page = 0;   // still complete the barrier (reading page 0); the tile is masked below
+        page = 0;   // still complete the barrier (reading page 0); the call's output is then
+                    // undefined and the status word reports the page
       }
       const int slot0 = h * kPage + (c & (kPage - 1));
       const uint32_t kdst = buf_addr(b), ndst = base + kQ1NrmOff + b * 128;
