@@ -716,7 +716,7 @@ namespace {
 int prefill_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int32_t* page_table, int32_t table_len,
                  int32_t prefix_len, const uint16_t* q, const uint16_t* k_chunk, const uint16_t* v_chunk,
                  int32_t n_tok, float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes,
-                 void* stream, bool reconstruct) {
+                 void* stream, bool reconstruct, int bits = 4) {
   if (!ctx || n_tok < 0 || prefix_len < 0) return TQ4_ERR_ARG;
   if (n_tok == 0) return TQ4_OK;
   if (!q || !k_chunk || !v_chunk || !out) return TQ4_ERR_ARG;
@@ -727,14 +727,15 @@ int prefill_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int32_
   if ((pool && !aligned(pool, 16)) || !aligned(q, 16) || !aligned(k_chunk, 16) || !aligned(v_chunk, 16) ||
       !aligned(out, 16))
     return TQ4_ERR_ARG;
-  const size_t need = tq4::prefill_workspace_bytes(n_tok) + (reconstruct ? tq4::prefill_prefix_rows_bytes(prefix_len) : 0);
+  const bool rows = reconstruct || bits != 4;   // the prefix rebuilt as dense rows first
+  const size_t need = tq4::prefill_workspace_bytes(n_tok) + (rows ? tq4::prefill_prefix_rows_bytes(prefix_len) : 0);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return TQ4_ERR_WORKSPACE;
   if (int rc = check_device(ctx)) return rc;
   return cuda_status(tq4::launch_prefill_tc(static_cast<const uint8_t*>(pool), num_pages, page_table,
                                             prefix_len, q, k_chunk, v_chunk, n_tok, scale, out, out_dtype,
                                             workspace, ctx->signs, ctx->d_status, ctx->wait_polls,
                                             ctx->withhold, static_cast<cudaStream_t>(stream), ctx->num_sms,
-                                            reconstruct));
+                                            reconstruct, bits));
 }
 
 }  // namespace
@@ -761,6 +762,15 @@ int tq4_prefill_attention_reconstructed(tq4_ctx* ctx, const void* pool, int32_t 
                                         void* stream) {
   return prefill_impl(ctx, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk, v_chunk, n_tok, scale, out,
                       out_dtype, workspace, workspace_bytes, stream, true);
+}
+
+int tq4_tqb_prefill_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t num_pages, const int32_t* page_table,
+                              int32_t table_len, int32_t prefix_len, const uint16_t* q, const uint16_t* k_chunk,
+                              const uint16_t* v_chunk, int32_t n_tok, float scale, void* out, int out_dtype,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+  if (bits != 2 && bits != 3) return ctx ? TQ4_ERR_UNSUPPORTED : TQ4_ERR_ARG;
+  return prefill_impl(ctx, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk, v_chunk, n_tok, scale, out,
+                      out_dtype, workspace, workspace_bytes, stream, true, bits);
 }
 
 int tq4_get_status(tq4_ctx* ctx, void* stream) {

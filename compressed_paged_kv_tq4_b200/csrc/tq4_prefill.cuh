@@ -104,6 +104,55 @@ __global__ void __launch_bounds__(256) prefill_reconstruct_rows_kernel(
   *reinterpret_cast<uint4*>((kv ? vrlo : krlo) + row) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
 }
 
+// The same rebuild for a 2- or 3-bit pool (bit-plane words, the 2^b-level codebook
+// of g_codebook_b): lane l's eight indices are the two-bit fields of plane-0 word
+// l / 2 (its half l & 1) and, with 3 bits, the bits of byte l & 3 of plane-1 word
+// 16 + l / 4 as their bit 2.
+template <int kBits>
+__global__ void __launch_bounds__(256) prefill_reconstruct_rows_bits_kernel(
+    const uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table, int32_t prefix_len,
+    __half* __restrict__ kr, __half* __restrict__ krlo, __half* __restrict__ vr, __half* __restrict__ vrlo,
+    int* status) {
+  __shared__ float cb[1 << kBits];
+  if (threadIdx.x < (1 << kBits)) cb[threadIdx.x] = g_codebook_b[kBits - 2].c[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);   // (pos, h, kv)
+  pdl_wait();   // the pool may be written by the previous kernel
+  pdl_launch_dependents();
+  if (vec >= int64_t(prefix_len) * kHkv * 2) return;
+  const int kv = int(vec & 1), h = int((vec >> 1) % kHkv);
+  const int64_t pos = (vec >> 1) / kHkv;
+  const int32_t page = __ldg(page_table + (pos >> 8));
+  float v[8];
+  if (page >= 0 && page < num_pages) {
+    const uint8_t* pg = pool + int64_t(page) * tqb_page_bytes<kBits>();
+    const int slot = h * kPage + int(pos & (kPage - 1));
+    const uint32_t* words = reinterpret_cast<const uint32_t*>(pg + (kv ? tqb_v_words<kBits>() : 0) +
+                                                              int64_t(slot) * tqb_row_bytes<kBits>());
+    const uint32_t lo = __ldg(words + (lane >> 1)) >> (16 * (lane & 1));
+    uint32_t hb = 0;
+    if constexpr (kBits == 3) hb = __ldg(words + 16 + (lane >> 2)) >> (8 * (lane & 3));
+    const float n = ldg_half(pg + (kv ? tqb_v_norms<kBits>() : tqb_k_norms<kBits>()) + slot * 2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = n * cb[((lo >> (2 * i)) & 3u) | (((hb >> i) & 1u) << 2)];
+  } else {
+    if (lane == 0) record_error(status, TQ4_ERR_PAGE_RANGE);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  }
+  uint32_t hi[4], lo16[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    hi[i] = pack_half2(v[2 * i], v[2 * i + 1]);
+    const float2 hf = __half22float2(*reinterpret_cast<const __half2*>(&hi[i]));
+    lo16[i] = pack_half2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
+  }
+  const int64_t row = (pos * kHkv + h) * kD + lane * 8;
+  *reinterpret_cast<uint4*>((kv ? vr : kr) + row) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  *reinterpret_cast<uint4*>((kv ? vrlo : krlo) + row) = make_uint4(lo16[0], lo16[1], lo16[2], lo16[3]);
+}
+
 // one warp per vector: rotate queries (with scale) and the chunk's K/V; f16 hi + lo
 __global__ void __launch_bounds__(256) prefill_rotate_kernel(
     const uint16_t* __restrict__ q, const uint16_t* __restrict__ kc, const uint16_t* __restrict__ vc,

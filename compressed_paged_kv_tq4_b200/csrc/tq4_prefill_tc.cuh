@@ -861,12 +861,15 @@ inline cudaError_t prefill_tc_set_attrs() {
 }
 
 // rotate prologue (and, with reconstruct, the prefix's dense rows), then the
-// tcgen05 attention kernel (clusters of two CTAs)
+// tcgen05 attention kernel (clusters of two CTAs). bits: 4 (TQ4 pool), or 2 / 3,
+// whose pools are always rebuilt as dense rows first and are read by that rebuild
+// only (the attention kernel gets no packed pool).
 inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,
                                      int32_t prefix_len, const uint16_t* q, const uint16_t* kc,
                                      const uint16_t* vc, int32_t n_tok, float scale, void* out, int out_dtype,
                                      void* workspace, const Signs& signs, int* status, uint32_t spin_limit,
-                                     int test_withhold, cudaStream_t stream, int num_sms, bool reconstruct = false) {
+                                     int test_withhold, cudaStream_t stream, int num_sms, bool reconstruct = false,
+                                     int bits = 4) {
   __half* qr = static_cast<__half*>(workspace);
   __half* qlo = qr + size_t(n_tok) * kHq * kD;
   __half* kr = qlo + size_t(n_tok) * kHq * kD;
@@ -883,7 +886,7 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
   p.n_seg = prefill_segments(n_tok, prefix_len, num_sms);
   p.ws_po = reinterpret_cast<float*>(vrlo + size_t(n_tok) * kHkv * kD);
   p.ws_pml = reinterpret_cast<float2*>(p.ws_po + size_t(pairs) * kPfMaxSegments * kHkv * (2 * kPfRows) * kD);
-  if (reconstruct && prefix_len > 0) {   // rows after the partials: [prefix_len][4][256] each
+  if ((reconstruct || bits != 4) && prefix_len > 0) {   // rows after the partials: [prefix_len][4][256] each
     __half* rows = reinterpret_cast<__half*>(p.ws_pml + size_t(pairs) * kPfMaxSegments * kHkv * (2 * kPfRows));
     const size_t n = size_t(prefix_len) * kHkv * kD;
     p.pkr = rows;
@@ -891,12 +894,20 @@ inline cudaError_t launch_prefill_tc(const uint8_t* pool, int32_t num_pages, con
     p.pvr = rows + 2 * n;
     p.pvrlo = rows + 3 * n;
     const int64_t rvecs = int64_t(prefix_len) * kHkv * 2;
-    e = launch_pdl(prefill_reconstruct_rows_kernel, dim3(unsigned((rvecs + 7) / 8)), dim3(256), 0, stream, pool,
-                   num_pages, page_table, prefix_len, rows, rows + n, rows + 2 * n, rows + 3 * n, status);
+    const dim3 rgrid(unsigned((rvecs + 7) / 8));
+    if (bits == 2)
+      e = launch_pdl(prefill_reconstruct_rows_bits_kernel<2>, rgrid, dim3(256), 0, stream, pool, num_pages,
+                     page_table, prefix_len, rows, rows + n, rows + 2 * n, rows + 3 * n, status);
+    else if (bits == 3)
+      e = launch_pdl(prefill_reconstruct_rows_bits_kernel<3>, rgrid, dim3(256), 0, stream, pool, num_pages,
+                     page_table, prefix_len, rows, rows + n, rows + 2 * n, rows + 3 * n, status);
+    else
+      e = launch_pdl(prefill_reconstruct_rows_kernel, rgrid, dim3(256), 0, stream, pool, num_pages, page_table,
+                     prefix_len, rows, rows + n, rows + 2 * n, rows + 3 * n, status);
     if (e != cudaSuccess) return e;
   }
-  p.pool = pool;
-  p.num_pages = num_pages;
+  p.pool = bits == 4 ? pool : nullptr;   // a b-bit pool has been read by the rebuild above
+  p.num_pages = bits == 4 ? num_pages : 0;
   p.page_table = page_table;
   p.prefix_len = prefix_len;
   p.n_tok = n_tok;

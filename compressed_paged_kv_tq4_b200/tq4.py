@@ -51,7 +51,7 @@ EXPORTS = (
     "tq4_decode_shared_workspace_bytes", "tq4_decode_attention_shared",
     "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
     "tq4_ctx_set_decode_path", "tq4_tqb_codebook", "tq4_tqb_encode_append", "tq4_tqb_decode_attention",
-    "tq4_tqb_decode_append_attention",
+    "tq4_tqb_decode_append_attention", "tq4_tqb_prefill_attention",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -95,6 +95,8 @@ _sig = {
                               ctypes.c_int),
     "tq4_tqb_decode_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p,
                                   ctypes.c_int, _p, _sz, _p], ctypes.c_int),
+    "tq4_tqb_prefill_attention": ([_p, ctypes.c_int, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p,
+                                   ctypes.c_int, _p, _sz, _p], ctypes.c_int),
     "tq4_tqb_decode_append_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32,
                                          _i32, _i64, _f, _p, ctypes.c_int, _p, _sz, _p], ctypes.c_int),
     "tq4_int8_encode_append": ([_p, _p, _i32, _p, _i32, _i32, _i32, _p, _p, ctypes.c_int, _p], ctypes.c_int),
@@ -304,6 +306,13 @@ def tq4_tqb_decode_append_attention(ctx, bits, pool, num_pages, k_new, v_new, ne
                                                 new_dtype, _ptr(q), _ptr(page_tables), max_pages, _ptr(seq_lens),
                                                 n_req, n_q, total_seq_len, scale, _ptr(out), out_dtype,
                                                 _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_tqb_prefill_attention(ctx, bits, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk, v_chunk,
+                              n_tok, scale, out, out_dtype, workspace, workspace_bytes, stream=None) -> int:
+    return _lib.tq4_tqb_prefill_attention(ctx, bits, _ptr(pool), num_pages, _ptr(page_table), table_len, prefix_len,
+                                          _ptr(q), _ptr(k_chunk), _ptr(v_chunk), n_tok, scale, _ptr(out), out_dtype,
+                                          _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def tq4_ctx_set_wait_limit(ctx, polls, withhold_signal=0) -> int:
@@ -675,4 +684,22 @@ class Context:
         fn = tq4_prefill_attention_reconstructed if reconstruct else tq4_prefill_attention
         _check(fn(self.handle, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk, v_chunk, n_tok, scale, out,
                   od, workspace, workspace.numel(), stream), fn.__name__)
+        return out
+
+    def tqb_prefill_attention(self, bits, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,
+                              out_dtype=torch.bfloat16, workspace=None, stream=None):
+        """prefill_attention over a 2- or 3-bit pool (the prefix rebuilt as dense rows first)."""
+        _need_cuda(q, k_chunk, v_chunk)
+        n_tok = q.shape[0]
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        if workspace is None:
+            nbytes = tq4_prefill_reconstructed_workspace_bytes(prefix_len, n_tok)
+            workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+        num_pages = pool.numel() // TQB_PAGE_BYTES[bits] if pool is not None else 0
+        tlen = page_table.numel() if page_table is not None else 0
+        _check(tq4_tqb_prefill_attention(self.handle, bits, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk,
+                                         v_chunk, n_tok, scale, out, od, workspace, workspace.numel(), stream),
+               "tq4_tqb_prefill_attention")
         return out

@@ -374,6 +374,10 @@ int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
  * inside the decode kernel; more: a tail-encode kernel ahead of it), then
  * decoded as tq4_tqb_decode_attention does. k_new, v_new, new_dtype and the
  * pool's ownership are as for tq4_decode_append_attention.
+ * tq4_tqb_prefill_attention is tq4_prefill_attention_reconstructed over a b-bit
+ * pool: the prefix is rebuilt as dense rows n * c[idx] (the 2^b-level codebook)
+ * in the workspace, then the same causal attention of the chunk runs over them;
+ * workspace size tq4_prefill_reconstructed_workspace_bytes(prefix_len, n_tok).
  * tq4_tqb_codebook copies the fp64 centroids (2^b) and boundaries (2^b - 1). */
 int tq4_tqb_codebook(const tq4_ctx* ctx, int bits, double* centroids, double* boundaries);
 int tq4_tqb_encode_append(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
@@ -386,6 +390,12 @@ int tq4_tqb_decode_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t n
                              int64_t total_seq_len, float scale,
                              void* out, int out_dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
+int tq4_tqb_prefill_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t num_pages,
+                              const int32_t* page_table, int32_t table_len,
+                              int32_t prefix_len, const uint16_t* q,
+                              const uint16_t* k_chunk, const uint16_t* v_chunk,
+                              int32_t n_tok, float scale, void* out, int out_dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
 int tq4_tqb_decode_append_attention(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
                                     const void* k_new, const void* v_new, int new_dtype,
                                     const uint16_t* q, const int32_t* page_tables, int32_t max_pages,

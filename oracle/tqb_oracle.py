@@ -184,3 +184,23 @@ def decode_attention(pool, page_tables, seq_lens, q, scale, signs, centroids, bi
                 g = h // GROUP
                 out[r, t, h] = T4.sdpa_row(q[r, t, h], K[:visible, g], V[:visible, g], scale)
     return out
+
+
+def prefill_attention(pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, signs, centroids, bits: int,
+                      rows=None):
+    """Causal attention of a query chunk against the b-bit prefix plus the chunk itself
+    (the four-bit oracle's rule: token i sees prefix positions [0, prefix_len) and chunk
+    tokens 0..i; the chunk's K/V at full precision). ``rows`` selects chunk tokens."""
+    q = np.asarray(q, dtype=np.float64)
+    n_tok = q.shape[0]
+    rows = np.arange(n_tok) if rows is None else np.asarray(rows)
+    Kp, Vp = reconstruct(pool, page_table, 0, prefix_len, signs, centroids, bits)
+    K = np.concatenate([Kp, np.asarray(k_chunk, dtype=np.float64)], axis=0)
+    V = np.concatenate([Vp, np.asarray(v_chunk, dtype=np.float64)], axis=0)
+    out = np.zeros((len(rows), H_Q, D), np.float64)
+    for j, i in enumerate(rows):
+        visible = prefix_len + int(i) + 1
+        for h in range(H_Q):
+            g = h // GROUP
+            out[j, h] = T4.sdpa_row(q[i, h], K[:visible, g], V[:visible, g], scale)
+    return out

@@ -202,6 +202,72 @@ def test_tqb_fused_append(bits, seq_lens, n_q, new_dtype):
 
 
 @pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("prefix_len,n_tok,outliers", [
+    (0, 40, 0.0), (300, 100, 0.05), (1000, 257, 0.0), (4096, 64, 0.05),
+])
+def test_tqb_prefill_parity(bits, prefix_len, n_tok, outliers):
+    """The prefill over a b-bit prefix (rebuilt as dense rows, then the tcgen05
+    attention) against the b-bit oracle: every row, bf16 on the GPU-encoded pool and
+    1e-4 in fp32 on the oracle's own pool bytes."""
+    c, _ = OB.codebook(bits)
+    signs = I.signs(5)
+    ctx = tq4.Context(signs)
+    npg = max(1, (prefix_len + 255) // 256)
+    table = I.page_table_scattered(5, npg, npg + 2)
+    tt = torch.from_numpy(table).cuda()
+    pool = tq4.Context.new_tqb_pool(bits, npg + 2)
+    opool = OB.new_pool(npg + 2, bits)
+    if prefix_len:
+        k, v = I.kv_vectors(5, 0, prefix_len, outlier_frac=outliers)
+        ctx.tqb_encode_append(bits, pool, tt, 0, torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+        OB.encode_append(opool, table, 0, k, v, signs, c, bits)
+    qb = I.queries(5, 0, (n_tok, 24, 256))
+    kb, vb = I.chunk_kv(5, 0, n_tok)
+    args = (_bf16_tensor(qb), _bf16_tensor(kb), _bf16_tensor(vb), SCALE)
+    out = ctx.tqb_prefill_attention(bits, pool, tt, prefix_len, *args)
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    exp = OB.prefill_attention(opool, table, prefix_len, I.bf16_bits_to_f32(qb), I.bf16_bits_to_f32(kb),
+                               I.bf16_bits_to_f32(vb), SCALE, signs, c, bits)
+    H.assert_bf16_close(out.float().cpu().numpy(), exp, f"{bits}-bit prefill {prefix_len}+{n_tok}")
+    out32 = ctx.tqb_prefill_attention(bits, torch.from_numpy(opool).cuda(), tt, prefix_len, *args,
+                                      out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    err = np.abs(out32.cpu().numpy().astype(np.float64) - exp).max()
+    assert err <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max()), (bits, prefix_len, n_tok, err)
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+def test_tqb_prefill_2k_on_32k_sampled(bits):
+    """The prefill workload's shape (2,048 chunk tokens on a 32,768-position prefix) over a
+    b-bit pool, checked on sampled chunk tokens (first and last included)."""
+    c, _ = OB.codebook(bits)
+    signs = I.signs(6)
+    ctx = tq4.Context(signs)
+    prefix_len, n_tok = 32768, 2048
+    npg = prefix_len // 256
+    table = I.page_table_scattered(6, npg, npg + 8)
+    tt = torch.from_numpy(table).cuda()
+    k, v = I.kv_vectors(6, 0, prefix_len)
+    pool = tq4.Context.new_tqb_pool(bits, npg + 8)
+    opool = OB.new_pool(npg + 8, bits)
+    ctx.tqb_encode_append(bits, pool, tt, 0, torch.from_numpy(k).cuda(), torch.from_numpy(v).cuda())
+    OB.encode_append(opool, table, 0, k, v, signs, c, bits)
+    qb = I.queries(6, 0, (n_tok, 24, 256))
+    kb, vb = I.chunk_kv(6, 0, n_tok)
+    rows = np.array([0, 1, 255, 256, 1023, 1500, 2046, 2047])
+    out = ctx.tqb_prefill_attention(bits, torch.from_numpy(opool).cuda(), tt, prefix_len, _bf16_tensor(qb),
+                                    _bf16_tensor(kb), _bf16_tensor(vb), SCALE, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    exp = OB.prefill_attention(opool, table, prefix_len, I.bf16_bits_to_f32(qb), I.bf16_bits_to_f32(kb),
+                               I.bf16_bits_to_f32(vb), SCALE, signs, c, bits, rows=rows)
+    got = out.cpu().numpy().astype(np.float64)[rows]
+    assert np.abs(got - exp).max() <= H.F32_ABS_TOL * max(1.0, np.abs(exp).max())
+
+
+@pytest.mark.parametrize("bits", [2, 3])
 def test_tqb_bad_page_id(bits):
     """A page id outside the pool is reported (TQ4_ERR_PAGE_RANGE) by the encode, the
     one-token decode and the fused step, and nothing is written outside the pool's

@@ -129,3 +129,45 @@ def test_attention_closed_forms(bits):
         assert np.allclose(out[0, 0, h], V[0, h // 6], rtol=0, atol=1e-12)
         # token 1 sees positions 0 and 1, whose keys are equal: the mean of their values
         assert np.allclose(out[0, 1, h], 0.5 * (V[0, h // 6] + V[1, h // 6]), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("bits", OB.BITS)
+def test_prefill_without_prefix_is_bit_width_independent(bits):
+    """With no prefix the chunk attends to itself at full precision, so the b-bit
+    prefill must equal the four-bit oracle's prefill of the same chunk."""
+    c, _ = OB.codebook(bits)
+    c4, _ = O4.codebook()
+    signs = I.signs(3)
+    rng = np.random.default_rng(11)
+    n_tok = 5
+    q = rng.standard_normal((n_tok, 24, 256))
+    kc = rng.standard_normal((n_tok, 4, 256))
+    vc = rng.standard_normal((n_tok, 4, 256))
+    got = OB.prefill_attention(OB.new_pool(1, bits), np.zeros(1, np.int32), 0, q, kc, vc, 1 / 16, signs, c, bits)
+    exp = O4.prefill_attention(O4.new_pool(1), np.zeros(1, np.int32), 0, q, kc, vc, 1 / 16, signs, c4)
+    assert np.array_equal(got, exp)
+
+
+@pytest.mark.parametrize("bits", OB.BITS)
+def test_prefill_zero_query_is_the_mean_of_visible_values(bits):
+    """q = 0 makes every visible score equal: token i's output is the plain mean of the
+    rebuilt prefix values and the chunk values of tokens 0..i (a wrong window, a
+    missing prefix or a wrong page fails it)."""
+    c, _ = OB.codebook(bits)
+    signs = I.signs(4)
+    rng = np.random.default_rng(12)
+    table = np.array([2, 0, 1], np.int32)
+    pool = OB.new_pool(3, bits)
+    prefix = 600
+    k = rng.standard_normal((prefix, 4, 256))
+    v = rng.standard_normal((prefix, 4, 256)) * rng.uniform(0.5, 2.0, (prefix, 1, 1))
+    OB.encode_append(pool, table, 0, k, v, signs, c, bits)
+    _, Vp = OB.reconstruct(pool, table, 0, prefix, signs, c, bits)
+    n_tok = 4
+    kc = rng.standard_normal((n_tok, 4, 256))
+    vc = rng.standard_normal((n_tok, 4, 256))
+    out = OB.prefill_attention(pool, table, prefix, np.zeros((n_tok, 24, 256)), kc, vc, 1 / 16, signs, c, bits)
+    for i in range(n_tok):
+        mean = (Vp.sum(axis=0) + vc[:i + 1].sum(axis=0)) / (prefix + i + 1)   # [4, 256]
+        for h in range(24):
+            assert np.allclose(out[i, h], mean[h // 6], rtol=0, atol=1e-12)
