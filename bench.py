@@ -112,16 +112,16 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
 # ncu capture of that workload (summarised under profiles/). The figures count only
 # while the kernel sources hash to the value they had when the counters were taken.
-MEASURED_TRAFFIC_SOURCES = "c55ea038a632a82a45a04e315fe82ab50fb31824d9444e21d1b8ebe0efe9e6bc"
+MEASURED_TRAFFIC_SOURCES = "77f1d4daf355955e90fd304e7088022c3f9387a60aa30b1838bd864660b05603"
 MEASURED_TRAFFIC = {
-    "decode_32k": 34_186_240,              # decode_q1_kernel<0,4>: 34,183,680 read + 2,560 written
-    "decode_213k_outliers": 225_153_024,   # decode_q1_kernel<0,4>: 221,978,880 read + 3,174,144 written
-    "verify_2req_229k": 224_915_968,       # decode_splitk_kernel<3,3>: 221,715,968 read + 3,200,000 written
-    "shared_prefix_8req_33k": 43_089_664,  # decode_splitk_kernel<1,6> (grouped): 42,842,880 read + 246,784 written
-    "int8_decode_32k": 68_684_288,         # decode_splitk_kernel<1,1,INT8>: 67,694,336 read + 989,952 written
-    "prefill_2k_on_32k": 203_094_528,      # prefill_tc_kernel: 101,441,792 read + 101,652,736 written (segment partials)
-    "tqb3_decode_32k": 25_805_056,         # decode_q1_kernel<0,3>: 25,803,008 read + 2,048 written
-    "tqb2_decode_32k": 17_409_024,         # decode_q1_kernel<0,2>: 17,408,512 read + 512 written
+    "decode_32k": 34_185_984,              # decode_q1_kernel<0,4>: 34,183,936 read + 2,048 written
+    "decode_213k_outliers": 225_362_688,   # decode_q1_kernel<0,4>: 221,952,768 read + 3,409,920 written
+    "verify_2req_229k": 225_369_856,       # decode_splitk_kernel<3,3>: 221,754,624 read + 3,615,232 written
+    "shared_prefix_8req_33k": 43_039_744,  # decode_splitk_kernel<1,6> (grouped): 42,842,880 read + 196,864 written
+    "int8_decode_32k": 68_565_248,         # decode_splitk_kernel<1,1,INT8>: 67,694,592 read + 870,656 written
+    "prefill_2k_on_32k": 203_565_568,      # prefill_tc_kernel: 101,913,344 read + 101,652,224 written (segment partials)
+    "tqb3_decode_32k": 25_802_496,         # decode_q1_kernel<0,3>: 25,802,496 read + 0 written
+    "tqb2_decode_32k": 17_408_512,         # decode_q1_kernel<0,2>: 17,408,512 read + 0 written
 }
 
 

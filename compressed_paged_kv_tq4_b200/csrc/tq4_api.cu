@@ -477,6 +477,20 @@ int tq4_reconstruct(tq4_ctx* ctx, const void* pool, int32_t num_pages, const int
                                              static_cast<cudaStream_t>(stream)));
 }
 
+int tq4_tqb_reconstruct(tq4_ctx* ctx, int bits, const void* pool, int32_t num_pages, const int32_t* page_table,
+                        int32_t table_len, int32_t start, int32_t n, float* k_out, float* v_out, void* stream) {
+  if (bits != 2 && bits != 3) return ctx ? TQ4_ERR_UNSUPPORTED : TQ4_ERR_ARG;
+  if (!ctx || n < 0 || start < 0) return TQ4_ERR_ARG;
+  if (n == 0) return TQ4_OK;
+  if (!pool || !page_table || !k_out || !v_out || num_pages <= 0 || table_len <= 0) return TQ4_ERR_ARG;
+  if ((int64_t(start) + n + tq4::kPage - 1) / tq4::kPage > table_len) return TQ4_ERR_ARG;
+  if (!aligned(pool, 16) || !aligned(k_out, 16) || !aligned(v_out, 16)) return TQ4_ERR_ARG;
+  if (int rc = check_device(ctx)) return rc;
+  return cuda_status(tq4::launch_reconstruct(static_cast<const uint8_t*>(pool), num_pages, page_table, start, n,
+                                             k_out, v_out, ctx->signs, ctx->d_status,
+                                             static_cast<cudaStream_t>(stream), bits));
+}
+
 size_t tq4_decode_workspace_bytes(const tq4_ctx* ctx, int32_t n_req, int32_t n_q, int64_t total_seq_len) {
   if (!ctx || n_req <= 0 || n_q < 1 || n_q > TQ4_MAX_QUERY_TOKENS || total_seq_len <= 0) return 0;
   return plan_decode(ctx, n_req, n_q, total_seq_len).total;

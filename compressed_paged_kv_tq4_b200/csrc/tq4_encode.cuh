@@ -108,13 +108,20 @@ __global__ void __launch_bounds__(256) encode_append_kernel(
   store_packed_warp(pool, num_pages, page_table, start_pos + tok, head, kv, word, n, status);
 }
 
-// grid: ceil(n * 8 / warps_per_block); writes fp32 [n][4][256] for K and V
+// grid: ceil(n * 8 / warps_per_block); writes fp32 [n][4][256] for K and V.
+// kBits: 4 (TQ4 pool), or 2 / 3 (bit-plane pool: lane l's indices are the two-bit
+// fields of plane-0 word l / 2, half l & 1, and with 3 bits byte l & 3 of plane-1
+// word 16 + l / 4 as their bit 2; the 2^b-level codebook).
+template <int kBits>
 __global__ void __launch_bounds__(256) reconstruct_kernel(
     const uint8_t* __restrict__ pool, int32_t num_pages, const int32_t* __restrict__ page_table,
     int32_t start, int32_t n, float* __restrict__ k_out, float* __restrict__ v_out, Signs signs,
     int* status) {
-  __shared__ float cb[16];
-  if (threadIdx.x < 16) cb[threadIdx.x] = g_codebook.c[threadIdx.x];
+  __shared__ float cb[1 << kBits];
+  if (threadIdx.x < (1 << kBits)) {
+    if constexpr (kBits == 4) cb[threadIdx.x] = g_codebook.c[threadIdx.x];
+    else cb[threadIdx.x] = g_codebook_b[kBits - 2].c[threadIdx.x];
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t vec = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -135,12 +142,22 @@ __global__ void __launch_bounds__(256) reconstruct_kernel(
     return;
   }
   const int slot = p & (kPage - 1);
-  const uint8_t* base = pool + int64_t(page) * kPageBytes;
-  const uint32_t word = ldg32(base + (kv ? kVWords : kKWords) + ((head * kPage + slot) * kWords + lane) * 4);
-  const float nrm = ldg_half(base + (kv ? kVNorms : kKNorms) + (head * kPage + slot) * 2);
-  float v[8];
+  float v[8], nrm;
+  if constexpr (kBits == 4) {
+    const uint8_t* base = pool + int64_t(page) * kPageBytes;
+    const uint32_t word = ldg32(base + (kv ? kVWords : kKWords) + ((head * kPage + slot) * kWords + lane) * 4);
+    nrm = ldg_half(base + (kv ? kVNorms : kKNorms) + (head * kPage + slot) * 2);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = cb[(word >> (4 * i)) & 15u];
+    for (int i = 0; i < 8; ++i) v[i] = cb[(word >> (4 * i)) & 15u];
+  } else {
+    const uint8_t* base = pool + int64_t(page) * tqb_page_bytes<kBits>();
+    const uint8_t* row = base + (kv ? tqb_v_words<kBits>() : 0) + int64_t(head * kPage + slot) * tqb_row_bytes<kBits>();
+    const uint32_t lo = ldg32(row + (lane >> 1) * 4) >> (16 * (lane & 1));
+    const uint32_t hb = kBits == 3 ? ldg32(row + (16 + (lane >> 2)) * 4) >> (8 * (lane & 3)) : 0u;
+    nrm = ldg_half(base + (kv ? tqb_v_norms<kBits>() : tqb_k_norms<kBits>()) + (head * kPage + slot) * 2);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = cb[((lo >> (2 * i)) & 3u) | (((hb >> i) & 1u) << 2)];
+  }
   warp_fwht256(v);
   float o[8];
 #pragma unroll
@@ -393,14 +410,16 @@ inline cudaError_t launch_encode_tail(uint8_t* pool, int32_t num_pages, const in
   }
 }
 
+// bits: 4 (TQ4 pool), 2 or 3
 cudaError_t launch_reconstruct(const uint8_t* pool, int32_t num_pages, const int32_t* page_table,
                                int32_t start, int32_t n, float* k_out, float* v_out,
-                               const Signs& signs, int* status, cudaStream_t stream) {
+                               const Signs& signs, int* status, cudaStream_t stream, int bits = 4) {
   const int threads = 256, wpb = threads / 32;
   const int64_t vecs = int64_t(n) * 2 * kHkv;
   const unsigned blocks = unsigned((vecs + wpb - 1) / wpb);
-  return launch_pdl(reconstruct_kernel, dim3(blocks), dim3(threads), 0, stream, pool, num_pages, page_table, start,
-                    n, k_out, v_out, signs, status);
+  auto kernel = bits == 2 ? reconstruct_kernel<2> : bits == 3 ? reconstruct_kernel<3> : reconstruct_kernel<4>;
+  return launch_pdl(kernel, dim3(blocks), dim3(threads), 0, stream, pool, num_pages, page_table, start, n, k_out,
+                    v_out, signs, status);
 }
 
 }  // namespace tq4

@@ -51,7 +51,7 @@ EXPORTS = (
     "tq4_decode_shared_workspace_bytes", "tq4_decode_attention_shared",
     "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
     "tq4_ctx_set_decode_path", "tq4_tqb_codebook", "tq4_tqb_encode_append", "tq4_tqb_decode_attention",
-    "tq4_tqb_decode_append_attention", "tq4_tqb_prefill_attention",
+    "tq4_tqb_decode_append_attention", "tq4_tqb_prefill_attention", "tq4_tqb_reconstruct",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -95,6 +95,7 @@ _sig = {
                               ctypes.c_int),
     "tq4_tqb_decode_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p,
                                   ctypes.c_int, _p, _sz, _p], ctypes.c_int),
+    "tq4_tqb_reconstruct": ([_p, ctypes.c_int, _p, _i32, _p, _i32, _i32, _i32, _p, _p, _p], ctypes.c_int),
     "tq4_tqb_prefill_attention": ([_p, ctypes.c_int, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p,
                                    ctypes.c_int, _p, _sz, _p], ctypes.c_int),
     "tq4_tqb_decode_append_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32,
@@ -306,6 +307,11 @@ def tq4_tqb_decode_append_attention(ctx, bits, pool, num_pages, k_new, v_new, ne
                                                 new_dtype, _ptr(q), _ptr(page_tables), max_pages, _ptr(seq_lens),
                                                 n_req, n_q, total_seq_len, scale, _ptr(out), out_dtype,
                                                 _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_tqb_reconstruct(ctx, bits, pool, num_pages, page_table, table_len, start, n, k_out, v_out, stream=None) -> int:
+    return _lib.tq4_tqb_reconstruct(ctx, bits, _ptr(pool), num_pages, _ptr(page_table), table_len, start, n,
+                                    _ptr(k_out), _ptr(v_out), _stream(stream))
 
 
 def tq4_tqb_prefill_attention(ctx, bits, pool, num_pages, page_table, table_len, prefix_len, q, k_chunk, v_chunk,
@@ -685,6 +691,14 @@ class Context:
         _check(fn(self.handle, pool, num_pages, page_table, tlen, prefix_len, q, k_chunk, v_chunk, n_tok, scale, out,
                   od, workspace, workspace.numel(), stream), fn.__name__)
         return out
+
+    def tqb_reconstruct(self, bits, pool, page_table, start, n, stream=None):
+        _need_cuda(pool, page_table)
+        k = torch.empty((n, KV_HEADS, HEAD_DIM), dtype=torch.float32, device=pool.device)
+        v = torch.empty_like(k)
+        _check(tq4_tqb_reconstruct(self.handle, bits, pool, pool.numel() // TQB_PAGE_BYTES[bits], page_table,
+                                   page_table.numel(), start, n, k, v, stream), "tq4_tqb_reconstruct")
+        return k, v
 
     def tqb_prefill_attention(self, bits, pool, page_table, prefix_len, q, k_chunk, v_chunk, scale, out=None,
                               out_dtype=torch.bfloat16, workspace=None, stream=None):

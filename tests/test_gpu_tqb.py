@@ -202,6 +202,26 @@ def test_tqb_fused_append(bits, seq_lens, n_q, new_dtype):
 
 
 @pytest.mark.parametrize("bits", [2, 3])
+def test_tqb_reconstruct_matches_oracle(bits):
+    """Explicit K/V from the oracle's own b-bit pool bytes against the oracle's
+    reconstruction (per vector, relative), over scattered pages and a ragged range."""
+    c, _ = OB.codebook(bits)
+    signs = I.signs(1)
+    ctx = tq4.Context(signs)
+    table = np.array([3, 0, 2], np.int32)
+    k, v = I.kv_vectors(1, 1, 700, outlier_frac=0.05)
+    opool = OB.new_pool(4, bits)
+    OB.encode_append(opool, table, 0, k, v, signs, c, bits)
+    kr, vr = ctx.tqb_reconstruct(bits, torch.from_numpy(opool).cuda(), torch.from_numpy(table).cuda(), 5, 690)
+    torch.cuda.synchronize()
+    assert ctx.status() == tq4.TQ4_OK
+    ko, vo = OB.reconstruct(opool, table, 5, 690, signs, c, bits)
+    for got, exp in ((kr.cpu().numpy(), ko), (vr.cpu().numpy(), vo)):
+        rel = np.linalg.norm(got - exp, axis=-1) / np.maximum(np.linalg.norm(exp, axis=-1), 1e-30)
+        assert rel.max() < 1e-6, rel.max()
+
+
+@pytest.mark.parametrize("bits", [2, 3])
 @pytest.mark.parametrize("prefix_len,n_tok,outliers", [
     (0, 40, 0.0), (300, 100, 0.05), (1000, 257, 0.0), (4096, 64, 0.05),
 ])
