@@ -114,24 +114,36 @@ cudaError_t launch_decode_tc(int nt, dim3 grid, cudaStream_t st, const tq4::Deco
                : tq4::launch_pdl(tq4::decode_tc_kernel<3, false>, grid, block, smem, st, p);
 }
 
+// shared memory of a b-bit split-K launch: the wider of its two item bodies
+template <int NT, int NTG, int kBits>
+constexpr size_t bits_smem_bytes() {
+  return std::max(tq4::decode_item_smem_bytes<NT, false, kBits>(), tq4::decode_item_smem_bytes<NTG, false, kBits>());
+}
 template <int kBits>
 cudaError_t set_decode_bits_attrs() {
   cudaError_t e = cudaSuccess;
   auto set = [&e](auto kernel, size_t bytes) {
     if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes));
   };
-  set(tq4::decode_bits_kernel<2, false, kBits>, tq4::decode_item_smem_bytes<2, false, kBits>());
-  set(tq4::decode_bits_kernel<2, true, kBits>, tq4::decode_item_smem_bytes<2, false, kBits>());
-  set(tq4::decode_bits_kernel<3, false, kBits>, tq4::decode_item_smem_bytes<3, false, kBits>());
-  set(tq4::decode_bits_kernel<3, true, kBits>, tq4::decode_item_smem_bytes<3, false, kBits>());
+  constexpr int G = tq4::kShareNT;
+  set(tq4::decode_bits_kernel<2, 2, false, kBits>, bits_smem_bytes<2, 2, kBits>());
+  set(tq4::decode_bits_kernel<2, 2, true, kBits>, bits_smem_bytes<2, 2, kBits>());
+  set(tq4::decode_bits_kernel<3, 3, false, kBits>, bits_smem_bytes<3, 3, kBits>());
+  set(tq4::decode_bits_kernel<3, 3, true, kBits>, bits_smem_bytes<3, 3, kBits>());
+  set(tq4::decode_bits_kernel<1, G, false, kBits>, bits_smem_bytes<1, G, kBits>());
+  set(tq4::decode_bits_kernel<1, G, true, kBits>, bits_smem_bytes<1, G, kBits>());
+  set(tq4::decode_bits_kernel<2, G, false, kBits>, bits_smem_bytes<2, G, kBits>());
+  set(tq4::decode_bits_kernel<2, G, true, kBits>, bits_smem_bytes<2, G, kBits>());
+  set(tq4::decode_bits_kernel<3, G, false, kBits>, bits_smem_bytes<3, G, kBits>());
+  set(tq4::decode_bits_kernel<3, G, true, kBits>, bits_smem_bytes<3, G, kBits>());
   return e;
 }
-template <int NT, int kBits>
+template <int NT, int NTG, int kBits>
 cudaError_t launch_bits_nt(dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
-  const size_t smem = tq4::decode_item_smem_bytes<NT, false, kBits>();
+  const size_t smem = bits_smem_bytes<NT, NTG, kBits>();
   if (p.out_dtype == TQ4_DTYPE_F32)
-    return tq4::launch_pdl(tq4::decode_bits_kernel<NT, true, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
-  return tq4::launch_pdl(tq4::decode_bits_kernel<NT, false, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
+    return tq4::launch_pdl(tq4::decode_bits_kernel<NT, NTG, true, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
+  return tq4::launch_pdl(tq4::decode_bits_kernel<NT, NTG, false, kBits>, grid, dim3(tq4::kDecThreads), smem, st, p);
 }
 // One query token over a b-bit pool: the one-token kernel (tiles by bulk copies,
 // so the tensor map argument is unused).
@@ -145,10 +157,23 @@ cudaError_t launch_q1_bits(bool exact, dim3 grid, cudaStream_t st, const tq4::De
                          tq4::decode_q1_smem_bytes(), st, p, unused);
 }
 
-// a 2- or 3-bit pool's split-K decode (two to four query tokens)
-cudaError_t launch_decode_bits(int bits, int nt, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
-  if (bits == 2) return nt == 2 ? launch_bits_nt<2, 2>(grid, st, p) : launch_bits_nt<3, 2>(grid, st, p);
-  return nt == 2 ? launch_bits_nt<2, 3>(grid, st, p) : launch_bits_nt<3, 3>(grid, st, p);
+// a 2- or 3-bit pool's split-K decode: two to four query tokens, or any count with
+// shared-prefix group items (kShareNT n-tiles)
+template <int kBits>
+cudaError_t launch_decode_bits_b(int nt, bool groups, dim3 grid, cudaStream_t st, const tq4::DecodeParams& p) {
+  constexpr int G = tq4::kShareNT;
+  if (groups) {
+    switch (nt) {
+      case 1: return launch_bits_nt<1, G, kBits>(grid, st, p);
+      case 2: return launch_bits_nt<2, G, kBits>(grid, st, p);
+      default: return launch_bits_nt<3, G, kBits>(grid, st, p);
+    }
+  }
+  return nt == 2 ? launch_bits_nt<2, 2, kBits>(grid, st, p) : launch_bits_nt<3, 3, kBits>(grid, st, p);
+}
+cudaError_t launch_decode_bits(int bits, int nt, bool groups, dim3 grid, cudaStream_t st,
+                               const tq4::DecodeParams& p) {
+  return bits == 2 ? launch_decode_bits_b<2>(nt, groups, grid, st, p) : launch_decode_bits_b<3>(nt, groups, grid, st, p);
 }
 
 // one split-K decode launch with the output precision chosen at run time
@@ -582,10 +607,10 @@ int decode_impl(tq4_ctx* ctx, const void* pool, int32_t num_pages, const uint16_
   const dim3 grid(unsigned(pl.items_ub), tq4::kHkv);
   if (bits != 4) {
     const bool exact = out_dtype == TQ4_DTYPE_F32;
-    if (tq4::decode_nt(n_q) == 1)
+    if (tq4::decode_nt(n_q) == 1 && !groups)
       e = bits == 2 ? launch_q1_bits<2>(exact, grid, st, p) : launch_q1_bits<3>(exact, grid, st, p);
     else
-      e = launch_decode_bits(bits, tq4::decode_nt(n_q), grid, st, p);
+      e = launch_decode_bits(bits, tq4::decode_nt(n_q), groups, grid, st, p);
   } else if (int8) {
     e = launch_splitk_nt<true>(tq4::decode_nt(n_q), false, grid, st, p);
   } else if (groups) {     // group items and the requests' own items in one launch
@@ -646,6 +671,20 @@ int tq4_decode_attention_shared(tq4_ctx* ctx, void* pool, int32_t num_pages, con
   return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
                      out, out_dtype, workspace, workspace_bytes, stream, k_new ? &app : nullptr, false, prefix_leader,
                      prefix_pages);
+}
+
+int tq4_tqb_decode_attention_shared(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages, const void* k_new,
+                                    const void* v_new, int new_dtype, const uint16_t* q, const int32_t* page_tables,
+                                    int32_t max_pages, const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                    int64_t total_seq_len, const int32_t* prefix_leader, const int32_t* prefix_pages,
+                                    float scale, void* out, int out_dtype, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (bits != 2 && bits != 3) return ctx ? TQ4_ERR_UNSUPPORTED : TQ4_ERR_ARG;
+  if (!prefix_leader || !prefix_pages || (k_new == nullptr) != (v_new == nullptr)) return TQ4_ERR_ARG;
+  const AppendArgs app{pool, k_new, v_new, new_dtype};
+  return decode_impl(ctx, pool, num_pages, q, page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len, scale,
+                     out, out_dtype, workspace, workspace_bytes, stream, k_new ? &app : nullptr, false, prefix_leader,
+                     prefix_pages, bits);
 }
 
 int tq4_int8_encode_append(tq4_ctx* ctx, void* pool, int32_t num_pages, const int32_t* page_table,

@@ -135,6 +135,7 @@ constexpr size_t decode_smem_bytes() {
 }
 static_assert(decode_item_smem_bytes<kShareNT, false>() <= 227u * 1024u, "group items fit shared memory");
 static_assert(decode_item_smem_bytes<3, false, 3>() <= 227u * 1024u, "3-bit items fit shared memory");
+static_assert(decode_item_smem_bytes<kShareNT, false, 3>() <= 227u * 1024u, "3-bit group items fit shared memory");
 
 __device__ __forceinline__ int warp_incl_scan(int v) {
   const int lane = threadIdx.x & 31;
@@ -820,6 +821,31 @@ __device__ __forceinline__ void check_item_records(const DecodeParams& p, int* s
   }
 }
 
+// Warp-collective: group item x (x < share.n_gitems): group gi, split sp of its
+// shared positions, one record per member.
+__device__ __forceinline__ void describe_group_item(const DecodeParams& p, int x, int* s_item) {
+  const int lane = threadIdx.x & 31;
+  int gi = 0;
+  while (gi + 1 < p.share.n_groups && x >= p.share.item0[gi + 1]) ++gi;
+  const int sp = x - p.share.item0[gi];
+  const int nm = p.share.n_mem[gi];
+  const int gl = p.share.split_len;
+  for (int k = 0; k < nm; ++k) {
+    const int rq = p.share.mem[gi][k];
+    const int first = request_first_record(p, rq);
+    if (lane == 0) {
+      s_item[kItReq + k] = rq;
+      s_item[kItRec + k] = first + sp;
+    }
+  }
+  if (lane == 0) {
+    s_item[kItPosB] = sp * gl;
+    s_item[kItPosE] = min((sp + 1) * gl, p.share.pos[gi]);
+    s_item[kItTable] = p.share.mem[gi][0];
+    s_item[kItNMem] = nm;
+  }
+}
+
 // Split-K decode: grid (items, 4 KV heads). Items [0, share.n_gitems) are group
 // items (NTG n-tiles), the rest the requests' own items (NT n-tiles).
 template <int NT, int NTG, bool kI8, bool kExact>
@@ -833,29 +859,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   const int x = int(blockIdx.x);
   const bool group = x < p.share.n_gitems;
   if (w == 0) {
-    if (group) {   // group gi, split s of its shared positions; one record per member
-      int gi = 0;
-      while (gi + 1 < p.share.n_groups && x >= p.share.item0[gi + 1]) ++gi;
-      const int sp = x - p.share.item0[gi];
-      const int nm = p.share.n_mem[gi];
-      const int gl = p.share.split_len;
-      for (int k = 0; k < nm; ++k) {
-        const int rq = p.share.mem[gi][k];
-        const int first = request_first_record(p, rq);
-        if (lane == 0) {
-          s_item[kItReq + k] = rq;
-          s_item[kItRec + k] = first + sp;
-        }
-      }
-      if (lane == 0) {
-        s_item[kItPosB] = sp * gl;
-        s_item[kItPosE] = min((sp + 1) * gl, p.share.pos[gi]);
-        s_item[kItTable] = p.share.mem[gi][0];
-        s_item[kItNMem] = nm;
-      }
-    } else {       // request req, split sp of its own positions
-      describe_private_item(p, x, h, s_item);
-    }
+    if (group) describe_group_item(p, x, s_item);
+    else describe_private_item(p, x, h, s_item);   // request req, split sp of its own positions
   }
   if (w == 0 && lane == 0) check_item_records(p, s_item);
   __syncthreads();
@@ -869,10 +874,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_splitk_kernel(const Dec
   decode_item<NT, kI8, kExact>(p, smem, s_item);
 }
 
-// Split-K decode of two to four query tokens over a 2- or 3-bit pool (one token
-// takes the one-token kernel): grid (items, 4 KV heads), the requests' own items
-// only (no shared-prefix groups).
-template <int NT, bool kExact, int kBits>
+// Split-K decode over a 2- or 3-bit pool: grid (items, 4 KV heads). Without
+// shared-prefix groups it serves two to four query tokens (one token takes the
+// one-token kernel); with groups, items [0, share.n_gitems) are group items (NTG
+// n-tiles) and the rest the requests' own items (NT n-tiles), as in the four-bit
+// split-K kernel.
+template <int NT, int NTG, bool kExact, int kBits>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_bits_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_item[kItWords];
@@ -881,10 +888,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_bits_kernel(const Decod
   const int x = int(blockIdx.x);
   pdl_wait();
   pdl_launch_dependents();
-  if (w == 0) describe_private_item(p, x, h, s_item);
+  const bool group = x < p.share.n_gitems;
+  if (w == 0) {
+    if (group) describe_group_item(p, x, s_item);
+    else describe_private_item(p, x, h, s_item);
+  }
   if (threadIdx.x == 0) check_item_records(p, s_item);
   __syncthreads();
   if (s_item[kItNMem] == 0 || x >= p.items_ub) return;
+  if constexpr (NTG != NT) {
+    if (group) {
+      decode_item<NTG, false, kExact, kBits>(p, smem, s_item);
+      return;
+    }
+  }
   decode_item<NT, false, kExact, kBits>(p, smem, s_item);
 }
 

@@ -52,6 +52,7 @@ EXPORTS = (
     "tq4_prefill_reconstructed_workspace_bytes", "tq4_prefill_attention_reconstructed",
     "tq4_ctx_set_decode_path", "tq4_tqb_codebook", "tq4_tqb_encode_append", "tq4_tqb_decode_attention",
     "tq4_tqb_decode_append_attention", "tq4_tqb_prefill_attention", "tq4_tqb_reconstruct",
+    "tq4_tqb_decode_attention_shared",
     # host page pool (include/tq4_pages.h)
     "tq4_pages_create", "tq4_pages_destroy", "tq4_pages_reservation", "tq4_pages_admit", "tq4_pages_grow",
     "tq4_pages_finish", "tq4_pages_step_boundary", "tq4_pages_table", "tq4_pages_free_count",
@@ -95,6 +96,8 @@ _sig = {
                               ctypes.c_int),
     "tq4_tqb_decode_attention": ([_p, ctypes.c_int, _p, _i32, _p, _p, _i32, _p, _i32, _i32, _i64, _f, _p,
                                   ctypes.c_int, _p, _sz, _p], ctypes.c_int),
+    "tq4_tqb_decode_attention_shared": ([_p, ctypes.c_int, _p, _i32, _p, _p, ctypes.c_int, _p, _p, _i32, _p, _i32,
+                                         _i32, _i64, _p, _p, _f, _p, ctypes.c_int, _p, _sz, _p], ctypes.c_int),
     "tq4_tqb_reconstruct": ([_p, ctypes.c_int, _p, _i32, _p, _i32, _i32, _i32, _p, _p, _p], ctypes.c_int),
     "tq4_tqb_prefill_attention": ([_p, ctypes.c_int, _p, _i32, _p, _i32, _i32, _p, _p, _p, _i32, _f, _p,
                                    ctypes.c_int, _p, _sz, _p], ctypes.c_int),
@@ -307,6 +310,17 @@ def tq4_tqb_decode_append_attention(ctx, bits, pool, num_pages, k_new, v_new, ne
                                                 new_dtype, _ptr(q), _ptr(page_tables), max_pages, _ptr(seq_lens),
                                                 n_req, n_q, total_seq_len, scale, _ptr(out), out_dtype,
                                                 _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def tq4_tqb_decode_attention_shared(ctx, bits, pool, num_pages, k_new, v_new, new_dtype, q, page_tables, max_pages,
+                                    seq_lens, n_req, n_q, total_seq_len, prefix_leader, prefix_pages, scale, out,
+                                    out_dtype, workspace, workspace_bytes, stream=None) -> int:
+    ld, pg = _host_i32(prefix_leader), _host_i32(prefix_pages)
+    return _lib.tq4_tqb_decode_attention_shared(ctx, bits, _ptr(pool), num_pages, _ptr(k_new), _ptr(v_new),
+                                                new_dtype, _ptr(q), _ptr(page_tables), max_pages, _ptr(seq_lens),
+                                                n_req, n_q, total_seq_len, ld.ctypes.data, pg.ctypes.data, scale,
+                                                _ptr(out), out_dtype, _ptr(workspace), workspace_bytes,
+                                                _stream(stream))
 
 
 def tq4_tqb_reconstruct(ctx, bits, pool, num_pages, page_table, table_len, start, n, k_out, v_out, stream=None) -> int:
@@ -580,6 +594,37 @@ class Context:
                                            page_tables, max_pages, seq_lens, n_req, n_q, total_seq_len,
                                            prefix_leader, prefix_pages, scale, out, od, workspace,
                                            workspace.numel(), stream), "tq4_decode_attention_shared")
+        return out
+
+    def tqb_decode_attention_shared(self, bits, pool, q, page_tables, seq_lens, total_seq_len, scale, prefix_leader,
+                                    prefix_pages, k_new=None, v_new=None, out=None, out_dtype=torch.bfloat16,
+                                    workspace=None, stream=None):
+        """decode_attention_shared over a 2- or 3-bit pool."""
+        _need_cuda(pool, q, page_tables, seq_lens)
+        if q.dtype != torch.bfloat16:
+            raise ValueError("q must be bfloat16")
+        n_req, n_q = q.shape[0], q.shape[1]
+        nd = DTYPE_F32
+        if k_new is not None:
+            _need_cuda(k_new, v_new)
+            nd = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(k_new.dtype)
+            if nd is None or v_new.dtype != k_new.dtype or tuple(k_new.shape) != (n_req, n_q, KV_HEADS, HEAD_DIM):
+                raise ValueError("k_new/v_new must be float32 or bfloat16 [n_req, n_q, 4, 256]")
+        if out is None:
+            out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+        od = DTYPE_F32 if out.dtype == torch.float32 else DTYPE_BF16
+        max_pages = page_tables.shape[1]
+        if workspace is None:
+            nbytes = tq4_decode_shared_workspace_bytes(self.handle, n_req, n_q, total_seq_len, max_pages,
+                                                       prefix_leader, prefix_pages)
+            if nbytes == 0:
+                raise TQ4Error(TQ4_ERR_ARG, "tq4_decode_shared_workspace_bytes")
+            workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+        _check(tq4_tqb_decode_attention_shared(self.handle, bits, pool, pool.numel() // TQB_PAGE_BYTES[bits], k_new,
+                                               v_new, nd, q, page_tables, max_pages, seq_lens, n_req, n_q,
+                                               total_seq_len, prefix_leader, prefix_pages, scale, out, od,
+                                               workspace, workspace.numel(), stream),
+               "tq4_tqb_decode_attention_shared")
         return out
 
     # -- the uniform INT8 comparison arm

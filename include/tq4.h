@@ -379,6 +379,8 @@ int tq4_int8_decode_attention(tq4_ctx* ctx, const void* pool, int32_t num_pages,
  * in the workspace, then the same causal attention of the chunk runs over them;
  * workspace size tq4_prefill_reconstructed_workspace_bytes(prefix_len, n_tok).
  * tq4_tqb_reconstruct is tq4_reconstruct for a b-bit pool (explicit fp32 K/V).
+ * tq4_tqb_decode_attention_shared is tq4_decode_attention_shared for a b-bit pool
+ * (the same group description, workspace and append arguments).
  * tq4_tqb_codebook copies the fp64 centroids (2^b) and boundaries (2^b - 1). */
 int tq4_tqb_codebook(const tq4_ctx* ctx, int bits, double* centroids, double* boundaries);
 int tq4_tqb_encode_append(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
@@ -391,6 +393,14 @@ int tq4_tqb_decode_attention(tq4_ctx* ctx, int bits, const void* pool, int32_t n
                              int64_t total_seq_len, float scale,
                              void* out, int out_dtype,
                              void* workspace, size_t workspace_bytes, void* stream);
+int tq4_tqb_decode_attention_shared(tq4_ctx* ctx, int bits, void* pool, int32_t num_pages,
+                                    const void* k_new, const void* v_new, int new_dtype,
+                                    const uint16_t* q, const int32_t* page_tables, int32_t max_pages,
+                                    const int32_t* seq_lens, int32_t n_req, int32_t n_q,
+                                    int64_t total_seq_len, const int32_t* prefix_leader,
+                                    const int32_t* prefix_pages, float scale,
+                                    void* out, int out_dtype,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 int tq4_tqb_reconstruct(tq4_ctx* ctx, int bits, const void* pool, int32_t num_pages,
                         const int32_t* page_table, int32_t table_len,
                         int32_t start, int32_t n, float* k_out, float* v_out, void* stream);

@@ -100,6 +100,8 @@ def test_argument_errors_return_before_any_launch():
     assert lib.tq4_tqb_decode_attention(None, 3, None, 0, None, None, 0, None, 1, 1, 1, 0.0625, None, 1, None, 0,
                                         None) == E
     assert lib.tq4_tqb_reconstruct(None, 3, None, 0, None, 0, 0, 1, None, None, None) == E
+    assert lib.tq4_tqb_decode_attention_shared(None, 2, None, 0, None, None, 1, None, None, 0, None, 1, 1, 1, None,
+                                               None, 0.0625, None, 1, None, 0, None) == E
     assert lib.tq4_tqb_prefill_attention(None, 2, None, 0, None, 0, 0, None, None, None, 1, 0.0625, None, 1, None, 0,
                                          None) == E
     assert lib.tq4_tqb_decode_append_attention(None, 2, None, 0, None, None, 1, None, None, 0, None, 1, 1, 1, 0.0625,
