@@ -112,15 +112,15 @@ def workload_config(name, world):
 # DRAM bytes (read + write) per launch of each workload's dominant kernel, from one
 # ncu capture of that workload (summarised under profiles/). The figures count only
 # while the kernel sources hash to the value they had when the counters were taken.
-MEASURED_TRAFFIC_SOURCES = "77f1d4daf355955e90fd304e7088022c3f9387a60aa30b1838bd864660b05603"
+MEASURED_TRAFFIC_SOURCES = "7628c67e128fb178515366d470678ff947cab69f7aea0ee838a90e1407f5a6d7"
 MEASURED_TRAFFIC = {
-    "decode_32k": 34_185_984,              # decode_q1_kernel<0,4>: 34,183,936 read + 2,048 written
-    "decode_213k_outliers": 225_362_688,   # decode_q1_kernel<0,4>: 221,952,768 read + 3,409,920 written
-    "verify_2req_229k": 225_369_856,       # decode_splitk_kernel<3,3>: 221,754,624 read + 3,615,232 written
-    "shared_prefix_8req_33k": 43_039_744,  # decode_splitk_kernel<1,6> (grouped): 42,842,880 read + 196,864 written
-    "int8_decode_32k": 68_565_248,         # decode_splitk_kernel<1,1,INT8>: 67,694,592 read + 870,656 written
-    "prefill_2k_on_32k": 203_565_568,      # prefill_tc_kernel: 101,913,344 read + 101,652,224 written (segment partials)
-    "tqb3_decode_32k": 25_802_496,         # decode_q1_kernel<0,3>: 25,802,496 read + 0 written
+    "decode_32k": 34_219_008,              # decode_q1_kernel<0,4>: 34,183,936 read + 35,072 written
+    "decode_213k_outliers": 225_226_496,   # decode_q1_kernel<0,4>: 221,925,888 read + 3,300,608 written
+    "verify_2req_229k": 224_868_096,       # decode_splitk_kernel<3,3>: 221,704,960 read + 3,163,136 written
+    "shared_prefix_8req_33k": 43_067_392,  # decode_splitk_kernel<1,6> (grouped): 42,843,136 read + 224,256 written
+    "int8_decode_32k": 68_552_448,         # decode_splitk_kernel<1,1,INT8>: 67,694,080 read + 858,368 written
+    "prefill_2k_on_32k": 203_590_912,      # prefill_tc_kernel: 102,009,600 read + 101,581,312 written (segment partials)
+    "tqb3_decode_32k": 25_804_288,         # decode_q1_kernel<0,3>: 25,802,240 read + 2,048 written
     "tqb2_decode_32k": 17_408_512,         # decode_q1_kernel<0,2>: 17,408,512 read + 0 written
 }
 
